@@ -1,0 +1,147 @@
+"""fp64 CPU oracle for causal grouped-query attention (forward).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product path
+(the CUDA library and its Python binding) never imports, links or calls it,
+and it shares no code with that path.
+
+The arithmetic lives in ``attn_ref.c`` (plain C, fp64, one query row at a
+time); this module compiles it with gcc and marshals numpy arrays through
+ctypes.  What it computes is the scaled-dot-product attention that the Tessera
+pages name ("a FlashAttention forward kernel with online softmax, causal
+masking, grouped-query attention" -- hysenlabs.com Tessera review, "The kernel
+set and its torch fallback"), written out as its definition:
+
+    s_ij = scale * <Q[b,h,i], K[b,h//G,j]>,  j <= i when causal
+    O[b,h,i] = sum_j softmax_j(s_i) V[b,h//G,j]
+    LSE[b,h,i] = logsumexp_j(s_ij)            (natural log)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "attn_ref.c")
+LIB = os.path.join(_HERE, "liboracle_attn.so")
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(src_path: str = SRC, out_path: str = LIB) -> str:
+    """Compile the C oracle into a shared library (gcc, -O2, strict IEEE fp64).
+
+    -ffp-contract=off keeps every multiply and add separately rounded, as the
+    source is written; no -ffast-math.
+    """
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+           "-o", out_path, src_path, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
+def _stale(lib_path: str, src_path: str) -> bool:
+    return (not os.path.exists(lib_path)
+            or os.path.getmtime(lib_path) < os.path.getmtime(src_path))
+
+
+def load(lib_path: str | None = None) -> ctypes.CDLL:
+    """Load the oracle library, building it first when missing or stale.
+
+    With ``lib_path`` given, load that file as is (used to test planted
+    mistakes in a modified copy of the source).
+    """
+    global _lib
+    if lib_path is not None:
+        return _bind(ctypes.CDLL(lib_path))
+    with _lock:
+        if _lib is None:
+            if _stale(LIB, SRC):
+                build()
+            _lib = _bind(ctypes.CDLL(LIB))
+    return _lib
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    dp = ctypes.POINTER(ctypes.c_double)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    ci = ctypes.c_int
+    lib.oracle_attn_fwd_f64.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci,
+                                        ci, ctypes.c_double]
+    lib.oracle_attn_fwd_f64.restype = ci
+    lib.oracle_attn_rows_bf16.argtypes = [u16p, u16p, u16p, ci, ci, ci, ci, ci,
+                                          ci, ctypes.c_double, i64p,
+                                          ctypes.c_int64, dp, dp]
+    lib.oracle_attn_rows_bf16.restype = ci
+    return lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def attn_fwd_f64(q, k, v, causal: bool = True, scale: float | None = None,
+                 lib: ctypes.CDLL | None = None):
+    """Full attention in fp64.
+
+    q: [B,Hq,T,d], k and v: [B,Hkv,T,d] (anything numpy can view as float64).
+    Returns (O [B,Hq,T,d] float64, LSE [B,Hq,T] float64).  ``scale`` defaults
+    to 1/sqrt(d).
+    """
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B,Hkv,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, Hq, T, d), dtype=np.float64)
+    lse = np.zeros((B, Hq, T), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_fwd_f64(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                                 _ptr(v, ctypes.c_double), _ptr(o, ctypes.c_double),
+                                 _ptr(lse, ctypes.c_double), B, Hq, Hkv, T, d,
+                                 int(bool(causal)), float(scale))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_f64 failed with code {rc}")
+    return o, lse
+
+
+def attn_rows_bf16(q_bits, k_bits, v_bits, rows, causal: bool = True,
+                   scale: float | None = None, lib: ctypes.CDLL | None = None):
+    """Selected output rows, reading bf16 inputs given as uint16 bit patterns.
+
+    q_bits: uint16 [B,Hq,T,d]; k_bits, v_bits: uint16 [B,Hkv,T,d];
+    rows: int64 [n,3] of (b, h, i).  Rows sorted by (b, h // G) reuse the
+    widened key/value head.  Returns (O rows [n,d], LSE rows [n]) in fp64.
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    B, Hq, T, d = q_bits.shape
+    Hkv = k_bits.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    n = rows.shape[0]
+    o = np.zeros((n, d), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_rows_bf16(_ptr(q_bits, ctypes.c_uint16),
+                                   _ptr(k_bits, ctypes.c_uint16),
+                                   _ptr(v_bits, ctypes.c_uint16), B, Hq, Hkv, T,
+                                   d, int(bool(causal)), float(scale),
+                                   _ptr(rows, ctypes.c_int64), n,
+                                   _ptr(o, ctypes.c_double),
+                                   _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_rows_bf16 failed with code {rc}")
+    return o, lse

@@ -1,0 +1,173 @@
+/*
+ * Plain fp64 CPU oracle for causal grouped-query attention (forward).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
+ * this file: only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark use it.  It shares no code, header or constant with the CUDA path.
+ *
+ * What it computes (the textbook scaled-dot-product attention that the Tessera
+ * pages name as "a FlashAttention forward kernel with online softmax, causal
+ * masking, grouped-query attention" -- hysenlabs.com Tessera review, section
+ * "The kernel set and its torch fallback"; Tessera README, "What's in it" /
+ * "Kernels"; the decoder it serves has "grouped-query attention", README
+ * "What's in it" / "Training side"):
+ *
+ *   G = Hq / Hkv, query head h reads key/value head g = floor(h / G)
+ *   J(i) = {0..i} when causal, {0..T-1} otherwise
+ *   s_ij   = scale * sum_c Q[b,h,i,c] * K[b,g,j,c]          j in J(i)
+ *   m_i    = max_j s_ij
+ *   l_i    = sum_j exp(s_ij - m_i)
+ *   O[b,h,i,:] = sum_j exp(s_ij - m_i) * V[b,g,j,:] / l_i
+ *   LSE[b,h,i] = m_i + ln(l_i)                    (natural log, scaled logits)
+ *
+ * The FlashAttention tiling and online softmax reach exactly this result up to
+ * rounding, so the oracle is the definition written out, one row at a time,
+ * with no blocking, fusion or reordering.  Layouts are contiguous row-major:
+ * Q, O [B,Hq,T,d]; K, V [B,Hkv,T,d]; LSE [B,Hq,T].
+ *
+ * Return codes: 0 ok, 1 invalid argument, 2 out of memory.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 -> fp64: a bf16 is the top 16 bits of an IEEE fp32, so widening is exact. */
+static double bf16_bits_to_f64(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * One query row against the first n_keys rows of one key/value head.
+ * q: [d]; kh, vh: [*, d] (row j at offset j*d); s: scratch of n_keys doubles.
+ * Writes o[0..d) and *lse.
+ */
+static void attend_one_row(const double *q, const double *kh, const double *vh,
+                           int64_t n_keys, int d, double scale, double *s,
+                           double *o, double *lse)
+{
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+            dot += q[c] * kh[j * d + c];
+        s[j] = scale * dot;
+        if (s[j] > m)
+            m = s[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        s[j] = exp(s[j] - m); /* unnormalised probability */
+        l += s[j];
+    }
+    for (int c = 0; c < d; ++c)
+        o[c] = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j)
+        for (int c = 0; c < d; ++c)
+            o[c] += s[j] * vh[j * d + c];
+    for (int c = 0; c < d; ++c)
+        o[c] /= l;
+    *lse = m + log(l);
+}
+
+static int check_shape(int B, int Hq, int Hkv, int T, int d)
+{
+    if (B < 0 || Hq < 1 || Hkv < 1 || T < 0 || d < 1)
+        return 1;
+    if (Hq % Hkv != 0)
+        return 1;
+    return 0;
+}
+
+/*
+ * Full attention on fp64 inputs.  lse may be NULL.
+ */
+int oracle_attn_fwd_f64(const double *q, const double *k, const double *v,
+                        double *o, double *lse, int B, int Hq, int Hkv, int T,
+                        int d, int causal, double scale)
+{
+    if (check_shape(B, Hq, Hkv, T, d))
+        return 1;
+    if (B == 0 || T == 0)
+        return 0;
+    const int G = Hq / Hkv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    if (!s)
+        return 2;
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            const double *kh = k + ((int64_t)b * Hkv + g) * T * d;
+            const double *vh = v + ((int64_t)b * Hkv + g) * T * d;
+            for (int i = 0; i < T; ++i) {
+                const int64_t row = ((int64_t)b * Hq + h) * T + i;
+                const int64_t n_keys = causal ? (int64_t)i + 1 : (int64_t)T;
+                double lse_i;
+                attend_one_row(q + row * d, kh, vh, n_keys, d, scale, s,
+                               o + row * d, &lse_i);
+                if (lse)
+                    lse[row] = lse_i;
+            }
+        }
+    }
+    free(s);
+    return 0;
+}
+
+/*
+ * Selected rows of attention on bf16 inputs (raw bf16 bit patterns), widened
+ * exactly to fp64 on read.  rows: n_rows triples (b, h, i).  Outputs:
+ * o_rows [n_rows, d] and lse_rows [n_rows] in fp64.  Used to check outputs of
+ * workloads too large to run through the oracle in full.
+ */
+int oracle_attn_rows_bf16(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int B, int Hq, int Hkv, int T,
+                          int d, int causal, double scale,
+                          const int64_t *rows, int64_t n_rows, double *o_rows,
+                          double *lse_rows)
+{
+    if (check_shape(B, Hq, Hkv, T, d))
+        return 1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= T)
+            return 1;
+    }
+    if (n_rows == 0)
+        return 0;
+    const int G = Hq / Hkv;
+    double *kh = (double *)malloc(sizeof(double) * (size_t)T * d);
+    double *vh = (double *)malloc(sizeof(double) * (size_t)T * d);
+    double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    if (!kh || !vh || !qi || !s) {
+        free(kh); free(vh); free(qi); free(s);
+        return 2;
+    }
+    int64_t cur_b = -1, cur_g = -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        const int64_t g = h / G;
+        if (b != cur_b || g != cur_g) { /* widen this key/value head once */
+            const int64_t base = (b * Hkv + g) * (int64_t)T * d;
+            for (int64_t e = 0; e < (int64_t)T * d; ++e) {
+                kh[e] = bf16_bits_to_f64(k[base + e]);
+                vh[e] = bf16_bits_to_f64(v[base + e]);
+            }
+            cur_b = b;
+            cur_g = g;
+        }
+        const int64_t qrow = (b * Hq + h) * (int64_t)T + i;
+        for (int c = 0; c < d; ++c)
+            qi[c] = bf16_bits_to_f64(q[qrow * d + c]);
+        const int64_t n_keys = causal ? i + 1 : (int64_t)T;
+        attend_one_row(qi, kh, vh, n_keys, d, scale, s, o_rows + r * d,
+                       &lse_rows[r]);
+    }
+    free(kh); free(vh); free(qi); free(s);
+    return 0;
+}

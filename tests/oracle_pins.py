@@ -1,0 +1,220 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function takes a loaded oracle library (the real one, or one
+built from a copy of the source with a planted mistake) and raises
+AssertionError when the oracle disagrees with what the mathematics fixes:
+
+* hand-derived closed forms (tests/golden/closed_forms.yaml);
+* a library routine: torch's CPU scaled_dot_product_attention in float64,
+  with K/V heads repeated for grouped-query attention, and torch.logsumexp
+  for the LSE;
+* exact arithmetic: Python Decimal at 60 significant digits on tiny inputs
+  whose logits are far beyond exp's fp64 range;
+* invariants: causal row 0, identical V rows, uniform weights for zero
+  queries (prefix means, LSE = ln(i+1)), GQA == MHA with repeated K/V,
+  invariance to a common shift of every key, joint key/value permutation,
+  scale homogeneity, convexity of O.
+"""
+from __future__ import annotations
+
+import math
+import os
+from decimal import Decimal, getcontext
+
+import numpy as np
+import torch
+import yaml
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                      "closed_forms.yaml")
+
+_MATH_NAMES = {"sqrt": math.sqrt, "log": math.log, "exp": math.exp}
+
+
+def _eval(expr: str) -> float:
+    return float(eval(expr, {"__builtins__": {}}, _MATH_NAMES))
+
+
+def _rand(shape, seed, sigma=1.0):
+    return np.random.default_rng(seed).normal(0.0, sigma, size=shape)
+
+
+def pin_closed_forms(lib):
+    with open(GOLDEN) as f:
+        cases = yaml.safe_load(f)
+    for name, c in cases.items():
+        B, Hq, Hkv, T, d = c["B"], c["Hq"], c["Hkv"], c["T"], c["d"]
+        q = np.array([_eval(x) for x in c["q"]]).reshape(B, Hq, T, d)
+        k = np.array([_eval(x) for x in c["k"]]).reshape(B, Hkv, T, d)
+        v = np.array([_eval(x) for x in c["v"]]).reshape(B, Hkv, T, d)
+        scale = _eval(c["scale"])
+        for mode, causal in (("causal", True), ("full", False)):
+            o, lse = oracle.attn_fwd_f64(q, k, v, causal=causal, scale=scale, lib=lib)
+            want_o = np.array([_eval(x) for x in c[mode]["o"]]).reshape(o.shape)
+            want_lse = np.array([_eval(x) for x in c[mode]["lse"]]).reshape(lse.shape)
+            assert np.allclose(o, want_o, rtol=0, atol=1e-14), (name, mode, o, want_o)
+            assert np.allclose(lse, want_lse, rtol=0, atol=1e-14), (name, mode, lse, want_lse)
+
+
+def _torch_reference(q, k, v, causal, scale):
+    """torch CPU float64 SDPA with K/V heads repeated (repeat_interleave)."""
+    G = q.shape[1] // k.shape[1]
+    qt = torch.from_numpy(q)
+    kt = torch.from_numpy(k).repeat_interleave(G, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(G, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal,
+                                                         scale=scale)
+    s = scale * (qt @ kt.transpose(-1, -2))
+    if causal:
+        T = q.shape[2]
+        s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return o.numpy(), lse.numpy()
+
+
+def pin_library_sdpa(lib):
+    shapes = [  # (B, Hq, Hkv, T, d, causal, sigma)
+        (1, 1, 1, 1, 4, True, 1.0),
+        (2, 4, 2, 17, 8, True, 1.0),
+        (1, 6, 3, 33, 16, False, 1.0),
+        (2, 8, 2, 40, 64, True, 4.0),
+        (1, 4, 1, 65, 32, True, 2.0),
+        (1, 3, 3, 9, 5, False, 3.0),
+    ]
+    for n, (B, Hq, Hkv, T, d, causal, sigma) in enumerate(shapes):
+        q = _rand((B, Hq, T, d), 10 + n, sigma)
+        k = _rand((B, Hkv, T, d), 20 + n, sigma)
+        v = _rand((B, Hkv, T, d), 30 + n)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.attn_fwd_f64(q, k, v, causal=causal, scale=scale, lib=lib)
+        ro, rlse = _torch_reference(q, k, v, causal, scale)
+        assert np.max(np.abs(o - ro)) <= 1e-12, ("O", n, np.max(np.abs(o - ro)))
+        assert np.max(np.abs(lse - rlse)) <= 1e-12, ("LSE", n, np.max(np.abs(lse - rlse)))
+
+
+def _decimal_attention(q, k, v, causal, scale):
+    """Exact-ish attention in Decimal arithmetic (60 digits), one row at a time."""
+    getcontext().prec = 60
+    B, Hq, T, d = q.shape
+    G = Hq // k.shape[1]
+    o = np.zeros(q.shape)
+    lse = np.zeros(q.shape[:3])
+    sc = Decimal(scale)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for i in range(T):
+                keys = range(i + 1) if causal else range(T)
+                s = [sc * sum(Decimal(float(q[b, h, i, c])) * Decimal(float(k[b, g, j, c]))
+                              for c in range(d)) for j in keys]
+                e = [x.exp() for x in s]  # Decimal has no overflow at these magnitudes
+                z = sum(e)
+                for c in range(d):
+                    o[b, h, i, c] = float(sum(e[n] * Decimal(float(v[b, g, j, c]))
+                                              for n, j in enumerate(keys)) / z)
+                lse[b, h, i] = float(z.ln())
+    return o, lse
+
+
+def pin_decimal_large_logits(lib):
+    for n, (B, Hq, Hkv, T, d, causal, sigma) in enumerate([
+            (1, 2, 1, 5, 3, True, 30.0),     # logits ~ +-1500: exp overflows in fp64
+            (1, 2, 2, 4, 2, False, 25.0),
+            (1, 4, 2, 3, 4, True, 0.5)]):
+        q = _rand((B, Hq, T, d), 40 + n, sigma)
+        k = _rand((B, Hkv, T, d), 50 + n, sigma)
+        v = _rand((B, Hkv, T, d), 60 + n)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.attn_fwd_f64(q, k, v, causal=causal, scale=scale, lib=lib)
+        eo, else_ = _decimal_attention(q, k, v, causal, scale)
+        assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), ("non-finite", n)
+        assert np.max(np.abs(o - eo)) <= 1e-12 * max(1.0, np.max(np.abs(eo))), ("O", n)
+        assert np.max(np.abs(lse - else_)) <= 1e-12 * max(1.0, np.max(np.abs(else_))), ("LSE", n)
+
+
+def pin_invariants(lib):
+    B, Hq, Hkv, T, d = 2, 6, 2, 37, 8
+    G = Hq // Hkv
+    scale = 0.3
+    q = _rand((B, Hq, T, d), 1)
+    k = _rand((B, Hkv, T, d), 2)
+    v = _rand((B, Hkv, T, d), 3)
+    o, lse = oracle.attn_fwd_f64(q, k, v, causal=True, scale=scale, lib=lib)
+
+    # causal row 0 attends to key 0 only: O = V[g, 0] exactly, LSE = s_00
+    for h in range(Hq):
+        g = h // G
+        assert np.array_equal(o[:, h, 0], v[:, g, 0]), "causal row 0 != V[0]"
+        s00 = scale * np.einsum("bc,bc->b", q[:, h, 0], k[:, g, 0])
+        assert np.allclose(lse[:, h, 0], s00, rtol=0, atol=1e-14), "LSE row 0 != s00"
+
+    # identical V rows give that row back
+    c = _rand((B, Hkv, 1, d), 4)
+    o_c, _ = oracle.attn_fwd_f64(q, k, np.repeat(c, T, axis=2), causal=True, scale=scale, lib=lib)
+    assert np.allclose(o_c, np.repeat(np.repeat(c, G, axis=1), T, axis=2), rtol=0, atol=1e-14)
+
+    # zero queries: uniform weights over the visible prefix
+    z = np.zeros_like(q)
+    o_z, lse_z = oracle.attn_fwd_f64(z, k, v, causal=True, scale=scale, lib=lib)
+    prefix_mean = np.cumsum(v, axis=2) / np.arange(1, T + 1)[None, None, :, None]
+    assert np.allclose(o_z, np.repeat(prefix_mean, G, axis=1), rtol=0, atol=1e-13)
+    assert np.allclose(lse_z, np.log(np.arange(1, T + 1))[None, None, :], rtol=0, atol=1e-14)
+    o_zf, lse_zf = oracle.attn_fwd_f64(z, k, v, causal=False, scale=scale, lib=lib)
+    assert np.allclose(o_zf, np.repeat(v.mean(axis=2, keepdims=True), Hq // Hkv, axis=1)
+                       .repeat(T, axis=2), rtol=0, atol=1e-13)
+    assert np.allclose(lse_zf, math.log(T), rtol=0, atol=1e-14)
+
+    # GQA equals MHA with K/V heads repeated, bit for bit
+    o_m, lse_m = oracle.attn_fwd_f64(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1),
+                                     causal=True, scale=scale, lib=lib)
+    assert np.array_equal(o_m, o) and np.array_equal(lse_m, lse), "GQA != repeated MHA"
+
+    # the last causal row sees every key: equal to the non-causal last row
+    o_f, lse_f = oracle.attn_fwd_f64(q, k, v, causal=False, scale=scale, lib=lib)
+    assert np.array_equal(o_f[:, :, -1], o[:, :, -1]) and np.array_equal(lse_f[:, :, -1], lse[:, :, -1])
+
+    # adding one vector to every key shifts each row's logits by a constant
+    shift = _rand((B, Hkv, 1, d), 5)
+    o_s, lse_s = oracle.attn_fwd_f64(q, k + shift, v, causal=True, scale=scale, lib=lib)
+    delta = scale * np.einsum("bhtc,bhc->bht", q, np.repeat(shift[:, :, 0], G, axis=1))
+    assert np.allclose(o_s, o, rtol=0, atol=1e-12), "O not shift invariant"
+    assert np.allclose(lse_s, lse + delta, rtol=0, atol=1e-12), "LSE shift wrong"
+
+    # permuting keys and values together leaves non-causal attention unchanged
+    perm = np.random.default_rng(6).permutation(T)
+    o_p, lse_p = oracle.attn_fwd_f64(q, k[:, :, perm], v[:, :, perm], causal=False,
+                                     scale=scale, lib=lib)
+    assert np.allclose(o_p, o_f, rtol=0, atol=1e-13) and np.allclose(lse_p, lse_f, rtol=0, atol=1e-13)
+
+    # scale is a plain multiplier of the logits
+    o_h, lse_h = oracle.attn_fwd_f64(2.0 * q, k, v, causal=True, scale=scale / 2.0, lib=lib)
+    assert np.allclose(o_h, o, rtol=0, atol=1e-13) and np.allclose(lse_h, lse, rtol=0, atol=1e-13)
+
+    # O is a convex combination of the visible V rows
+    for h in range(Hq):
+        g = h // G
+        lo = np.minimum.accumulate(v[:, g], axis=1)
+        hi = np.maximum.accumulate(v[:, g], axis=1)
+        assert np.all(o[:, h] >= lo - 1e-13) and np.all(o[:, h] <= hi + 1e-13)
+
+
+def pin_rows_entry(lib):
+    """The bf16 row entry agrees bit for bit with the full fp64 entry."""
+    from causal_gqa_attention_03_b200.inputs import make_qkv, bf16_bits, sample_rows
+    B, Hq, Hkv, T, d = 2, 4, 2, 150, 64
+    q, k, v = make_qkv(B, Hq, Hkv, T, d, seed=7, sigma_qk=2.0)
+    scale = 1.0 / 8.0
+    for causal in (True, False):
+        o, lse = oracle.attn_fwd_f64(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                     causal=causal, scale=scale, lib=lib)
+        rows = sample_rows(B, Hq, T, 64, seed=8)
+        ro, rlse = oracle.attn_rows_bf16(bf16_bits(q), bf16_bits(k), bf16_bits(v), rows,
+                                         causal=causal, scale=scale, lib=lib)
+        b, h, i = rows.T
+        assert np.array_equal(ro, o[b, h, i]) and np.array_equal(rlse, lse[b, h, i])
+
+
+ALL_PINS = [pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
+            pin_rows_entry]
