@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark: causal GQA attention forward TFLOP/s (bf16) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl tessera|reference]
+
+One step = one attention forward (the whole hot path) over one batch of the
+workload's synthetic inputs, already resident in HBM.  Each timed step is
+preceded by an L2 flush (a 256 MB write) and timed with CUDA events on the
+launching stream; the flush is outside the events.  For N > 1 (torchrun, one
+rank per GPU) every rank runs the same workload on its own inputs (weak
+scaling: independent batches, no collective on the data path); the reported
+time is the max over ranks.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead, on a bounded sample of rows of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_gqa_attention_03_b200 import inputs  # noqa: E402
+
+METRIC = "causal GQA attn fwd TFLOP/s (bf16) and % of B200 roofline vs fp64 CPU oracle"
+UNIT = "TFLOP/s"
+FLUSH_BYTES = 256 << 20
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch; rank 0 uses the workload's own seed."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 100):
+        self.index = index
+        self.period_ms = period_ms
+        self.lines = []
+        self.proc = None
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for t, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append(dict(t=t, sm=float(parts[2]), smax=float(parts[3]),
+                                 power=float(parts[4]) if parts[4] not in ("[N/A]", "N/A") else None,
+                                 hw=parts[6], hwt=parts[7], swt=parts[8], swp=parts[9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        inside = [r for r in rows if any(a - 0.15 <= r["t"] <= b + 0.15 for a, b in self.windows)]
+        use = inside or rows
+        reasons = set()
+        for r in use:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in use),
+                "sm_max_mhz": max(r["smax"] for r in use),
+                "reasons": sorted(reasons),
+                "samples": len(use),
+                "samples_in_timed_region": len(inside),
+                "power_w_max": max((r["power"] for r in use if r["power"] is not None), default=None)}
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_rows_rate(w, q, k, v, seconds: float, seed: int, max_rows: int | None = None):
+    """Time the fp64 oracle on random rows of the workload for about `seconds`.
+
+    Returns (TFLOP/s, rows done, flops done, elapsed).  A row i costs
+    4*d*(i+1) flops of causal attention (2*d per key for QK^T and for PV),
+    summing to the metric's 2*B*Hq*T^2*d over the whole workload (up to T+1/T).
+    """
+    import numpy as np
+    import oracle
+    qb, kb, vb = inputs.bf16_bits(q), inputs.bf16_bits(k), inputs.bf16_bits(v)
+    rng = np.random.default_rng(seed)
+    flops = 0.0
+    rows_done = 0
+    t0 = time.perf_counter()
+    while True:
+        n = 16
+        rows = np.stack([rng.integers(0, w.B, n), rng.integers(0, w.Hq, n),
+                         rng.integers(0, w.T, n)], axis=1).astype(np.int64)
+        rows = rows[np.lexsort((rows[:, 2], rows[:, 1], rows[:, 0]))]
+        oracle.attn_rows_bf16(qb, kb, vb, rows, causal=w.causal, scale=w.scale)
+        flops += float(np.sum(4.0 * w.d * (rows[:, 2] + 1)))
+        rows_done += n
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_rows is not None and rows_done >= max_rows):
+            break
+    return flops / el / 1e12, rows_done, flops, el
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    q, k, v = inputs.workload_inputs(w)
+    step_seconds = 0.5
+    for i in range(args.warmup):
+        oracle_rows_rate(w, q, k, v, step_seconds, seed=100 + i)
+    flops = 0.0
+    el = 0.0
+    rows = 0
+    for i in range(args.steps):
+        _, r, f, e = oracle_rows_rate(w, q, k, v, step_seconds, seed=1000 + i)
+        flops += f
+        el += e
+        rows += r
+    value = flops / el / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, **{k_: getattr(w, k_) for k_ in
+                                          ("B", "T", "Hq", "Hkv", "d", "causal")}},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} random (b,h,i) rows of {w.name}, "
+                                   f"{args.steps} steps of ~{step_seconds}s, single thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- GPU arm
+def time_kernel(w, q, k, v, steps, warmup, flush, stream, tess, torch):
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=q.device)
+    launches = 0
+    for _ in range(warmup):
+        flush.zero_()
+        tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        launches += tess.tessera_attn_last_launch_count()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return times, launches, o, lse
+
+
+def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
+    """Public API end to end: pinned host inputs -> device -> attention -> host outputs."""
+    q_d = torch.empty(q_h.shape, dtype=q_h.dtype, device=dev)
+    k_d = torch.empty(k_h.shape, dtype=k_h.dtype, device=dev)
+    v_d = torch.empty(v_h.shape, dtype=v_h.dtype, device=dev)
+    o_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
+    l_h = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, pin_memory=True)
+
+    def step():
+        with torch.cuda.stream(stream):
+            q_d.copy_(q_h, non_blocking=True)
+            k_d.copy_(k_h, non_blocking=True)
+            v_d.copy_(v_h, non_blocking=True)
+            o, lse = tess.attn_fwd(q_d, k_d, v_d, causal=w.causal, scale=w.scale, stream=stream)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+    d2h = o_h.numel() * 2 + l_h.numel() * 4
+    return ms, h2d, d2h
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=inputs.LARGEST, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="tessera", choices=["tessera", "reference"])
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import causal_gqa_attention_03_b200 as tess
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+    tess.load_library()
+
+    q_h, k_h, v_h = inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
+                                    rank_seed(w.seed, rank), w.sigma_qk)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    times, launches, _, _ = time_kernel(w, q, k, v, args.steps, args.warmup, flush, stream,
+                                        tess, torch)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.mark(t_wall0, t_wall1)
+    err = tess.tessera_attn_device_error()
+    if err != 0:
+        raise SystemExit(f"device-side wait gave up (code {err})")
+
+    kernel_ms = sum(times)
+    max_ms = max_over_ranks(kernel_ms, dev)
+    total_flops = w.flops * args.steps * world
+    value = total_flops / (max_ms * 1e-3) / 1e12
+    ms_per_step = max_ms / args.steps
+    per_launch_ms = statistics.mean(times)
+    achieved = w.flops / (per_launch_ms * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    q_pin, k_pin, v_pin = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    e2e_ms, h2d, d2h = time_e2e(w, q_pin, k_pin, v_pin, args.e2e_steps, 3, stream, tess, torch,
+                                dev)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_value = w.flops * world / (e2e_ms * 1e-3) / 1e12
+
+    sweep = {}
+    if not args.no_sweep and world == 1:
+        for name, ws in inputs.WORKLOADS.items():
+            if name == w.name:
+                sweep[name] = {"tflops": round(value, 1), "ms": round(ms_per_step, 4)}
+                continue
+            qs, ks, vs = (t.to(dev) for t in inputs.workload_inputs(ws))
+            n = max(5, min(200, int(0.5 / max(ws.flops / 1.2e15, 1e-6))))
+            ts, _, _, _ = time_kernel(ws, qs, ks, vs, n, 3, flush, stream, tess, torch)
+            ms = statistics.median(ts)
+            sweep[name] = {"tflops": round(ws.flops / (ms * 1e-3) / 1e12, 1),
+                           "ms": round(ms, 4)}
+            del qs, ks, vs
+        err = tess.tessera_attn_device_error()
+        if err != 0:
+            raise SystemExit(f"device-side wait gave up in the sweep (code {err})")
+
+    clocks.stop()
+    clk = clocks.summary()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    traffic = None
+    prof_traffic = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof_traffic):
+        with open(prof_traffic) as f:
+            tr = json.load(f)
+        if tr.get("workload") == w.name and tr.get("kernel_source_sha") == kernel_source_sha():
+            traffic = tr.get("bytes_per_launch")
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+                "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        rate, rows, _, el = oracle_rows_rate(w, q_h, k_h, v_h, args.cpu_seconds, seed=1)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{rows} random (b,h,i) rows of {w.name} in {el:.1f}s, "
+                         "fp64, single thread"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "causal": w.causal, "sigma_qk": w.sigma_qk, "seed": w.seed,
+                   "l2": "flushed before every timed step (256 MB write, outside the events)",
+                   "parallelism": f"dp{world} (independent batch per GPU)"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "path": "pinned host Q/K/V -> device, attn_fwd, O/LSE -> pinned host"},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "sweep": sweep or None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_gqa_attention_03_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,123 @@
+"""Causal grouped-query FlashAttention forward for B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/tessera_attn.h``; every
+step of the computation runs in the CUDA library ``libtessera_attn.so``
+built in this directory (``python -m causal_gqa_attention_03_b200.build``).
+There is no fallback: if the library is missing, every call raises.
+
+Raw C-ABI names (integer pointers, sizes, stream handle):
+    tessera_attn_fwd, tessera_attn_device_error, tessera_status_str,
+    tessera_attn_last_launch_count
+Tensor convenience wrapper (PyTorch used only for memory and streams):
+    attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_attn.so")
+
+# Symbols declared in include/tessera_attn.h.
+EXPORTED = ("tessera_attn_fwd", "tessera_attn_device_error", "tessera_status_str",
+            "tessera_attn_last_launch_count")
+
+STATUS = {0: "TESSERA_OK", 1: "TESSERA_ERR_INVALID_ARG", 2: "TESSERA_ERR_UNSUPPORTED",
+          3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TesseraError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({tessera_status_str(status)})")
+        self.status = status
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libtessera_attn.so; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"CUDA library not built: {LIB_PATH} is missing "
+                    "(run python -m causal_gqa_attention_03_b200.build)")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp = ctypes.c_void_p
+            ci = ctypes.c_int
+            lib.tessera_attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci,
+                                             ctypes.c_float, vp]
+            lib.tessera_attn_fwd.restype = ci
+            lib.tessera_attn_device_error.argtypes = [ctypes.POINTER(ci)]
+            lib.tessera_attn_device_error.restype = ci
+            lib.tessera_status_str.argtypes = [ci]
+            lib.tessera_status_str.restype = ctypes.c_char_p
+            lib.tessera_attn_last_launch_count.argtypes = []
+            lib.tessera_attn_last_launch_count.restype = ci
+            _lib = lib
+    return _lib
+
+
+def tessera_attn_fwd(q: int, k: int, v: int, o: int, lse: int | None, B: int, Hq: int,
+                     Hkv: int, T: int, d: int, causal: int, scale: float,
+                     stream: int | None) -> int:
+    """The C entry point with integer device pointers; returns the status code."""
+    return load_library().tessera_attn_fwd(q, k, v, o, lse or None, B, Hq, Hkv, T, d,
+                                           int(causal), float(scale), stream or None)
+
+
+def tessera_attn_device_error() -> int:
+    """Read and clear the device-side error word (synchronises the device)."""
+    code = ctypes.c_int(0)
+    st = load_library().tessera_attn_device_error(ctypes.byref(code))
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_device_error")
+    return code.value
+
+
+def tessera_status_str(status: int) -> str:
+    return load_library().tessera_status_str(int(status)).decode()
+
+
+def tessera_attn_last_launch_count() -> int:
+    return load_library().tessera_attn_last_launch_count()
+
+
+def attn_fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=None,
+             stream=None, want_lse: bool = True):
+    """Attention forward on CUDA bf16 tensors q [B,Hq,T,d], k/v [B,Hkv,T,d].
+
+    Returns (o, lse): o bf16 [B,Hq,T,d]; lse fp32 [B,Hq,T] (None when
+    want_lse is False and no lse buffer is given).  Outputs are allocated with
+    torch unless given.  The kernel is queued on ``stream`` (default: torch's
+    current stream) and the call does not synchronise.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D tensor [B,H,T,d]")
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, T, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B,Hkv,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = tessera_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, B, Hq, Hkv, T, d,
+                          int(bool(causal)), float(scale), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_fwd")
+    return out, lse

@@ -1,0 +1,173 @@
+// C ABI of the causal grouped-query attention forward (see include/tessera_attn.h).
+//
+// Host side: argument checks, TMA tensor maps for Q/K/V, work decomposition,
+// and the kernel launch on the caller's stream.  Nothing here allocates device
+// memory or synchronises.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tessera_attn.h"
+#include "attn_fwd_sm100.cuh"
+
+namespace {
+
+using tessera::FwdCfg;
+using tessera::FwdParams;
+
+thread_local int g_last_launches = 0;
+std::atomic<unsigned long long> g_launch_counter{1};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [planes, T, d] bf16 viewed as a 3-D tensor (d innermost); boxes of
+// 64 columns x 128 rows x 1 plane with the 128-byte swizzle.  Rows at or past
+// T read as zero.
+bool make_map(CUtensorMap* map, const void* base, int planes, int T, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int T, int causal, float scale, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TESSERA_ERR_CUDA;
+  static std::atomic<bool> attr_set[64];
+  if (dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(tessera::attn_fwd_sm100_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return TESSERA_ERR_CUDA;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
+      !make_map(&tm_v, v, B * Hkv, T, D))
+    return TESSERA_ERR_CUDA;
+
+  FwdParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = T;
+  p.G = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.nqb = (T + C::BM - 1) / C::BM;
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  long long units;
+  if (p.pair_heads) {
+    p.units_per_step = B * Hkv * (p.G / 2);
+    units = static_cast<long long>(p.units_per_step) * p.nqb;
+  } else {
+    p.units_per_step = B * Hq;
+    units = static_cast<long long>(p.units_per_step) * ((p.nqb + 1) / 2);
+  }
+  if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+
+  tessera::attn_fwd_sm100_kernel<D>
+      <<<static_cast<unsigned>(units), C::THREADS, C::SMEM_BYTES, stream>>>(tm_q, tm_k, tm_v, p);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  g_last_launches = 1;
+  return TESSERA_OK;
+}
+
+}  // namespace
+
+extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int T, int d, int causal, float scale,
+                                tessera_stream_t stream) {
+  g_last_launches = 0;
+  if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TESSERA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return TESSERA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TESSERA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TESSERA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return TESSERA_OK;
+  // sizes in bytes; every product below stays far inside 64 bits for int inputs
+  const size_t q_bytes = static_cast<size_t>(B) * Hq * T * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * T * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(B) * Hq * T * 4;
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned16(lse)))
+    return TESSERA_ERR_MISALIGNED;
+  if (overlaps(o, q_bytes, q, q_bytes) || overlaps(o, q_bytes, k, kv_bytes) ||
+      overlaps(o, q_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+      overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes) ||
+      overlaps(lse, lse_bytes, o, q_bytes))
+    return TESSERA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch<64>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
+  return launch<128>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
+}
+
+extern "C" int tessera_attn_device_error(int* code) {
+  if (!code) return TESSERA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TESSERA_ERR_CUDA;
+  unsigned long long w = 0;
+  if (cudaMemcpyFromSymbol(&w, tessera::g_tessera_err, sizeof(w)) != cudaSuccess)
+    return TESSERA_ERR_CUDA;
+  const unsigned long long zero = 0;
+  if (cudaMemcpyToSymbol(tessera::g_tessera_err, &zero, sizeof(zero)) != cudaSuccess)
+    return TESSERA_ERR_CUDA;
+  *code = static_cast<int>(w & 0xffffffffull);
+  return TESSERA_OK;
+}
+
+extern "C" const char* tessera_status_str(int status) {
+  switch (status) {
+    case TESSERA_OK: return "ok";
+    case TESSERA_ERR_INVALID_ARG: return "invalid argument";
+    case TESSERA_ERR_UNSUPPORTED: return "unsupported head dimension (64 or 128)";
+    case TESSERA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case TESSERA_ERR_CUDA: return "CUDA runtime error";
+    case TESSERA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int tessera_attn_last_launch_count(void) { return g_last_launches; }

@@ -1,0 +1,413 @@
+// Causal grouped-query FlashAttention forward for B200 (sm_100a).
+//
+// Method: FlashAttention forward with online softmax, causal masking and
+// grouped-query attention, as named by the Tessera pages (hysenlabs.com
+// Tessera review, "The kernel set and its torch fallback"; Tessera README,
+// "What's in it" / "Kernels").  The tile design below is this library's own,
+// built for sm_100a: TMA + mbarrier pipeline, tcgen05 MMAs accumulating in
+// tensor memory, warp-specialised roles.
+//
+// One CTA processes one work unit: two 128-row query tiles that read the same
+// key/value head.  When the group size G is even the two tiles are two query
+// heads of one group at the same rows (so each K/V tile fetched into shared
+// memory feeds both); otherwise they are two consecutive 128-row blocks of one
+// head.  Units are numbered heaviest-first so the causal triangle balances.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue for query tile 0 (thread r owns row r)
+//   warps 4-7  softmax + epilogue for query tile 1
+//   warp  8    MMA issue (one lane) and TMEM allocation
+//   warp  9    TMA producer (one lane)
+//
+// Tensor memory (512 columns x 128 lanes, fp32 cells):
+//   S_t = Q_t K_j^T  columns [128 t, 128 t + 128)      (t = 0, 1)
+//   P_t (bf16 pairs) columns [128 t, 128 t + 64), written over S_t
+//   O_t             columns [256 + D t, 256 + D t + D)
+//
+// Per key tile j and query tile t the MMA warp issues PV_t(j-1) then S_t(j);
+// tcgen05 MMAs from one thread execute in order, so S_t(j) cannot overwrite
+// P_t(j-1) before PV_t(j-1) has read it.  The softmax of tile t overlaps the
+// MMAs of the other tile.  The running max is rescaled lazily: O and l keep a
+// stale max until the row max grows by more than 2^8, which is exact because
+// both carry the same max.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace tessera {
+
+// Device error word: high 32 bits = launch id, low 32 bits = code of the wait
+// that gave up.  Nonzero only after a bounded wait expired.
+__device__ unsigned long long g_tessera_err = 0ull;
+
+enum WaitCode : uint32_t {
+  kErrWaitQ = 1,
+  kErrWaitKvEmpty = 2,
+  kErrWaitKvFull = 3,
+  kErrWaitSFull = 4,
+  kErrWaitPFull = 5,
+  kErrWaitOFull = 6,
+  kErrWaitDrain = 7,
+};
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
+constexpr float kRescaleThreshold = 8.0f;          // log2 units: rescale when the max grows > 2^8
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+  static constexpr int BM = 128;                  // query rows per tile
+  static constexpr int BN = 128;                  // keys per tile
+  static constexpr int NQ = 2;                    // query tiles per CTA
+  static constexpr int SUB = D / 64;              // 128-byte-wide column sub-tiles per tile
+  static constexpr int SUB_BYTES = 128 * 128;     // one [128 rows x 64 bf16] sub-tile
+  static constexpr int TILE_BYTES = 128 * D * 2;  // one [128 x D] bf16 tile
+  static constexpr int NSTAGE = (D == 128) ? 5 : 8;
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = NQ * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
+  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ + 1;
+  static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack to align the base to 1 KB
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int S_COL = 0;
+  static constexpr int O_COL = 256;
+  static constexpr int THREADS = 320;
+  static constexpr int MMA_WARP = 8;
+  static constexpr int TMA_WARP = 9;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(O_COL + NQ * D <= 512, "tensor memory budget");
+};
+
+struct FwdParams {
+  int B, Hq, Hkv, T, G;
+  int causal;
+  float scale_log2;          // scale * log2(e)
+  int nqb;                   // ceil(T / 128)
+  int pair_heads;            // 1: tiles are heads (2p, 2p+1) of a group; 0: q-blocks (2p, 2p+1)
+  int units_per_step;        // units sharing one position in the heaviest-first order
+  __nv_bfloat16* o;
+  float* lse;
+  unsigned long long launch_id;
+};
+
+// Wait for the phase of `parity` on `bar`, giving up after kWaitLimitNs or as
+// soon as another CTA of the same launch has given up.  Returns false on give-up.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t code,
+                                             unsigned long long launch_id) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 1023u) == 0) {
+      const unsigned long long w = *reinterpret_cast<volatile unsigned long long*>(&g_tessera_err);
+      if ((w >> 32) == (launch_id & 0xffffffffull) && (w & 0xffffffffull) != 0) return false;
+      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicExch(&g_tessera_err, ((launch_id & 0xffffffffull) << 32) | code);
+        return false;
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+
+  uint8_t* sQ = smem + C::Q_OFF;
+  uint8_t* sKV = smem + C::KV_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + C::NSTAGE;
+  uint64_t* s_full = kv_empty + C::NSTAGE;
+  uint64_t* p_full = s_full + C::NQ;
+  uint64_t* o_full = p_full + C::NQ;
+  uint64_t* drain = o_full + C::NQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SLOT_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- decode the work unit (heaviest first) --------------------------------
+  const int u = blockIdx.x;
+  const int step = u / p.units_per_step;
+  const int r = u % p.units_per_step;
+  int b, g, head[2], qblk[2];
+  if (p.pair_heads) {
+    const int half = p.G >> 1;
+    const int hp = r % half;
+    const int bg = r / half;
+    b = bg / p.Hkv;
+    g = bg % p.Hkv;
+    head[0] = g * p.G + 2 * hp;
+    head[1] = head[0] + 1;
+    qblk[0] = qblk[1] = p.nqb - 1 - step;
+  } else {
+    const int npairs = (p.nqb + 1) >> 1;
+    const int pr = npairs - 1 - step;
+    b = r / p.Hq;
+    head[0] = head[1] = r % p.Hq;
+    g = head[0] / p.G;
+    qblk[0] = 2 * pr;
+    qblk[1] = 2 * pr + 1;
+  }
+  const int nkv = p.nqb;
+  int ntile[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const bool valid = qblk[t] < p.nqb;
+    ntile[t] = !valid ? 0 : (p.causal ? min(qblk[t] + 1, nkv) : nkv);
+  }
+  const int nmax = max(ntile[0], ntile[1]);
+  const int kv_plane = b * p.Hkv + g;
+
+  // ---- set-up ---------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < C::NQ; ++t) {
+      ptx::mbar_init(&s_full[t], 1);
+      ptx::mbar_init(&p_full[t], 4);  // one arrival per softmax warp
+      ptx::mbar_init(&o_full[t], 1);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::TMA_WARP && lane == 0) {
+    ptx::prefetch_tensormap(&tm_q);
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+  }
+  if (warp == C::MMA_WARP) {
+    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::TMA_WARP) {
+    // ======================= TMA producer ===================================
+    if (lane == 0) {
+      const int nvalid = (ntile[0] > 0) + (ntile[1] > 0);
+      ptx::mbar_arrive_expect_tx(q_full, nvalid * C::TILE_BYTES);
+      for (int t = 0; t < C::NQ; ++t) {
+        if (ntile[t] == 0) continue;
+        for (int c = 0; c < C::SUB; ++c)
+          ptx::tma_load_3d(sQ + t * C::TILE_BYTES + c * C::SUB_BYTES, &tm_q, q_full, c * 64,
+                           qblk[t] * C::BM, b * p.Hq + head[t]);
+      }
+      int issued = 0;
+      for (int idx = 0; idx < 2 * nmax; ++idx) {  // K_0, V_0, K_1, V_1, ...
+        const int s = idx % C::NSTAGE;
+        const uint32_t ph = (idx / C::NSTAGE) & 1;
+        if (!wait_bounded(&kv_empty[s], ph ^ 1u, kErrWaitKvEmpty, p.launch_id)) break;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+        const CUtensorMap* map = (idx & 1) ? &tm_v : &tm_k;
+        const int j = idx >> 1;
+        for (int c = 0; c < C::SUB; ++c)
+          ptx::tma_load_3d(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s], c * 64,
+                           j * C::BN, kv_plane);
+        ++issued;
+      }
+      if (issued < 2 * nmax) {
+        // Gave up: let the copies already in flight land before the CTA exits.
+        wait_bounded(q_full, 0, kErrWaitQ, p.launch_id);
+        for (int idx = max(0, issued - C::NSTAGE); idx < issued; ++idx)
+          wait_bounded(&kv_full[idx % C::NSTAGE], (idx / C::NSTAGE) & 1, kErrWaitKvFull,
+                       p.launch_id);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::MMA_WARP) {
+    // ======================= MMA issue ======================================
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
+      bool ok = wait_bounded(q_full, 0, kErrWaitQ, p.launch_id);
+      const uint32_t q_addr = ptx::smem_u32(sQ);
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      for (int j = 0; ok && j <= nmax; ++j) {
+        const int kidx = 2 * j, vidx = 2 * j - 1;
+        if (j < nmax)
+          ok = wait_bounded(&kv_full[kidx % C::NSTAGE], (kidx / C::NSTAGE) & 1, kErrWaitKvFull,
+                            p.launch_id);
+        if (ok && j > 0)
+          ok = wait_bounded(&kv_full[vidx % C::NSTAGE], (vidx / C::NSTAGE) & 1, kErrWaitKvFull,
+                            p.launch_id);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        for (int t = 0; t < C::NQ && ok; ++t) {
+          if (j >= 1 && j <= ntile[t]) {
+            // O_t += P_t(j-1) V_{j-1}; A = P from TMEM, B = V (MN-major in smem)
+            ok = wait_bounded(&p_full[t], (j - 1) & 1, kErrWaitPFull, p.launch_id);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t v_base = kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 16; ++kk) {
+              const uint64_t bdesc = ptx::sdesc_sw128(v_base + kk * 16 * 128, C::SUB_BYTES, 1024);
+              ptx::mma_ts(tmem + C::O_COL + D * t, tmem + C::S_COL + 128 * t + kk * 8, bdesc,
+                          kIdescO, (j > 1 || kk > 0) ? 1u : 0u);
+            }
+            if (j == ntile[t]) ptx::tc_commit(&o_full[t]);
+          }
+          if (j < ntile[t]) {
+            // S_t = Q_t K_j^T; both operands K-major in smem
+            const uint32_t qa = q_addr + t * C::TILE_BYTES;
+            const uint32_t kb = kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
+              ptx::mma_ss(tmem + C::S_COL + 128 * t, ptx::sdesc_sw128(qa + off, 16, 1024),
+                          ptx::sdesc_sw128(kb + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+            }
+            ptx::tc_commit(&s_full[t]);
+          }
+        }
+        if (!ok) break;
+        if (j < nmax) ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);
+        if (j > 0) ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);
+      }
+      // Every MMA issued must finish before tensor memory is released.
+      ptx::tc_commit(drain);
+      wait_bounded(drain, 0, kErrWaitDrain, p.launch_id);
+    }
+    __syncwarp();
+  } else {
+    // ======================= softmax + epilogue =============================
+    const int t = warp >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int n_t = ntile[t];
+    if (n_t > 0) {
+      const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+      const uint32_t s_addr = tmem + lane_base + C::S_COL + 128 * t;
+      const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
+      const int q_row = qblk[t] * C::BM + row;
+      const float sl2 = p.scale_log2;
+      float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale)
+      float l = 0.f;        // running sum of 2^(x - m)
+      bool ok = true;
+      for (int j = 0; j < n_t; ++j) {
+        // every lane polls; the warp proceeds only if all saw the phase complete
+        if (!__all_sync(0xffffffffu, wait_bounded(&s_full[t], j & 1, kErrWaitSFull, p.launch_id))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_addr + 32 * c, sr[c]);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::reg_fence(sr[c]);
+
+        const int kv0 = j * C::BN;
+        const bool edge = p.causal ? (kv0 + C::BN - 1 > q_row - row) : (kv0 + C::BN > p.T);
+        if (edge) {
+          const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (kv0 + c > lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
+        const float m_tile = mx * sl2;
+        float alpha = 1.f;
+        const bool rescale = m_tile > m + kRescaleThreshold;
+        if (rescale) {
+          alpha = ptx::ex2(m - m_tile);  // 0 on the first tile (m = -inf)
+          m = m_tile;
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        float rowsum = 0.f;
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x0 = __uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]);
+          const float x1 = __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
+          const float p0 = ptx::ex2(fmaf(x0, sl2, neg_m));
+          const float p1 = ptx::ex2(fmaf(x1, sl2, neg_m));
+          rowsum += p0 + p1;
+          pk[c >> 5][c & 31] = ptx::pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + rowsum;
+        ptx::tmem_st32(s_addr + 0, pk[0]);
+        ptx::tmem_st32(s_addr + 32, pk[1]);
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O_t *= alpha (PV_t(j-1) is complete: S_t(j) was committed after it)
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(o_addr + 32 * c, ov);
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            ptx::tmem_st32(o_addr + 32 * c, ov);
+          }
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&p_full[t]);
+      }
+
+      // ---- epilogue: O / l -> bf16, LSE ---------------------------------------
+      if (ok) ok = wait_bounded(&o_full[t], 0, kErrWaitOFull, p.launch_id);
+      if (__all_sync(0xffffffffu, ok)) {
+        ptx::tc_fence_after();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const bool store = q_row < p.T;
+        const int64_t orow = (static_cast<int64_t>(b) * p.Hq + head[t]) * p.T + q_row;
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(o_addr + 32 * c, ov);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(ov);
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            packed[i] = ptx::pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
+                                         __uint_as_float(ov[2 * i + 1]) * inv_l);
+          if (store) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[c * 4 + v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2],
+                                           packed[4 * v4 + 3]);
+          }
+        }
+        if (store && p.lse != nullptr)
+          p.lse[orow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  // ---- teardown -------------------------------------------------------------
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace tessera

@@ -1,0 +1,94 @@
+/*
+ * tessera_attn.h -- C ABI of the causal grouped-query FlashAttention forward
+ * pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the attention forward kernel that the Tessera pages name:
+ * "a FlashAttention forward kernel with online softmax, causal masking,
+ * grouped-query attention" (hysenlabs.com Tessera review, section "The kernel
+ * set and its torch fallback"; Tessera README, "What's in it" / "Kernels"),
+ * used by the decoder with "RMSNorm, RoPE, grouped-query attention and
+ * SwiGLU" (Tessera README, "What's in it" / "Training side").  The pages give
+ * no formula; the plain reading adopted here is scaled-dot-product attention:
+ *
+ *   G = Hq / Hkv; query head h reads key/value head floor(h / G)
+ *   s_ij = scale * dot(Q[b,h,i,:], K[b,g,j,:]),  j <= i when causal
+ *   O[b,h,i,:] = sum_j softmax_j(s_i) * V[b,g,j,:]
+ *   LSE[b,h,i] = ln sum_j exp(s_ij)     (natural log of the scaled logits)
+ *
+ * No C++ or CUDA types appear in this header; the library links the CUDA
+ * runtime statically and needs a CUDA driver only when a function below that
+ * launches work is called.
+ */
+#ifndef TESSERA_ATTN_H
+#define TESSERA_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL means the legacy default stream. */
+typedef struct CUstream_st *tessera_stream_t;
+
+typedef enum {
+    TESSERA_OK = 0,
+    TESSERA_ERR_INVALID_ARG = 1, /* bad size, null pointer, aliasing, bad scale */
+    TESSERA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128 */
+    TESSERA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
+    TESSERA_ERR_CUDA = 4,        /* the CUDA runtime reported an error */
+    TESSERA_ERR_TIMEOUT = 5      /* a device-side wait gave up (see below) */
+} tessera_status;
+
+/*
+ * Causal (or full) grouped-query attention forward on one GPU.
+ *
+ * q    bf16 [B, Hq,  T, d]  device memory, contiguous row-major, read only
+ * k    bf16 [B, Hkv, T, d]  device memory, contiguous row-major, read only
+ * v    bf16 [B, Hkv, T, d]  device memory, contiguous row-major, read only
+ * o    bf16 [B, Hq,  T, d]  device memory, written (rounded to nearest even)
+ * lse  fp32 [B, Hq,  T]     device memory, written; may be NULL to skip it
+ * B, Hq, Hkv, T  sizes; B >= 0, T >= 0 (either 0 returns TESSERA_OK and
+ *      launches nothing), Hq >= 1, Hkv >= 1, Hq % Hkv == 0
+ * d    head dimension: 64 or 128, else TESSERA_ERR_UNSUPPORTED
+ * causal  1: row i attends to keys j <= i; 0: to every key j < T
+ * scale   positive finite multiplier of Q.K^T (typically 1/sqrt(d))
+ * stream  the CUDA stream the work is queued on
+ *
+ * All buffers are owned by the caller.  The call allocates no device memory,
+ * does not synchronise, and returns as soon as the kernel is queued.  Every
+ * pointer must be 16-byte aligned (TESSERA_ERR_MISALIGNED), non-NULL when its
+ * tensor is non-empty, and o / lse must not overlap q, k, v or each other
+ * (TESSERA_ERR_INVALID_ARG).  Arguments are checked before any CUDA call, so a
+ * rejected call has no effect.  Launch failures return TESSERA_ERR_CUDA.
+ *
+ * Every wait inside the kernel is bounded; if one gives up (it never does in
+ * a correct run) the kernel records the fact in a device-side error word and
+ * exits without hanging.  tessera_attn_device_error() reads that word.
+ */
+int tessera_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                     float *lse, int B, int Hq, int Hkv, int T, int d,
+                     int causal, float scale, tessera_stream_t stream);
+
+/*
+ * Reads and clears the device-side error word of the current device.  This
+ * synchronises the device.  *code receives 0 when no kernel reported a
+ * problem since the last call, else a nonzero code naming the wait that gave
+ * up.  Returns TESSERA_OK, or TESSERA_ERR_CUDA if the read failed.
+ */
+int tessera_attn_device_error(int *code);
+
+/* A static string naming a tessera_status value. */
+const char *tessera_status_str(int status);
+
+/*
+ * Kernel launches the last successful tessera_attn_fwd call on this thread
+ * queued (0 or 1).  Lets a caller count the library's own launches.
+ */
+int tessera_attn_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TESSERA_ATTN_H */

@@ -1,0 +1,93 @@
+"""The C-ABI library on CPU: it loads, exports what the header declares, and
+rejects bad arguments before touching the GPU (no compute calls here)."""
+import glob
+import os
+import re
+
+import pytest
+
+import causal_gqa_attention_03_b200 as tess
+from causal_gqa_attention_03_b200 import build as tbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tbuild.build()
+    return tess.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_]\w*\s*\**\s*(tessera_\w+)\s*\(",
+                            text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert "tessera_attn_fwd" in names
+    assert set(names) == set(tess.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_has_no_fallback_to_the_oracle():
+    # the product package never imports, loads or includes the oracle
+    pkg = os.path.join(ROOT, "causal_gqa_attention_03_b200")
+    bad = re.compile(r"^\s*(import|from)\s+oracle\b|liboracle|attn_ref|#include\s+\S*oracle",
+                     re.M)
+    for path in glob.glob(os.path.join(pkg, "**", "*"), recursive=True):
+        if path.endswith((".py", ".cu", ".cuh", ".h")):
+            assert not bad.search(open(path).read()), path
+
+
+ALIGNED = 0x10000000
+GOOD = dict(q=ALIGNED, k=ALIGNED + 0x1000000, v=ALIGNED + 0x2000000, o=ALIGNED + 0x3000000,
+            lse=ALIGNED + 0x4000000, B=1, Hq=4, Hkv=2, T=16, d=64, causal=1, scale=0.125,
+            stream=None)
+
+
+def call(**kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return tess.tessera_attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                 a["Hkv"], a["T"], a["d"], a["causal"], a["scale"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(T=-5), 1), (dict(Hq=0), 1), (dict(Hkv=0), 1),
+    (dict(Hq=6, Hkv=4), 1), (dict(d=96), 2), (dict(d=256), 2), (dict(d=0), 2),
+    (dict(scale=0.0), 1), (dict(scale=-0.5), 1), (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1), (dict(causal=2), 1),
+    (dict(q=0), 1), (dict(k=0), 1), (dict(v=0), 1), (dict(o=0), 1),
+    (dict(q=ALIGNED + 8), 3), (dict(o=ALIGNED + 0x3000002), 3), (dict(lse=ALIGNED + 0x4000004), 3),
+    (dict(o=ALIGNED + 0x40), 1),           # O overlaps Q
+    (dict(lse=ALIGNED + 0x3000000 + 64), 1),  # LSE overlaps O
+    (dict(B=0), 0), (dict(T=0), 0),        # empty: nothing to launch
+    (dict(B=0, q=0, k=0, v=0, o=0, lse=0), 0),
+])
+def test_argument_checks_before_any_cuda_call(lib, kw, status):
+    assert call(**kw) == status
+    if status != 0:
+        assert tess.tessera_attn_last_launch_count() == 0
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert tess.tessera_status_str(s)
+    assert tess.tessera_status_str(99) == "unknown status"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(tess, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(tess, "_lib", None)
+    with pytest.raises(ImportError):
+        tess.load_library()

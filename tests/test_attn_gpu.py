@@ -1,0 +1,238 @@
+"""Parity of the CUDA path with the fp64 oracle, through the C ABI, on a B200.
+
+Tolerances (stated for this path): bf16 O max |err| <= 2e-2 and mean |err|
+<= 2e-3; fp32 LSE |err| <= 1e-3, over every compared element.
+
+* small shapes and the two smallest synthetic workloads: every element;
+* the five large workloads, at full size in the launch configuration the
+  benchmark times: sampled rows computed one by one by the oracle, plus
+  properties that hold for every row (finite; O inside the convex hull of the
+  visible V rows; LSE >= the diagonal logit and >= the mean visible logit);
+* exact special cases: causal row 0, zero queries, constant V, GQA equal to
+  MHA with repeated K/V heads.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import causal_gqa_attention_03_b200 as tess
+from causal_gqa_attention_03_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    tess.load_library()
+    assert tess.tessera_attn_device_error() == 0
+
+
+def run_gpu(q, k, v, causal=True, scale=None):
+    """q, k, v: bf16 CPU tensors. Returns (o fp32 CPU, lse fp32 CPU)."""
+    dev = torch.device("cuda:0")
+    o, lse = tess.attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert tess.tessera_attn_device_error() == 0
+    return o.float().cpu(), lse.cpu()
+
+
+def check(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+    err = np.abs(o_gpu - o_ref)
+    lerr = np.abs(lse_gpu - lse_ref)
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(lse_gpu)), what
+    assert err.max() <= MAX_ABS, f"{what}: O max abs err {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: O mean abs err {err.mean():.3e}"
+    assert lerr.max() <= LSE_ABS, f"{what}: LSE max abs err {lerr.max():.3e}"
+
+
+def oracle_full(q, k, v, causal, scale):
+    return oracle.attn_fwd_f64(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                               causal=causal, scale=scale)
+
+
+# (B, Hq, Hkv, T, d, causal): tails, single tiles, G odd / even / 1, non-causal
+SMALL = [
+    (1, 2, 1, 1, 64, True), (1, 2, 1, 2, 128, True), (2, 4, 2, 63, 64, True),
+    (1, 2, 2, 127, 128, True), (1, 4, 1, 128, 64, True), (2, 2, 1, 129, 128, True),
+    (1, 3, 1, 255, 64, True), (1, 3, 3, 256, 128, True), (1, 6, 2, 300, 64, True),
+    (1, 8, 1, 385, 128, True), (1, 1, 1, 640, 64, True), (2, 6, 3, 200, 128, True),
+    (1, 2, 1, 1, 64, False), (1, 4, 2, 100, 64, False), (1, 3, 1, 129, 128, False),
+    (2, 2, 2, 256, 128, False), (1, 4, 4, 383, 64, False), (1, 8, 2, 520, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,d,causal", SMALL)
+def test_small_shapes_every_element(B, Hq, Hkv, T, d, causal):
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=1000 + T + d, sigma_qk=1.5)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_gpu(q, k, v, causal, scale)
+    ro, rlse = oracle_full(q, k, v, causal, scale)
+    check(o.numpy(), lse.numpy(), ro, rlse, f"{(B, Hq, Hkv, T, d, causal)}")
+
+
+@pytest.mark.parametrize("name", [inputs.SMALL, inputs.TAIL])
+def test_small_workloads_every_element(name):
+    w = inputs.WORKLOADS[name]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = run_gpu(q, k, v, True, w.scale)
+    ro, rlse = oracle_full(q, k, v, True, w.scale)
+    check(o.numpy(), lse.numpy(), ro, rlse, name)
+
+
+LARGE = [n for n in inputs.WORKLOADS if n not in (inputs.SMALL, inputs.TAIL)]
+
+
+def _row_properties(q, k, v, o, lse, scale, G):
+    """Checks that hold for every output row, computed on the GPU in fp32."""
+    dev = torch.device("cuda:0")
+    qf, kf, vf = q.to(dev).float(), k.to(dev).float(), v.to(dev).float()
+    kf = kf.repeat_interleave(G, dim=1)
+    vf = vf.repeat_interleave(G, dim=1)
+    of, lf = o.to(dev), lse.to(dev)
+    assert torch.isfinite(of).all() and torch.isfinite(lf).all()
+    # O is a convex combination of the visible V rows (bf16 rounding slack)
+    lo = torch.cummin(vf, dim=2).values
+    hi = torch.cummax(vf, dim=2).values
+    slack = 1e-2 * torch.maximum(lo.abs(), hi.abs()) + 1e-6
+    assert (of >= lo - slack).all() and (of <= hi + slack).all()
+    # LSE >= the diagonal logit, and >= the mean visible logit (Jensen)
+    diag = scale * (qf * kf).sum(-1)
+    assert (lf >= diag - 1e-3 - 1e-5 * diag.abs()).all()
+    T = q.shape[2]
+    kmean = torch.cumsum(kf.double(), dim=2) / torch.arange(1, T + 1, device=dev,
+                                                            dtype=torch.float64)[:, None]
+    jensen = scale * (qf.double() * kmean).sum(-1)
+    assert (lf.double() >= jensen - 1e-3 - 1e-5 * jensen.abs()).all()
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_large_workloads_sampled_rows(name):
+    w = inputs.WORKLOADS[name]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = run_gpu(q, k, v, True, w.scale)
+    rows = inputs.sample_rows(w.B, w.Hq, w.T, 192, seed=w.seed)
+    ro, rlse = oracle.attn_rows_bf16(inputs.bf16_bits(q), inputs.bf16_bits(k),
+                                     inputs.bf16_bits(v), rows, causal=True, scale=w.scale)
+    b, h, i = rows.T
+    check(o[b, h, i].numpy(), lse[b, h, i].numpy(), ro, rlse, name)
+    _row_properties(q, k, v, o, lse, w.scale, w.G)
+
+
+def test_long_sequence_beyond_the_largest_workload():
+    B, Hq, Hkv, T, d = 1, 2, 1, 32768 + 77, 128
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=99, sigma_qk=2.0)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_gpu(q, k, v, True, scale)
+    rows = inputs.sample_rows(B, Hq, T, 24, seed=5)
+    ro, rlse = oracle.attn_rows_bf16(inputs.bf16_bits(q), inputs.bf16_bits(k),
+                                     inputs.bf16_bits(v), rows, causal=True, scale=scale)
+    b, h, i = rows.T
+    check(o[b, h, i].numpy(), lse[b, h, i].numpy(), ro, rlse, "T=32845")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_causal_row_zero_is_exact(d):
+    B, Hq, Hkv, T = 2, 8, 2, 300
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=3, sigma_qk=4.0)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_gpu(q, k, v, True, scale)
+    vrep = v.float().repeat_interleave(Hq // Hkv, dim=1)
+    assert torch.equal(o[:, :, 0], vrep[:, :, 0])  # p = 1, l = 1: bit exact
+    s00 = scale * (q.double()[:, :, 0] * k.double().repeat_interleave(4, 1)[:, :, 0]).sum(-1)
+    assert torch.allclose(lse[:, :, 0].double(), s00, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_zero_queries_give_prefix_means(causal):
+    B, Hq, Hkv, T, d = 1, 4, 2, 333, 64
+    _, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=4)
+    q = torch.zeros((B, Hq, T, d), dtype=torch.bfloat16)
+    o, lse = run_gpu(q, k, v, causal, 0.125)
+    vd = v.double().repeat_interleave(2, dim=1)
+    n = torch.arange(1, T + 1, dtype=torch.float64)
+    want = torch.cumsum(vd, 2) / n[:, None] if causal else vd.mean(2, keepdim=True).expand_as(vd)
+    want_lse = torch.log(n) if causal else torch.full((T,), math.log(T), dtype=torch.float64)
+    check(o.numpy(), lse.numpy(), want.numpy(), want_lse.expand(B, Hq, T).numpy(), "Q=0")
+
+
+def test_constant_and_unit_values():
+    B, Hq, Hkv, T, d = 2, 4, 1, 260, 128
+    q, k, _ = inputs.make_qkv(B, Hq, Hkv, T, d, seed=6, sigma_qk=3.0)
+    c = torch.linspace(-3, 3, d).to(torch.bfloat16)
+    v = c.expand(B, Hkv, T, d).contiguous()
+    o, _ = run_gpu(q, k, v, True, 1.0 / math.sqrt(d))
+    # P is rounded to bf16, so O = c * (sum of rounded p) / l: within 2^-8 relative
+    assert torch.allclose(o, c.float().expand_as(o), rtol=2 ** -7, atol=1e-6)
+    ones = torch.ones((B, Hkv, T, d), dtype=torch.bfloat16)
+    o1, _ = run_gpu(q, k, ones, True, 1.0 / math.sqrt(d))
+    assert torch.allclose(o1, torch.ones_like(o1), rtol=0, atol=2 ** -7)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (6, 3), (4, 1)])
+def test_gqa_equals_mha_with_repeated_heads(Hq, Hkv):
+    B, T, d = 2, 410, 128
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=8)
+    G = Hq // Hkv
+    o, lse = run_gpu(q, k, v, True, 0.1)
+    om, lsem = run_gpu(q, k.repeat_interleave(G, 1).contiguous(),
+                       v.repeat_interleave(G, 1).contiguous(), True, 0.1)
+    # per-tile arithmetic does not depend on how tiles are paired in a CTA
+    assert torch.equal(o, om) and torch.equal(lse, lsem)
+
+
+def test_outputs_do_not_spill_past_their_buffers():
+    B, Hq, Hkv, T, d = 1, 4, 2, 200, 64
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=9)
+    dev = torch.device("cuda:0")
+    guard = 4096
+    n_o = B * Hq * T * d
+    n_l = B * Hq * T
+    obuf = torch.full((n_o + 2 * guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    lbuf = torch.full((n_l + 2 * guard,), -7.0, dtype=torch.float32, device=dev)
+    o = obuf[guard:guard + n_o].view(B, Hq, T, d)
+    lse = lbuf[guard:guard + n_l].view(B, Hq, T)
+    tess.attn_fwd(q.to(dev), k.to(dev), v.to(dev), out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert tess.tessera_attn_device_error() == 0
+    assert (obuf[:guard] == 7.0).all() and (obuf[guard + n_o:] == 7.0).all()
+    assert (lbuf[:guard] == -7.0).all() and (lbuf[guard + n_l:] == -7.0).all()
+    ro, rlse = oracle_full(q, k, v, True, 1.0 / math.sqrt(d))
+    check(o.float().cpu().numpy(), lse.cpu().numpy(), ro, rlse, "guarded")
+
+
+def test_lse_may_be_omitted_and_results_repeat_bitwise():
+    B, Hq, Hkv, T, d = 1, 8, 2, 700, 128
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=10)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o1, l1 = tess.attn_fwd(qd, kd, vd)
+    o2, l2 = tess.attn_fwd(qd, kd, vd, want_lse=False)
+    assert l2 is None
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o3, l3 = tess.attn_fwd(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert tess.tessera_attn_device_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(o1, o3) and torch.equal(l1, l3)
+
+
+def test_empty_inputs_launch_nothing():
+    dev = torch.device("cuda:0")
+    q = torch.empty((0, 4, 16, 64), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((0, 2, 16, 64), dtype=torch.bfloat16, device=dev)
+    o, lse = tess.attn_fwd(q, k, k)
+    assert o.numel() == 0 and tess.tessera_attn_last_launch_count() == 0
+    q = torch.empty((1, 4, 0, 64), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((1, 2, 0, 64), dtype=torch.bfloat16, device=dev)
+    o, lse = tess.attn_fwd(q, k, k)
+    assert o.numel() == 0 and tess.tessera_attn_last_launch_count() == 0
