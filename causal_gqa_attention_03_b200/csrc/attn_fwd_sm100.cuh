@@ -13,11 +13,12 @@
 // memory feeds both); otherwise they are two consecutive 128-row blocks of one
 // head.  Units are numbered heaviest-first so the causal triangle balances.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax + epilogue for query tile 0 (thread r owns row r)
 //   warps 4-7  softmax + epilogue for query tile 1
 //   warp  8    MMA issue (one lane) and TMEM allocation
 //   warp  9    TMA producer (one lane)
+//   warps 10-11 idle (they complete the third warpgroup for setmaxnreg)
 //
 // Tensor memory (512 columns x 128 lanes, fp32 cells):
 //   S_t = Q_t K_j^T  columns [128 t, 128 t + 128)      (t = 0, 1)
@@ -35,6 +36,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "exp2_fma.cuh"
 #include "sm100_ptx.cuh"
 
 namespace tessera {
@@ -55,6 +57,9 @@ enum WaitCode : uint32_t {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr float kRescaleThreshold = 8.0f;          // log2 units: rescale when the max grows > 2^8
+// Of the 128 exponentials per row and key tile, this many (the last columns)
+// run on the FMA pipe (exp2_fma2) instead of MUFU, in tiles without masking.
+constexpr int kEmuCols = 48;
 
 template <int D>
 struct FwdCfg {
@@ -75,10 +80,16 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int S_COL = 0;
   static constexpr int O_COL = 256;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;             // three warpgroups
+  // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
+  // the MMA/TMA warpgroup gives registers back, the softmax warpgroups take
+  // them: 2 x 128 x 216 + 128 x 56 = 62464 <= 64512.
+  static constexpr int REGS_SOFTMAX = 216;
+  static constexpr int REGS_OTHER = 56;
   static constexpr int MMA_WARP = 8;
   static constexpr int TMA_WARP = 9;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
   static_assert(O_COL + NQ * D <= 512, "tensor memory budget");
 };
 
@@ -111,6 +122,64 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uin
       }
     }
   }
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Online-softmax step for one row (this thread) and one 128-key tile.
+// s: the row's 128 raw scores.  Masked keys (kv0 + c > lim) become -inf when
+// kMasked.  Updates the running (possibly stale) max m in scaled log2 units,
+// sets alpha = 2^(m_old - m_new) (1 when m is kept) and rescale, writes P as
+// bf16 pairs into pk and returns the row sum of the fp32 p.
+template <bool kMasked>
+__device__ __forceinline__ float softmax_row_tile(float (&s)[128], uint32_t (&pk)[2][32], float& m,
+                                                  float& alpha, bool& rescale, float sl2, int kv0,
+                                                  int lim) {
+  if (kMasked) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (kv0 + c > lim) s[c] = -INFINITY;
+  }
+  // row max: eight independent chains of 3-input max
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+  for (int i = 0; i < 60; ++i) mx[i & 7] = max3f(mx[i & 7], s[8 + 2 * i], s[9 + 2 * i]);
+  const float mrow = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]),
+                           fmaxf(mx[6], mx[7]));
+  const float m_tile = mrow * sl2;
+  alpha = 1.f;
+  rescale = m_tile > m + kRescaleThreshold;  // always true on the first tile (m = -inf)
+  if (rescale) {
+    alpha = ptx::ex2(m - m_tile);
+    m = m_tile;
+  }
+  const float neg_m = (m == -INFINITY) ? 0.f : -m;
+  const float2 sl2_2 = make_float2(sl2, sl2);
+  const float2 nm_2 = make_float2(neg_m, neg_m);
+  float2 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2_2, nm_2);
+    float2 pv;
+    if (!kMasked && 2 * c >= 128 - kEmuCols) {
+      pv = exp2_fma2(x);
+    } else {
+      pv.x = ptx::ex2(x.x);
+      pv.y = ptx::ex2(x.y);
+    }
+    acc[c & 3] = __fadd2_rn(acc[c & 3], pv);
+    pk[c >> 5][c & 31] = ptx::pack_bf16x2(pv.x, pv.y);
+  }
+  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return a.x + a.y;
 }
 
 template <int D>
@@ -200,6 +269,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+    // ---- third warpgroup: gives registers back, then TMA and MMA issue ------
+    ptx::setmaxnreg_dec<C::REGS_OTHER>();
   if (warp == C::TMA_WARP) {
     // ======================= TMA producer ===================================
     if (lane == 0) {
@@ -238,6 +310,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, sm_100, 128-B swizzle
       bool ok = wait_bounded(q_full, 0, kErrWaitQ, p.launch_id);
       const uint32_t q_addr = ptx::smem_u32(sQ);
       const uint32_t kv_addr = ptx::smem_u32(sKV);
@@ -257,24 +330,30 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             ok = wait_bounded(&p_full[t], (j - 1) & 1, kErrWaitPFull, p.launch_id);
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t v_base = kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES;
+            // B descriptor low word of the V tile; K step kk is 16 keys = 2 KB further
+            const uint32_t vb_lo =
+                ptx::sdesc_sw128_lo(kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES, C::SUB_BYTES);
+            const uint32_t pa = tmem + C::S_COL + 128 * t;
+            ptx::mma_ts_lohi_rt(tmem + C::O_COL + D * t, pa, vb_lo, kDescHi, kIdescO,
+                                j > 1 ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < C::BN / 16; ++kk) {
-              const uint64_t bdesc = ptx::sdesc_sw128(v_base + kk * 16 * 128, C::SUB_BYTES, 1024);
-              ptx::mma_ts(tmem + C::O_COL + D * t, tmem + C::S_COL + 128 * t + kk * 8, bdesc,
-                          kIdescO, (j > 1 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 1; kk < C::BN / 16; ++kk)
+              ptx::mma_ts_lohi<1>(tmem + C::O_COL + D * t, pa + kk * 8, vb_lo + kk * (2048 >> 4),
+                                  kDescHi, kIdescO);
             if (j == ntile[t]) ptx::tc_commit(&o_full[t]);
           }
           if (j < ntile[t]) {
             // S_t = Q_t K_j^T; both operands K-major in smem
-            const uint32_t qa = q_addr + t * C::TILE_BYTES;
-            const uint32_t kb = kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES;
+            // A and B descriptor low words; K step kk: +32 B, or the next 16 KB sub-tile
+            const uint32_t qa_lo = ptx::sdesc_sw128_lo(q_addr + t * C::TILE_BYTES, 16);
+            const uint32_t kb_lo =
+                ptx::sdesc_sw128_lo(kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES, 16);
+            const uint32_t sd = tmem + C::S_COL + 128 * t;
+            ptx::mma_ss_lohi<0>(sd, qa_lo, kDescHi, kb_lo, kDescHi, kIdescS);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
-              ptx::mma_ss(tmem + C::S_COL + 128 * t, ptx::sdesc_sw128(qa + off, 16, 1024),
-                          ptx::sdesc_sw128(kb + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+            for (int kk = 1; kk < D / 16; ++kk) {
+              const uint32_t step = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
+              ptx::mma_ss_lohi<1>(sd, qa_lo + step, kDescHi, kb_lo + step, kDescHi, kIdescS);
             }
             ptx::tc_commit(&s_full[t]);
           }
@@ -288,7 +367,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       wait_bounded(drain, 0, kErrWaitDrain, p.launch_id);
     }
     __syncwarp();
+  }
   } else {
+    ptx::setmaxnreg_inc<C::REGS_SOFTMAX>();
     // ======================= softmax + epilogue =============================
     const int t = warp >> 2;
     const int quad = warp & 3;
@@ -317,36 +398,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::reg_fence(sr[c]);
 
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
         const int kv0 = j * C::BN;
         const bool edge = p.causal ? (kv0 + C::BN - 1 > q_row - row) : (kv0 + C::BN > p.T);
-        if (edge) {
-          const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (kv0 + c > lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
-        const float m_tile = mx * sl2;
-        float alpha = 1.f;
-        const bool rescale = m_tile > m + kRescaleThreshold;
-        if (rescale) {
-          alpha = ptx::ex2(m - m_tile);  // 0 on the first tile (m = -inf)
-          m = m_tile;
-        }
-        const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        float rowsum = 0.f;
+        const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
+        float alpha;
+        bool rescale;
         uint32_t pk[2][32];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x0 = __uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]);
-          const float x1 = __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
-          const float p0 = ptx::ex2(fmaf(x0, sl2, neg_m));
-          const float p1 = ptx::ex2(fmaf(x1, sl2, neg_m));
-          rowsum += p0 + p1;
-          pk[c >> 5][c & 31] = ptx::pack_bf16x2(p0, p1);
-        }
+        const float rowsum =
+            edge ? softmax_row_tile<true>(sv, pk, m, alpha, rescale, sl2, kv0, lim)
+                 : softmax_row_tile<false>(sv, pk, m, alpha, rescale, sl2, kv0, lim);
         l = l * alpha + rowsum;
         ptx::tmem_st32(s_addr + 0, pk[0]);
         ptx::tmem_st32(s_addr + 32, pk[1]);
