@@ -59,7 +59,11 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitima
 constexpr float kRescaleThreshold = 8.0f;          // log2 units: rescale when the max grows > 2^8
 // Of the 128 exponentials per row and key tile, this many (the last columns)
 // run on the FMA pipe (exp2_fma2) instead of MUFU, in tiles without masking.
-constexpr int kEmuCols = 48;
+// Measured on B200 at the 1 kW power cap: 0 is fastest for long sequences
+// (each emulated exp costs ~8 FMA-pipe instructions, which lowers the
+// power-capped clock more than the MUFU work it saves), 32 is marginally
+// faster for T = 4096.
+constexpr int kEmuCols = 0;
 
 template <int D>
 struct FwdCfg {
