@@ -70,14 +70,17 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   using C = FwdCfg<D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TESSERA_ERR_CUDA;
-  static std::atomic<bool> attr_set[64];
+  static std::atomic<int> sm_count[64];
   if (dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
-  if (!attr_set[dev].load(std::memory_order_acquire)) {
+  int sms = sm_count[dev].load(std::memory_order_acquire);
+  if (sms == 0) {
     if (cudaFuncSetAttribute(tessera::attn_fwd_sm100_kernel<D>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
+                             C::SMEM_BYTES) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
       return TESSERA_ERR_CUDA;
-    attr_set[dev].store(true, std::memory_order_release);
+    sm_count[dev].store(sms, std::memory_order_release);
   }
 
   CUtensorMap tm_q, tm_k, tm_v;
@@ -104,12 +107,15 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     units = static_cast<long long>(p.units_per_step) * ((p.nqb + 1) / 2);
   }
   if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  p.num_units = static_cast<int>(units);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
 
-  tessera::attn_fwd_sm100_kernel<D>
-      <<<static_cast<unsigned>(units), C::THREADS, C::SMEM_BYTES, stream>>>(tm_q, tm_k, tm_v, p);
+  // persistent: one CTA per SM, each walking its share of the units
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+  tessera::attn_fwd_sm100_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tm_q, tm_k, tm_v,
+                                                                                p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = 1;
   return TESSERA_OK;

@@ -5,19 +5,20 @@
 // Tessera review, "The kernel set and its torch fallback"; Tessera README,
 // "What's in it" / "Kernels").  The tile design below is this library's own,
 // built for sm_100a: TMA + mbarrier pipeline, tcgen05 MMAs accumulating in
-// tensor memory, warp-specialised roles.
+// tensor memory, warp-specialised roles, persistent CTAs.
 //
-// One CTA processes one work unit: two 128-row query tiles that read the same
-// key/value head.  When the group size G is even the two tiles are two query
-// heads of one group at the same rows (so each K/V tile fetched into shared
-// memory feeds both); otherwise they are two consecutive 128-row blocks of one
-// head.  Units are numbered heaviest-first so the causal triangle balances.
+// Work unit: two 128-row query tiles that read the same key/value head.  When
+// the group size G is even the two tiles are two query heads of one group at
+// the same rows (so each K/V tile fetched into shared memory feeds both);
+// otherwise they are two consecutive 128-row blocks of one head.  Units are
+// numbered heaviest-first (longest causal extent) and dealt to one CTA per SM
+// in snake order, so the causal triangle balances.
 //
 // Warp roles (384 threads, three warpgroups):
-//   warps 0-3  softmax + epilogue for query tile 0 (thread r owns row r)
-//   warps 4-7  softmax + epilogue for query tile 1
-//   warp  8    MMA issue (one lane) and TMEM allocation
-//   warp  9    TMA producer (one lane)
+//   warps 0-3   softmax + epilogue for query tile 0 (thread r owns row r)
+//   warps 4-7   softmax + epilogue for query tile 1
+//   warp  8     MMA issue (one lane) and TMEM allocation
+//   warp  9     TMA producer (one lane)
 //   warps 10-11 idle (they complete the third warpgroup for setmaxnreg)
 //
 // Tensor memory (512 columns x 128 lanes, fp32 cells):
@@ -28,7 +29,10 @@
 // Per key tile j and query tile t the MMA warp issues PV_t(j-1) then S_t(j);
 // tcgen05 MMAs from one thread execute in order, so S_t(j) cannot overwrite
 // P_t(j-1) before PV_t(j-1) has read it.  The softmax of tile t overlaps the
-// MMAs of the other tile.  The running max is rescaled lazily: O and l keep a
+// MMAs of the other tile.  Across units the same order holds: a unit's first
+// S_t follows the previous unit's last PV_t, and its first PV_t (which
+// overwrites O_t) waits for P_t, which the softmax writes only after its
+// epilogue has read O_t.  The running max is rescaled lazily: O and l keep a
 // stale max until the row max grows by more than 2^8, which is exact because
 // both carry the same max.
 #pragma once
@@ -53,6 +57,7 @@ enum WaitCode : uint32_t {
   kErrWaitPFull = 5,
   kErrWaitOFull = 6,
   kErrWaitDrain = 7,
+  kErrWaitQEmpty = 8,
 };
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
@@ -70,7 +75,7 @@ struct FwdCfg {
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
   static constexpr int BM = 128;                  // query rows per tile
   static constexpr int BN = 128;                  // keys per tile
-  static constexpr int NQ = 2;                    // query tiles per CTA
+  static constexpr int NQ = 2;                    // query tiles per unit
   static constexpr int SUB = D / 64;              // 128-byte-wide column sub-tiles per tile
   static constexpr int SUB_BYTES = 128 * 128;     // one [128 rows x 64 bf16] sub-tile
   static constexpr int TILE_BYTES = 128 * D * 2;  // one [128 x D] bf16 tile
@@ -78,23 +83,25 @@ struct FwdCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = NQ * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
-  static constexpr int NBAR = 1 + 2 * NSTAGE + 3 * NQ + 1;
+  // q_full, q_empty, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[NQ], p_full[NQ],
+  // o_full[NQ], drain
+  static constexpr int NBAR = 2 + 2 * NSTAGE + 3 * NQ + 1;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int S_COL = 0;
   static constexpr int O_COL = 256;
   static constexpr int THREADS = 384;             // three warpgroups
-  // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
-  // the MMA/TMA warpgroup gives registers back, the softmax warpgroups take
-  // them: 2 x 128 x 216 + 128 x 56 = 62464 <= 64512.
-  static constexpr int REGS_SOFTMAX = 216;
-  static constexpr int REGS_OTHER = 56;
   static constexpr int MMA_WARP = 8;
   static constexpr int TMA_WARP = 9;
+  // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
+  // the MMA/TMA warpgroup gives registers back, the softmax warpgroups take
+  // them: 2 x 128 x 200 + 128 x 96 = 63488 <= 64512.
+  static constexpr int REGS_SOFTMAX = 200;
+  static constexpr int REGS_OTHER = 96;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
   static_assert(O_COL + NQ * D <= 512, "tensor memory budget");
+  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
 };
 
 struct FwdParams {
@@ -104,10 +111,56 @@ struct FwdParams {
   int nqb;                   // ceil(T / 128)
   int pair_heads;            // 1: tiles are heads (2p, 2p+1) of a group; 0: q-blocks (2p, 2p+1)
   int units_per_step;        // units sharing one position in the heaviest-first order
+  int num_units;
   __nv_bfloat16* o;
   float* lse;
   unsigned long long launch_id;
 };
+
+// A work unit: batch b, key/value head g, the two tiles' query heads and
+// 128-row blocks, and how many key tiles each visits (0: tile absent).
+struct Unit {
+  int b, g;
+  int head[2], qblk[2], ntile[2];
+  int nmax;
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  Unit w;
+  const int step = u / p.units_per_step;
+  const int r = u % p.units_per_step;
+  if (p.pair_heads) {
+    const int half = p.G >> 1;
+    const int hp = r % half;
+    const int bg = r / half;
+    w.b = bg / p.Hkv;
+    w.g = bg % p.Hkv;
+    w.head[0] = w.g * p.G + 2 * hp;
+    w.head[1] = w.head[0] + 1;
+    w.qblk[0] = w.qblk[1] = p.nqb - 1 - step;
+  } else {
+    const int npairs = (p.nqb + 1) >> 1;
+    const int pr = npairs - 1 - step;
+    w.b = r / p.Hq;
+    w.head[0] = w.head[1] = r % p.Hq;
+    w.g = w.head[0] / p.G;
+    w.qblk[0] = 2 * pr;
+    w.qblk[1] = 2 * pr + 1;
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    w.ntile[t] = (w.qblk[t] >= p.nqb) ? 0 : (p.causal ? min(w.qblk[t] + 1, p.nqb) : p.nqb);
+  w.nmax = max(w.ntile[0], w.ntile[1]);
+  return w;
+}
+
+// The k-th unit of this CTA (snake order over the heaviest-first list), or -1.
+__device__ __forceinline__ int unit_of(const FwdParams& p, int k) {
+  const int c = (k & 1) ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
+                        : static_cast<int>(blockIdx.x);
+  const long long u = static_cast<long long>(k) * gridDim.x + c;
+  return u < p.num_units ? static_cast<int>(u) : -1;
+}
 
 // Wait for the phase of `parity` on `bar`, giving up after kWaitLimitNs or as
 // soon as another CTA of the same launch has given up.  Returns false on give-up.
@@ -126,6 +179,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uin
       }
     }
   }
+}
+
+// All lanes wait; the warp proceeds only if every lane saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t code,
+                                          unsigned long long launch_id) {
+  return __all_sync(0xffffffffu, wait_bounded(bar, parity, code, launch_id));
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -200,7 +259,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint8_t* sKV = smem + C::KV_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + C::NSTAGE;
   uint64_t* s_full = kv_empty + C::NSTAGE;
   uint64_t* p_full = s_full + C::NQ;
@@ -211,42 +271,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- decode the work unit (heaviest first) --------------------------------
-  const int u = blockIdx.x;
-  const int step = u / p.units_per_step;
-  const int r = u % p.units_per_step;
-  int b, g, head[2], qblk[2];
-  if (p.pair_heads) {
-    const int half = p.G >> 1;
-    const int hp = r % half;
-    const int bg = r / half;
-    b = bg / p.Hkv;
-    g = bg % p.Hkv;
-    head[0] = g * p.G + 2 * hp;
-    head[1] = head[0] + 1;
-    qblk[0] = qblk[1] = p.nqb - 1 - step;
-  } else {
-    const int npairs = (p.nqb + 1) >> 1;
-    const int pr = npairs - 1 - step;
-    b = r / p.Hq;
-    head[0] = head[1] = r % p.Hq;
-    g = head[0] / p.G;
-    qblk[0] = 2 * pr;
-    qblk[1] = 2 * pr + 1;
-  }
-  const int nkv = p.nqb;
-  int ntile[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const bool valid = qblk[t] < p.nqb;
-    ntile[t] = !valid ? 0 : (p.causal ? min(qblk[t] + 1, nkv) : nkv);
-  }
-  const int nmax = max(ntile[0], ntile[1]);
-  const int kv_plane = b * p.Hkv + g;
-
   // ---- set-up ---------------------------------------------------------------
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
+    ptx::mbar_init(q_empty, 1);
     for (int s = 0; s < C::NSTAGE; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
@@ -276,124 +304,170 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (warp >= 8) {
     // ---- third warpgroup: gives registers back, then TMA and MMA issue ------
     ptx::setmaxnreg_dec<C::REGS_OTHER>();
-  if (warp == C::TMA_WARP) {
-    // ======================= TMA producer ===================================
-    if (lane == 0) {
-      const int nvalid = (ntile[0] > 0) + (ntile[1] > 0);
-      ptx::mbar_arrive_expect_tx(q_full, nvalid * C::TILE_BYTES);
-      for (int t = 0; t < C::NQ; ++t) {
-        if (ntile[t] == 0) continue;
-        for (int c = 0; c < C::SUB; ++c)
-          ptx::tma_load_3d(sQ + t * C::TILE_BYTES + c * C::SUB_BYTES, &tm_q, q_full, c * 64,
-                           qblk[t] * C::BM, b * p.Hq + head[t]);
+    if (warp == C::TMA_WARP) {
+      // ======================= TMA producer =================================
+      // Per unit: Q tiles (once the previous unit's S products are done with
+      // the Q buffer), then K_0, V_0, K_1, V_1, ... into the ring.
+      if (lane == 0) {
+        // K/V tiles are re-read by the other units of the same key/value head:
+        // keep them in L2; Q is read once.
+        const uint64_t keep = ptx::policy_evict_last();
+        const uint64_t once = ptx::policy_evict_first();
+        int idx = 0;  // K/V tiles loaded so far (ring position)
+        int k = 0;
+        bool ok = true;
+        for (; ok; ++k) {
+          const int u = unit_of(p, k);
+          if (u < 0) break;
+          const Unit w = decode_unit(p, u);
+          // Q of this unit, once the previous unit's S products no longer
+          // read the Q buffer.
+          auto load_q = [&]() -> bool {
+            if (!wait_bounded(q_empty, (k & 1) ^ 1u, kErrWaitQEmpty, p.launch_id)) return false;
+            ptx::mbar_arrive_expect_tx(q_full,
+                                       ((w.ntile[0] > 0) + (w.ntile[1] > 0)) * C::TILE_BYTES);
+            for (int t = 0; t < C::NQ; ++t) {
+              if (w.ntile[t] == 0) continue;
+              for (int c = 0; c < C::SUB; ++c)
+                ptx::tma_load_3d_hint(sQ + t * C::TILE_BYTES + c * C::SUB_BYTES, &tm_q, q_full,
+                                      c * 64, w.qblk[t] * C::BM, w.b * p.Hq + w.head[t], once);
+            }
+            return true;
+          };
+          const int kv_plane = w.b * p.Hkv + w.g;
+          // K_0 and V_0 go first: they do not depend on the Q buffer
+          const int q_at = min(2, 2 * w.nmax);
+          for (int i = 0; i < 2 * w.nmax; ++i, ++idx) {  // K_0, V_0, K_1, V_1, ...
+            if (i == q_at && !load_q()) {
+              ok = false;
+              break;
+            }
+            const int s = idx % C::NSTAGE;
+            if (!wait_bounded(&kv_empty[s], ((idx / C::NSTAGE) & 1) ^ 1u, kErrWaitKvEmpty,
+                              p.launch_id)) {
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+            const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+            for (int c = 0; c < C::SUB; ++c)
+              ptx::tma_load_3d_hint(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s],
+                                    c * 64, (i >> 1) * C::BN, kv_plane, keep);
+          }
+          if (ok && q_at == 2 * w.nmax && !load_q()) ok = false;
+        }
+        if (!ok) {
+          // Gave up: let the copies already in flight land before the CTA exits.
+          if (k > 0) wait_bounded(q_full, (k - 1) & 1, kErrWaitQ, p.launch_id);
+          for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
+            wait_bounded(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrWaitKvFull,
+                         p.launch_id);
+        }
       }
-      int issued = 0;
-      for (int idx = 0; idx < 2 * nmax; ++idx) {  // K_0, V_0, K_1, V_1, ...
-        const int s = idx % C::NSTAGE;
-        const uint32_t ph = (idx / C::NSTAGE) & 1;
-        if (!wait_bounded(&kv_empty[s], ph ^ 1u, kErrWaitKvEmpty, p.launch_id)) break;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
-        const CUtensorMap* map = (idx & 1) ? &tm_v : &tm_k;
-        const int j = idx >> 1;
-        for (int c = 0; c < C::SUB; ++c)
-          ptx::tma_load_3d(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s], c * 64,
-                           j * C::BN, kv_plane);
-        ++issued;
-      }
-      if (issued < 2 * nmax) {
-        // Gave up: let the copies already in flight land before the CTA exits.
-        wait_bounded(q_full, 0, kErrWaitQ, p.launch_id);
-        for (int idx = max(0, issued - C::NSTAGE); idx < issued; ++idx)
-          wait_bounded(&kv_full[idx % C::NSTAGE], (idx / C::NSTAGE) & 1, kErrWaitKvFull,
-                       p.launch_id);
-      }
-    }
-    __syncwarp();
-  } else if (warp == C::MMA_WARP) {
-    // ======================= MMA issue ======================================
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
-      constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, sm_100, 128-B swizzle
-      bool ok = wait_bounded(q_full, 0, kErrWaitQ, p.launch_id);
-      const uint32_t q_addr = ptx::smem_u32(sQ);
-      const uint32_t kv_addr = ptx::smem_u32(sKV);
-      for (int j = 0; ok && j <= nmax; ++j) {
-        const int kidx = 2 * j, vidx = 2 * j - 1;
-        if (j < nmax)
-          ok = wait_bounded(&kv_full[kidx % C::NSTAGE], (kidx / C::NSTAGE) & 1, kErrWaitKvFull,
-                            p.launch_id);
-        if (ok && j > 0)
-          ok = wait_bounded(&kv_full[vidx % C::NSTAGE], (vidx / C::NSTAGE) & 1, kErrWaitKvFull,
-                            p.launch_id);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        for (int t = 0; t < C::NQ && ok; ++t) {
-          if (j >= 1 && j <= ntile[t]) {
-            // O_t += P_t(j-1) V_{j-1}; A = P from TMEM, B = V (MN-major in smem)
-            ok = wait_bounded(&p_full[t], (j - 1) & 1, kErrWaitPFull, p.launch_id);
+      __syncwarp();
+    } else if (warp == C::MMA_WARP) {
+      // ======================= MMA issue ====================================
+      if (lane == 0) {
+        constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
+        constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-B swizzle
+        const uint32_t q_addr = ptx::smem_u32(sQ);
+        const uint32_t kv_addr = ptx::smem_u32(sKV);
+        int base = 0;           // ring position of the unit's K_0
+        int pcnt[2] = {0, 0};   // P tiles consumed per query tile (p_full phases)
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int u = unit_of(p, k);
+          if (u < 0) break;
+          const Unit w = decode_unit(p, u);
+          if (!wait_bounded(q_full, k & 1, kErrWaitQ, p.launch_id)) break;
+          for (int j = 0; ok && j <= w.nmax; ++j) {
+            const int kidx = base + 2 * j, vidx = base + 2 * j - 1;
+            if (j < w.nmax)
+              ok = wait_bounded(&kv_full[kidx % C::NSTAGE], (kidx / C::NSTAGE) & 1,
+                                kErrWaitKvFull, p.launch_id);
+            if (ok && j > 0)
+              ok = wait_bounded(&kv_full[vidx % C::NSTAGE], (vidx / C::NSTAGE) & 1,
+                                kErrWaitKvFull, p.launch_id);
             if (!ok) break;
             ptx::tc_fence_after();
-            // B descriptor low word of the V tile; K step kk is 16 keys = 2 KB further
-            const uint32_t vb_lo =
-                ptx::sdesc_sw128_lo(kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES, C::SUB_BYTES);
-            const uint32_t pa = tmem + C::S_COL + 128 * t;
-            ptx::mma_ts_lohi_rt(tmem + C::O_COL + D * t, pa, vb_lo, kDescHi, kIdescO,
-                                j > 1 ? 1u : 0u);
+            for (int t = 0; t < C::NQ && ok; ++t) {
+              if (j >= 1 && j <= w.ntile[t]) {
+                // O_t += P_t(j-1) V_{j-1}; A = P from TMEM, B = V (MN-major in smem)
+                ok = wait_bounded(&p_full[t], pcnt[t] & 1, kErrWaitPFull, p.launch_id);
+                if (!ok) break;
+                ++pcnt[t];
+                ptx::tc_fence_after();
+                // B descriptor low word of the V tile; K step kk is 16 keys = 2 KB further
+                const uint32_t vb_lo =
+                    ptx::sdesc_sw128_lo(kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES, C::SUB_BYTES);
+                const uint32_t pa = tmem + C::S_COL + 128 * t;
+                ptx::mma_ts_lohi_rt(tmem + C::O_COL + D * t, pa, vb_lo, kDescHi, kIdescO,
+                                    j > 1 ? 1u : 0u);
 #pragma unroll
-            for (int kk = 1; kk < C::BN / 16; ++kk)
-              ptx::mma_ts_lohi<1>(tmem + C::O_COL + D * t, pa + kk * 8, vb_lo + kk * (2048 >> 4),
-                                  kDescHi, kIdescO);
-            if (j == ntile[t]) ptx::tc_commit(&o_full[t]);
-          }
-          if (j < ntile[t]) {
-            // S_t = Q_t K_j^T; both operands K-major in smem
-            // A and B descriptor low words; K step kk: +32 B, or the next 16 KB sub-tile
-            const uint32_t qa_lo = ptx::sdesc_sw128_lo(q_addr + t * C::TILE_BYTES, 16);
-            const uint32_t kb_lo =
-                ptx::sdesc_sw128_lo(kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES, 16);
-            const uint32_t sd = tmem + C::S_COL + 128 * t;
-            ptx::mma_ss_lohi<0>(sd, qa_lo, kDescHi, kb_lo, kDescHi, kIdescS);
+                for (int kk = 1; kk < C::BN / 16; ++kk)
+                  ptx::mma_ts_lohi<1>(tmem + C::O_COL + D * t, pa + kk * 8,
+                                      vb_lo + kk * (2048 >> 4), kDescHi, kIdescO);
+                if (j == w.ntile[t]) ptx::tc_commit(&o_full[t]);
+              }
+              if (j < w.ntile[t]) {
+                // S_t = Q_t K_j^T; both operands K-major in smem.  A and B
+                // descriptor low words; K step kk: +32 B, or the next 16 KB sub-tile
+                const uint32_t qa_lo = ptx::sdesc_sw128_lo(q_addr + t * C::TILE_BYTES, 16);
+                const uint32_t kb_lo =
+                    ptx::sdesc_sw128_lo(kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES, 16);
+                const uint32_t sd = tmem + C::S_COL + 128 * t;
+                ptx::mma_ss_lohi<0>(sd, qa_lo, kDescHi, kb_lo, kDescHi, kIdescS);
 #pragma unroll
-            for (int kk = 1; kk < D / 16; ++kk) {
-              const uint32_t step = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
-              ptx::mma_ss_lohi<1>(sd, qa_lo + step, kDescHi, kb_lo + step, kDescHi, kIdescS);
+                for (int kk = 1; kk < D / 16; ++kk) {
+                  const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
+                  ptx::mma_ss_lohi<1>(sd, qa_lo + st, kDescHi, kb_lo + st, kDescHi, kIdescS);
+                }
+                ptx::tc_commit(&s_full[t]);
+              }
             }
-            ptx::tc_commit(&s_full[t]);
+            if (!ok) break;
+            if (j < w.nmax) ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);
+            if (j > 0) ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);
+            // the unit's last S products: the Q buffer is free once they complete
+            if (j == w.nmax - 1) ptx::tc_commit(q_empty);
           }
+          base += 2 * w.nmax;
         }
-        if (!ok) break;
-        if (j < nmax) ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);
-        if (j > 0) ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);
+        // Every MMA issued must finish before tensor memory is released.
+        ptx::tc_commit(drain);
+        wait_bounded(drain, 0, kErrWaitDrain, p.launch_id);
       }
-      // Every MMA issued must finish before tensor memory is released.
-      ptx::tc_commit(drain);
-      wait_bounded(drain, 0, kErrWaitDrain, p.launch_id);
+      __syncwarp();
     }
-    __syncwarp();
-  }
   } else {
     ptx::setmaxnreg_inc<C::REGS_SOFTMAX>();
     // ======================= softmax + epilogue =============================
     const int t = warp >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int n_t = ntile[t];
-    if (n_t > 0) {
-      const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + C::S_COL + 128 * t;
-      const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
-      const int q_row = qblk[t] * C::BM + row;
-      const float sl2 = p.scale_log2;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + C::S_COL + 128 * t;
+    const uint32_t o_addr = tmem + lane_base + C::O_COL + D * t;
+    const float sl2 = p.scale_log2;
+    int scnt = 0;  // S tiles of this query tile seen so far (s_full phases)
+    int ocnt = 0;  // units of this query tile finished so far (o_full phases)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_of(p, k);
+      if (u < 0) break;
+      const Unit w = decode_unit(p, u);
+      const int n_t = w.ntile[t];
+      if (n_t == 0) continue;
+      const int q_row = w.qblk[t] * C::BM + row;
       float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale)
       float l = 0.f;        // running sum of 2^(x - m)
-      bool ok = true;
       for (int j = 0; j < n_t; ++j) {
-        // every lane polls; the warp proceeds only if all saw the phase complete
-        if (!__all_sync(0xffffffffu, wait_bounded(&s_full[t], j & 1, kErrWaitSFull, p.launch_id))) {
+        if (!warp_wait(&s_full[t], scnt & 1, kErrWaitSFull, p.launch_id)) {
           ok = false;
           break;
         }
+        ++scnt;
         ptx::tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
@@ -401,7 +475,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         ptx::tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::reg_fence(sr[c]);
-
         float sv[128];
 #pragma unroll
         for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
@@ -435,36 +508,40 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&p_full[t]);
       }
+      if (!ok) break;
 
-      // ---- epilogue: O / l -> bf16, LSE ---------------------------------------
-      if (ok) ok = wait_bounded(&o_full[t], 0, kErrWaitOFull, p.launch_id);
-      if (__all_sync(0xffffffffu, ok)) {
-        ptx::tc_fence_after();
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        const bool store = q_row < p.T;
-        const int64_t orow = (static_cast<int64_t>(b) * p.Hq + head[t]) * p.T + q_row;
-        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+      // ---- epilogue: O / l -> bf16, LSE -----------------------------------------
+      if (!warp_wait(&o_full[t], ocnt & 1, kErrWaitOFull, p.launch_id)) break;
+      ++ocnt;
+      ptx::tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const bool store = q_row < p.T;
+      const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + w.head[t]) * p.T + q_row;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(o_addr + 32 * c, ov);
-          ptx::tmem_ld_wait();
-          ptx::reg_fence(ov);
-          uint32_t packed[16];
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(o_addr + 32 * c, ov);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(ov);
+        uint32_t packed[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = ptx::pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
-                                         __uint_as_float(ov[2 * i + 1]) * inv_l);
-          if (store) {
+        for (int i = 0; i < 16; ++i)
+          packed[i] = ptx::pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
+                                       __uint_as_float(ov[2 * i + 1]) * inv_l);
+        if (store) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[c * 4 + v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2],
-                                           packed[4 * v4 + 3]);
-          }
+          for (int v4 = 0; v4 < 4; ++v4)
+            ptx::st_global_cs_v4(dst + c * 4 + v4,
+                                 make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2],
+                                            packed[4 * v4 + 3]));
         }
-        if (store && p.lse != nullptr)
-          p.lse[orow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
       }
+      if (store && p.lse != nullptr)
+        p.lse[orow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
+      // O_t has been read; the next unit's first P_t arrival (after this
+      // fence) is what lets the MMA warp overwrite it.
+      ptx::tc_fence_before();
     }
   }
 
