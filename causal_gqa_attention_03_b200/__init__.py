@@ -22,7 +22,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_
 
 # Symbols declared in include/tessera_attn.h.
 EXPORTED = ("tessera_attn_fwd", "tessera_attn_device_error", "tessera_status_str",
-            "tessera_attn_last_launch_count")
+            "tessera_attn_last_launch_count", "tessera_attn_selftest_timeout")
+
+# Device error code recorded by tessera_attn_selftest_timeout.
+DEVICE_ERR_SELFTEST = 9
 
 STATUS = {0: "TESSERA_OK", 1: "TESSERA_ERR_INVALID_ARG", 2: "TESSERA_ERR_UNSUPPORTED",
           3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT"}
@@ -58,6 +61,8 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_status_str.restype = ctypes.c_char_p
             lib.tessera_attn_last_launch_count.argtypes = []
             lib.tessera_attn_last_launch_count.restype = ci
+            lib.tessera_attn_selftest_timeout.argtypes = [ctypes.c_uint, vp]
+            lib.tessera_attn_selftest_timeout.restype = ci
             _lib = lib
     return _lib
 
@@ -85,6 +90,11 @@ def tessera_status_str(status: int) -> str:
 
 def tessera_attn_last_launch_count() -> int:
     return load_library().tessera_attn_last_launch_count()
+
+
+def tessera_attn_selftest_timeout(limit_us: int, stream: int | None = None) -> int:
+    """Queue the bounded-wait diagnostic (see include/tessera_attn.h); returns the status."""
+    return load_library().tessera_attn_selftest_timeout(int(limit_us), stream or None)
 
 
 def attn_fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=None,

@@ -164,6 +164,15 @@ extern "C" int tessera_attn_device_error(int* code) {
   return TESSERA_OK;
 }
 
+extern "C" int tessera_attn_selftest_timeout(unsigned int limit_us, tessera_stream_t stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return TESSERA_ERR_INVALID_ARG;
+  const unsigned long long id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+  tessera::attn_selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      id, static_cast<uint64_t>(limit_us) * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  return TESSERA_OK;
+}
+
 extern "C" const char* tessera_status_str(int status) {
   switch (status) {
     case TESSERA_OK: return "ok";

@@ -58,6 +58,7 @@ enum WaitCode : uint32_t {
   kErrWaitOFull = 6,
   kErrWaitDrain = 7,
   kErrWaitQEmpty = 8,
+  kErrSelfTest = 9,  // the deliberate timeout of attn_selftest_timeout_kernel
 };
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
@@ -162,10 +163,11 @@ __device__ __forceinline__ int unit_of(const FwdParams& p, int k) {
   return u < p.num_units ? static_cast<int>(u) : -1;
 }
 
-// Wait for the phase of `parity` on `bar`, giving up after kWaitLimitNs or as
+// Wait for the phase of `parity` on `bar`, giving up after limit_ns or as
 // soon as another CTA of the same launch has given up.  Returns false on give-up.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t code,
-                                             unsigned long long launch_id) {
+                                             unsigned long long launch_id,
+                                             uint64_t limit_ns = kWaitLimitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -173,12 +175,28 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uin
     if ((it & 1023u) == 0) {
       const unsigned long long w = *reinterpret_cast<volatile unsigned long long*>(&g_tessera_err);
       if ((w >> 32) == (launch_id & 0xffffffffull) && (w & 0xffffffffull) != 0) return false;
-      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (ptx::globaltimer_ns() - t0 > limit_ns) {
         atomicExch(&g_tessera_err, ((launch_id & 0xffffffffull) << 32) | code);
         return false;
       }
     }
   }
+}
+
+// Diagnostic: one warp waits, through wait_bounded, on an mbarrier that
+// nothing arrives at, so the wait gives up after limit_ns and records
+// kErrSelfTest in the error word.  It exercises the path every wait of the
+// attention kernel takes when it gives up, without faulting or hanging.
+__global__ void __launch_bounds__(32, 1)
+    attn_selftest_timeout_kernel(unsigned long long launch_id, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) wait_bounded(&bar, 0, kErrSelfTest, launch_id, limit_ns);
+  __syncwarp();
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete.

@@ -78,6 +78,18 @@ int tessera_attn_fwd(const void *q, const void *k, const void *v, void *o,
  */
 int tessera_attn_device_error(int *code);
 
+/*
+ * Diagnostic of the bounded-wait machinery: queues on `stream` one warp that
+ * waits, with the same bounded wait the attention kernel uses, on a barrier
+ * that nothing completes.  The wait gives up after limit_us microseconds
+ * (1 .. 10,000,000, else TESSERA_ERR_INVALID_ARG) and records code
+ * TESSERA_DEVICE_ERR_SELFTEST in the device error word, which
+ * tessera_attn_device_error() then returns.  Nothing faults or hangs and the
+ * CUDA context stays usable.  Returns TESSERA_OK once queued.
+ */
+#define TESSERA_DEVICE_ERR_SELFTEST 9
+int tessera_attn_selftest_timeout(unsigned int limit_us, tessera_stream_t stream);
+
 /* A static string naming a tessera_status value. */
 const char *tessera_status_str(int status);
 

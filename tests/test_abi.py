@@ -80,6 +80,11 @@ def test_argument_checks_before_any_cuda_call(lib, kw, status):
         assert tess.tessera_attn_last_launch_count() == 0
 
 
+@pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
+def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
+    assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1
+
+
 def test_status_strings(lib):
     for s in range(6):
         assert tess.tessera_status_str(s)

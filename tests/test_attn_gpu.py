@@ -236,3 +236,21 @@ def test_empty_inputs_launch_nothing():
     k = torch.empty((1, 2, 0, 64), dtype=torch.bfloat16, device=dev)
     o, lse = tess.attn_fwd(q, k, k)
     assert o.numel() == 0 and tess.tessera_attn_last_launch_count() == 0
+
+
+def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
+    import time
+    assert tess.tessera_attn_device_error() == 0
+    stream = torch.cuda.current_stream().cuda_stream
+    assert tess.tessera_attn_selftest_timeout(50_000, stream) == 0  # 50 ms limit
+    t0 = time.time()
+    code = tess.tessera_attn_device_error()
+    assert code == tess.DEVICE_ERR_SELFTEST
+    assert time.time() - t0 < 5.0
+    assert tess.tessera_attn_device_error() == 0  # read clears the word
+    # the context still works: a normal call afterwards is correct
+    B, Hq, Hkv, T, d = 1, 4, 2, 200, 128
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=11)
+    o, lse = run_gpu(q, k, v, True, 1.0 / math.sqrt(d))
+    ro, rlse = oracle_full(q, k, v, True, 1.0 / math.sqrt(d))
+    check(o.numpy(), lse.numpy(), ro, rlse, "after self-test")
