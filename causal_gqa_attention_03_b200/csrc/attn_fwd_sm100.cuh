@@ -325,23 +325,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (warp == C::TMA_WARP) {
       // ======================= TMA producer =================================
       // Per unit: Q tiles (once the previous unit's S products are done with
-      // the Q buffer), then K_0, V_0, K_1, V_1, ... into the ring.
-      if (lane == 0) {
-        // K/V tiles are re-read by the other units of the same key/value head:
-        // keep them in L2; Q is read once.
-        const uint64_t keep = ptx::policy_evict_last();
-        const uint64_t once = ptx::policy_evict_first();
-        int idx = 0;  // K/V tiles loaded so far (ring position)
-        int k = 0;
-        bool ok = true;
-        for (; ok; ++k) {
-          const int u = unit_of(p, k);
-          if (u < 0) break;
-          const Unit w = decode_unit(p, u);
-          // Q of this unit, once the previous unit's S products no longer
-          // read the Q buffer.
-          auto load_q = [&]() -> bool {
-            if (!wait_bounded(q_empty, (k & 1) ^ 1u, kErrWaitQEmpty, p.launch_id)) return false;
+      // the Q buffer), then K_0, V_0, K_1, V_1, ... into the ring.  The whole
+      // warp runs the loop and waits (a converged warp resumes from an
+      // mbarrier wait sooner than a single lane does); lane 0 issues.
+      const bool leader = lane == 0;
+      // K/V tiles are re-read by the other units of the same key/value head:
+      // keep them in L2; Q is read once.
+      const uint64_t keep = ptx::policy_evict_last();
+      const uint64_t once = ptx::policy_evict_first();
+      int idx = 0;  // K/V tiles loaded so far (ring position)
+      int k = 0;
+      bool ok = true;
+      for (; ok; ++k) {
+        const int u = unit_of(p, k);
+        if (u < 0) break;
+        const Unit w = decode_unit(p, u);
+        // Q of this unit, once the previous unit's S products no longer read
+        // the Q buffer.
+        auto load_q = [&]() -> bool {
+          if (!warp_wait(q_empty, (k & 1) ^ 1u, kErrWaitQEmpty, p.launch_id)) return false;
+          if (leader) {
             ptx::mbar_arrive_expect_tx(q_full,
                                        ((w.ntile[0] > 0) + (w.ntile[1] > 0)) * C::TILE_BYTES);
             for (int t = 0; t < C::NQ; ++t) {
@@ -350,72 +353,77 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 ptx::tma_load_3d_hint(sQ + t * C::TILE_BYTES + c * C::SUB_BYTES, &tm_q, q_full,
                                       c * 64, w.qblk[t] * C::BM, w.b * p.Hq + w.head[t], once);
             }
-            return true;
-          };
-          const int kv_plane = w.b * p.Hkv + w.g;
-          // K_0 and V_0 go first: they do not depend on the Q buffer
-          const int q_at = min(2, 2 * w.nmax);
-          for (int i = 0; i < 2 * w.nmax; ++i, ++idx) {  // K_0, V_0, K_1, V_1, ...
-            if (i == q_at && !load_q()) {
-              ok = false;
-              break;
-            }
-            const int s = idx % C::NSTAGE;
-            if (!wait_bounded(&kv_empty[s], ((idx / C::NSTAGE) & 1) ^ 1u, kErrWaitKvEmpty,
-                              p.launch_id)) {
-              ok = false;
-              break;
-            }
+          }
+          __syncwarp();
+          return true;
+        };
+        const int kv_plane = w.b * p.Hkv + w.g;
+        // K_0 and V_0 go first: they do not depend on the Q buffer
+        const int q_at = min(2, 2 * w.nmax);
+        for (int i = 0; i < 2 * w.nmax; ++i, ++idx) {  // K_0, V_0, K_1, V_1, ...
+          if (i == q_at && !load_q()) {
+            ok = false;
+            break;
+          }
+          const int s = idx % C::NSTAGE;
+          if (!warp_wait(&kv_empty[s], ((idx / C::NSTAGE) & 1) ^ 1u, kErrWaitKvEmpty,
+                         p.launch_id)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
             ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
             const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
             for (int c = 0; c < C::SUB; ++c)
               ptx::tma_load_3d_hint(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s],
                                     c * 64, (i >> 1) * C::BN, kv_plane, keep);
           }
-          if (ok && q_at == 2 * w.nmax && !load_q()) ok = false;
+          __syncwarp();
         }
-        if (!ok) {
-          // Gave up: let the copies already in flight land before the CTA exits.
-          if (k > 0) wait_bounded(q_full, (k - 1) & 1, kErrWaitQ, p.launch_id);
-          for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
-            wait_bounded(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrWaitKvFull,
-                         p.launch_id);
-        }
+        if (ok && q_at == 2 * w.nmax && !load_q()) ok = false;
       }
-      __syncwarp();
+      if (!ok) {
+        // Gave up: let the copies already in flight land before the CTA exits.
+        if (k > 0) warp_wait(q_full, (k - 1) & 1, kErrWaitQ, p.launch_id);
+        for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
+          warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrWaitKvFull, p.launch_id);
+      }
     } else if (warp == C::MMA_WARP) {
       // ======================= MMA issue ====================================
-      if (lane == 0) {
-        constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
-        constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-B swizzle
-        const uint32_t q_addr = ptx::smem_u32(sQ);
-        const uint32_t kv_addr = ptx::smem_u32(sKV);
-        int base = 0;           // ring position of the unit's K_0
-        int pcnt[2] = {0, 0};   // P tiles consumed per query tile (p_full phases)
-        bool ok = true;
-        for (int k = 0; ok; ++k) {
-          const int u = unit_of(p, k);
-          if (u < 0) break;
-          const Unit w = decode_unit(p, u);
-          if (!wait_bounded(q_full, k & 1, kErrWaitQ, p.launch_id)) break;
-          for (int j = 0; ok && j <= w.nmax; ++j) {
-            const int kidx = base + 2 * j, vidx = base + 2 * j - 1;
-            if (j < w.nmax)
-              ok = wait_bounded(&kv_full[kidx % C::NSTAGE], (kidx / C::NSTAGE) & 1,
-                                kErrWaitKvFull, p.launch_id);
-            if (ok && j > 0)
-              ok = wait_bounded(&kv_full[vidx % C::NSTAGE], (vidx / C::NSTAGE) & 1,
-                                kErrWaitKvFull, p.launch_id);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            for (int t = 0; t < C::NQ && ok; ++t) {
-              if (j >= 1 && j <= w.ntile[t]) {
-                // O_t += P_t(j-1) V_{j-1}; A = P from TMEM, B = V (MN-major in smem)
-                ok = wait_bounded(&p_full[t], pcnt[t] & 1, kErrWaitPFull, p.launch_id);
-                if (!ok) break;
-                ++pcnt[t];
-                ptx::tc_fence_after();
+      // The whole warp runs the loop and waits; lane 0 issues the MMAs and
+      // the commits (a commit tracks the MMAs of the thread that issues it).
+      const bool leader = lane == 0;
+      constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-B swizzle
+      const uint32_t q_addr = ptx::smem_u32(sQ);
+      const uint32_t kv_addr = ptx::smem_u32(sKV);
+      int base = 0;           // ring position of the unit's K_0
+      int pcnt[2] = {0, 0};   // P tiles consumed per query tile (p_full phases)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_of(p, k);
+        if (u < 0) break;
+        const Unit w = decode_unit(p, u);
+        if (!warp_wait(q_full, k & 1, kErrWaitQ, p.launch_id)) break;
+        for (int j = 0; ok && j <= w.nmax; ++j) {
+          const int kidx = base + 2 * j, vidx = base + 2 * j - 1;
+          if (j < w.nmax)
+            ok = warp_wait(&kv_full[kidx % C::NSTAGE], (kidx / C::NSTAGE) & 1, kErrWaitKvFull,
+                           p.launch_id);
+          if (ok && j > 0)
+            ok = warp_wait(&kv_full[vidx % C::NSTAGE], (vidx / C::NSTAGE) & 1, kErrWaitKvFull,
+                           p.launch_id);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          for (int t = 0; t < C::NQ && ok; ++t) {
+            if (j >= 1 && j <= w.ntile[t]) {
+              // O_t += P_t(j-1) V_{j-1}; A = P from TMEM, B = V (MN-major in smem)
+              ok = warp_wait(&p_full[t], pcnt[t] & 1, kErrWaitPFull, p.launch_id);
+              if (!ok) break;
+              ++pcnt[t];
+              ptx::tc_fence_after();
+              if (leader) {
                 // B descriptor low word of the V tile; K step kk is 16 keys = 2 KB further
                 const uint32_t vb_lo =
                     ptx::sdesc_sw128_lo(kv_addr + (vidx % C::NSTAGE) * C::TILE_BYTES, C::SUB_BYTES);
@@ -428,7 +436,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                                       vb_lo + kk * (2048 >> 4), kDescHi, kIdescO);
                 if (j == w.ntile[t]) ptx::tc_commit(&o_full[t]);
               }
-              if (j < w.ntile[t]) {
+              __syncwarp();
+            }
+            if (j < w.ntile[t]) {
+              if (leader) {
                 // S_t = Q_t K_j^T; both operands K-major in smem.  A and B
                 // descriptor low words; K step kk: +32 B, or the next 16 KB sub-tile
                 const uint32_t qa_lo = ptx::sdesc_sw128_lo(q_addr + t * C::TILE_BYTES, 16);
@@ -443,20 +454,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 }
                 ptx::tc_commit(&s_full[t]);
               }
+              __syncwarp();
             }
-            if (!ok) break;
+          }
+          if (!ok) break;
+          if (leader) {
             if (j < w.nmax) ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);
             if (j > 0) ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);
             // the unit's last S products: the Q buffer is free once they complete
             if (j == w.nmax - 1) ptx::tc_commit(q_empty);
           }
-          base += 2 * w.nmax;
+          __syncwarp();
         }
-        // Every MMA issued must finish before tensor memory is released.
-        ptx::tc_commit(drain);
-        wait_bounded(drain, 0, kErrWaitDrain, p.launch_id);
+        base += 2 * w.nmax;
       }
+      // Every MMA issued must finish before tensor memory is released.
+      if (leader) ptx::tc_commit(drain);
       __syncwarp();
+      warp_wait(drain, 0, kErrWaitDrain, p.launch_id);
     }
   } else {
     ptx::setmaxnreg_inc<C::REGS_SOFTMAX>();
