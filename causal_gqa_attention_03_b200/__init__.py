@@ -6,10 +6,13 @@ built in this directory (``python -m causal_gqa_attention_03_b200.build``).
 There is no fallback: if the library is missing, every call raises.
 
 Raw C-ABI names (integer pointers, sizes, stream handle):
-    tessera_attn_fwd, tessera_attn_device_error, tessera_status_str,
-    tessera_attn_last_launch_count
-Tensor convenience wrapper (PyTorch used only for memory and streams):
+    tessera_attn_fwd, tessera_attn_fwd_host, tessera_attn_device_error,
+    tessera_status_str, tessera_attn_last_launch_count,
+    tessera_attn_selftest_timeout
+Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
+    attn_fwd_host(q, k, v, causal=True, scale=None, out=None, lse=None,
+                  staging=None, chunks=0, stream=None)
 """
 from __future__ import annotations
 
@@ -21,8 +24,9 @@ import threading
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_attn.so")
 
 # Symbols declared in include/tessera_attn.h.
-EXPORTED = ("tessera_attn_fwd", "tessera_attn_device_error", "tessera_status_str",
-            "tessera_attn_last_launch_count", "tessera_attn_selftest_timeout")
+EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_device_error",
+            "tessera_status_str", "tessera_attn_last_launch_count",
+            "tessera_attn_selftest_timeout")
 
 # Device error code recorded by tessera_attn_selftest_timeout.
 DEVICE_ERR_SELFTEST = 9
@@ -55,6 +59,9 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci,
                                              ctypes.c_float, vp]
             lib.tessera_attn_fwd.restype = ci
+            lib.tessera_attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci,
+                                                  ci, ci, ci, ci, ctypes.c_float, ci, vp]
+            lib.tessera_attn_fwd_host.restype = ci
             lib.tessera_attn_device_error.argtypes = [ctypes.POINTER(ci)]
             lib.tessera_attn_device_error.restype = ci
             lib.tessera_status_str.argtypes = [ci]
@@ -73,6 +80,16 @@ def tessera_attn_fwd(q: int, k: int, v: int, o: int, lse: int | None, B: int, Hq
     """The C entry point with integer device pointers; returns the status code."""
     return load_library().tessera_attn_fwd(q, k, v, o, lse or None, B, Hq, Hkv, T, d,
                                            int(causal), float(scale), stream or None)
+
+
+def tessera_attn_fwd_host(q_h: int, k_h: int, v_h: int, o_h: int, lse_h: int | None, q_d: int,
+                          k_d: int, v_d: int, o_d: int, lse_d: int | None, B: int, Hq: int,
+                          Hkv: int, T: int, d: int, causal: int, scale: float, chunks: int,
+                          stream: int | None) -> int:
+    """The pipelined host-buffer C entry point; returns the status code."""
+    return load_library().tessera_attn_fwd_host(
+        q_h, k_h, v_h, o_h, lse_h or None, q_d, k_d, v_d, o_d, lse_d or None, B, Hq, Hkv, T, d,
+        int(causal), float(scale), int(chunks), stream or None)
 
 
 def tessera_attn_device_error() -> int:
@@ -130,4 +147,54 @@ def attn_fwd(q, k, v, causal: bool = True, scale: float | None = None, out=None,
                           int(bool(causal)), float(scale), stream.cuda_stream)
     if st != 0:
         raise TesseraError(st, "tessera_attn_fwd")
+    return out, lse
+
+
+def attn_fwd_host(q, k, v, causal: bool = True, scale: float | None = None, out=None, lse=None,
+                  staging=None, chunks: int = 0, stream=None, want_lse: bool = True,
+                  device=None):
+    """Attention forward on host (CPU) bf16 tensors q [B,Hq,T,d], k/v [B,Hkv,T,d].
+
+    The copies to and from the GPU are pipelined with the kernels by the C
+    entry point tessera_attn_fwd_host; pinned (page-locked) tensors let them
+    overlap.  Returns (o, lse) as host tensors (allocated pinned unless given).
+    ``staging`` is a dict with device tensors 'q', 'k', 'v', 'o' and 'lse' of
+    the full sizes (allocated with torch when None).  The call synchronises
+    ``stream`` (default: torch's current stream) before returning.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda:
+            raise TypeError(f"{name} must be a host bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D tensor [B,H,T,d]")
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, T, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B,Hkv,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
+    if staging is None:
+        staging = {"q": torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                   "k": torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
+                   "v": torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
+                   "o": torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                   "lse": torch.empty((B, Hq, T), dtype=torch.float32, device=dev)}
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    lse_d = staging["lse"].data_ptr() if lse is not None else None
+    st = tessera_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None,
+                               staging["q"].data_ptr(), staging["k"].data_ptr(),
+                               staging["v"].data_ptr(), staging["o"].data_ptr(), lse_d, B, Hq, Hkv,
+                               T, d, int(bool(causal)), float(scale), chunks, stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_fwd_host")
+    stream.synchronize()
     return out, lse

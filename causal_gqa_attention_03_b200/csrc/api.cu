@@ -1,8 +1,9 @@
 // C ABI of the causal grouped-query attention forward (see include/tessera_attn.h).
 //
 // Host side: argument checks, TMA tensor maps for Q/K/V, work decomposition,
-// and the kernel launch on the caller's stream.  Nothing here allocates device
-// memory or synchronises.
+// the kernel launch on the caller's stream, and the pipelined host-buffer
+// variant (copies on two library-owned streams).  Nothing here allocates
+// device memory or synchronises.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -121,17 +122,19 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   return TESSERA_OK;
 }
 
-}  // namespace
-
-extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                                int B, int Hq, int Hkv, int T, int d, int causal, float scale,
-                                tessera_stream_t stream) {
-  g_last_launches = 0;
+// Checks shared by the entry points (before any CUDA call).  Returns
+// TESSERA_OK with *empty set when there is nothing to compute.
+int check_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               int B, int Hq, int Hkv, int T, int d, int causal, float scale, bool* empty) {
+  *empty = false;
   if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TESSERA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return TESSERA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return TESSERA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return TESSERA_ERR_UNSUPPORTED;
-  if (B == 0 || T == 0) return TESSERA_OK;
+  if (B == 0 || T == 0) {
+    *empty = true;
+    return TESSERA_OK;
+  }
   // sizes in bytes; every product below stays far inside 64 bits for int inputs
   const size_t q_bytes = static_cast<size_t>(B) * Hq * T * d * 2;
   const size_t kv_bytes = static_cast<size_t>(B) * Hkv * T * d * 2;
@@ -146,9 +149,120 @@ extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, voi
       overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes) ||
       overlaps(lse, lse_bytes, o, q_bytes))
     return TESSERA_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return TESSERA_OK;
+}
+
+int launch_d(int d, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+             int Hq, int Hkv, int T, int causal, float scale, cudaStream_t s) {
   if (d == 64) return launch<64>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
   return launch<128>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
+}
+
+// Streams and events of the host-buffer pipeline, created on first use per
+// device and kept for the life of the process.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, in_done = nullptr, k_done = nullptr, out_done = nullptr;
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipes[64];
+
+HostPipe* host_pipe(int dev) {
+  HostPipe& h = g_pipes[dev];
+  if (h.ready) return &h;
+  if (cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess)
+    return nullptr;
+  for (cudaEvent_t* e : {&h.start, &h.in_done, &h.k_done, &h.out_done})
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+  h.ready = true;
+  return &h;
+}
+
+}  // namespace
+
+extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int T, int d, int causal, float scale,
+                                tessera_stream_t stream) {
+  g_last_launches = 0;
+  bool empty = false;
+  const int st = check_args(q, k, v, o, lse, B, Hq, Hkv, T, d, causal, scale, &empty);
+  if (st != TESSERA_OK || empty) return st;
+  return launch_d(d, q, k, v, o, lse, B, Hq, Hkv, T, causal, scale,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                                     float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d,
+                                     float* lse_d, int B, int Hq, int Hkv, int T, int d,
+                                     int causal, float scale, int chunks,
+                                     tessera_stream_t stream) {
+  g_last_launches = 0;
+  bool empty = false;
+  const int st = check_args(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, T, d, causal, scale, &empty);
+  if (st != TESSERA_OK) return st;
+  if ((lse_h == nullptr) != (lse_d == nullptr) || chunks < 0) return TESSERA_ERR_INVALID_ARG;
+  if (empty) return TESSERA_OK;
+  if (!q_h || !k_h || !v_h || !o_h) return TESSERA_ERR_INVALID_ARG;
+  // Chunks are contiguous ranges of the B*Hkv (batch, key/value head) slices;
+  // each is one launch over a [1, n*G, T, d] view of the buffers.
+  const int slices = static_cast<int>(static_cast<long long>(B) * Hkv);
+  const int n_chunks = chunks == 0 ? (slices < 8 ? slices : 8) : (chunks < slices ? chunks : slices);
+  const int G = Hq / Hkv;
+  const size_t kv_slice = static_cast<size_t>(T) * d * 2;   // bytes of one K (or V) head
+  const size_t q_slice = kv_slice * G;                      // bytes of one group of Q (or O) heads
+  const size_t lse_slice = static_cast<size_t>(T) * G * 4;  // bytes of one group of LSE rows
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = host_pipe(dev);
+  if (!hp) return TESSERA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Everything queued on `stream` before this call (readers or writers of the
+  // staging buffers) comes first.
+  if (cudaEventRecord(hp->start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
+    return TESSERA_ERR_CUDA;
+  const auto c8 = [](const void* p, size_t off) { return static_cast<const char*>(p) + off; };
+  const auto m8 = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
+  int launches = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int s0 = static_cast<int>(static_cast<long long>(slices) * c / n_chunks);
+    const int s1 = static_cast<int>(static_cast<long long>(slices) * (c + 1) / n_chunks);
+    const int n = s1 - s0;
+    if (n == 0) continue;
+    const size_t qo = q_slice * s0, ko = kv_slice * s0, lo = lse_slice * s0;
+    if (cudaMemcpyAsync(m8(q_d, qo), c8(q_h, qo), q_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(m8(k_d, ko), c8(k_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(m8(v_d, ko), c8(v_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+            cudaSuccess ||
+        cudaEventRecord(hp->in_done, hp->in) != cudaSuccess ||
+        cudaStreamWaitEvent(s, hp->in_done, 0) != cudaSuccess)
+      return TESSERA_ERR_CUDA;
+    const int lst = launch_d(d, m8(q_d, qo), m8(k_d, ko), m8(v_d, ko), m8(o_d, qo),
+                             lse_d ? reinterpret_cast<float*>(m8(lse_d, lo)) : nullptr, 1, n * G, n,
+                             T, causal, scale, s);
+    if (lst != TESSERA_OK) return lst;
+    ++launches;
+    if (cudaEventRecord(hp->k_done, s) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->k_done, 0) != cudaSuccess ||
+        cudaMemcpyAsync(m8(o_h, qo), c8(o_d, qo), q_slice * n, cudaMemcpyDeviceToHost, hp->out) !=
+            cudaSuccess)
+      return TESSERA_ERR_CUDA;
+    if (lse_h && cudaMemcpyAsync(m8(lse_h, lo), c8(lse_d, lo), lse_slice * n,
+                                 cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+      return TESSERA_ERR_CUDA;
+  }
+  // Work queued on `stream` after this call sees the host outputs complete.
+  if (cudaEventRecord(hp->out_done, hp->out) != cudaSuccess ||
+      cudaStreamWaitEvent(s, hp->out_done, 0) != cudaSuccess)
+    return TESSERA_ERR_CUDA;
+  g_last_launches = launches;
+  return TESSERA_OK;
 }
 
 extern "C" int tessera_attn_device_error(int* code) {

@@ -71,6 +71,36 @@ int tessera_attn_fwd(const void *q, const void *k, const void *v, void *o,
                      int causal, float scale, tessera_stream_t stream);
 
 /*
+ * The same operation on host buffers, pipelined over the host link.  (The
+ * pages describe the kernel only; this transfer pipeline is this library's.)
+ * The B*Hkv (batch, key/value head) slices are cut into `chunks` contiguous
+ * ranges; for each range Q/K/V are copied host -> device, the kernel of
+ * tessera_attn_fwd runs on it, and O/LSE are copied device -> host.  Copies
+ * run on two streams the library creates per device on first use (kept for
+ * the life of the process), so one range's copies overlap the others' kernels
+ * and copies; the kernels run on `stream`.
+ *
+ * q_h, k_h, v_h  host inputs, layouts as in tessera_attn_fwd.  Page-locked
+ *                memory (cudaHostAlloc / cudaHostRegister) lets the copies
+ *                overlap; pageable memory gives the same results, serialised.
+ * o_h, lse_h     host outputs; lse_h may be NULL (then lse_d must be NULL).
+ * q_d .. lse_d   device buffers of the full sizes, owned by the caller, with
+ *                the rules of tessera_attn_fwd; they also hold the results.
+ * chunks         0: the library's choice (min(B*Hkv, 8)); else clamped to B*Hkv.
+ * stream         the host outputs are complete once the work queued on
+ *                `stream` before the call returns has finished plus this
+ *                call's work: synchronise `stream` before reading them.
+ *
+ * Arguments are checked as in tessera_attn_fwd (plus non-NULL host pointers
+ * and chunks >= 0) before any CUDA call.  Calls are serialised by a mutex.
+ * tessera_attn_last_launch_count() then reports the number of launches.
+ */
+int tessera_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h, void *o_h,
+                          float *lse_h, void *q_d, void *k_d, void *v_d, void *o_d,
+                          float *lse_d, int B, int Hq, int Hkv, int T, int d, int causal,
+                          float scale, int chunks, tessera_stream_t stream);
+
+/*
  * Reads and clears the device-side error word of the current device.  This
  * synchronises the device.  *code receives 0 when no kernel reported a
  * problem since the last call, else a nonzero code naming the wait that gave
@@ -94,8 +124,9 @@ int tessera_attn_selftest_timeout(unsigned int limit_us, tessera_stream_t stream
 const char *tessera_status_str(int status);
 
 /*
- * Kernel launches the last successful tessera_attn_fwd call on this thread
- * queued (0 or 1).  Lets a caller count the library's own launches.
+ * Kernel launches the last successful tessera_attn_fwd (0 or 1) or
+ * tessera_attn_fwd_host (one per chunk) call on this thread queued.  Lets a
+ * caller count the library's own launches.
  */
 int tessera_attn_last_launch_count(void);
 

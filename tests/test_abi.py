@@ -80,6 +80,31 @@ def test_argument_checks_before_any_cuda_call(lib, kw, status):
         assert tess.tessera_attn_last_launch_count() == 0
 
 
+HOST = 0x7f0000000000  # host pointers are never dereferenced by a rejected call
+
+
+def call_host(**kw):
+    a = dict(GOOD, q_h=HOST, k_h=HOST + 0x1000000, v_h=HOST + 0x2000000, o_h=HOST + 0x3000000,
+             lse_h=HOST + 0x4000000, chunks=0)
+    a.update(kw)
+    return tess.tessera_attn_fwd_host(a["q_h"], a["k_h"], a["v_h"], a["o_h"], a["lse_h"], a["q"],
+                                      a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                                      a["T"], a["d"], a["causal"], a["scale"], a["chunks"],
+                                      a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(Hq=6, Hkv=4), 1), (dict(d=96), 2), (dict(scale=0.0), 1),
+    (dict(q=ALIGNED + 8), 3), (dict(o=ALIGNED + 0x40), 1),
+    (dict(chunks=-1), 1), (dict(lse_h=0), 1), (dict(lse=0), 1),
+    (dict(q_h=0), 1), (dict(k_h=0), 1), (dict(v_h=0), 1), (dict(o_h=0), 1),
+    (dict(B=0), 0), (dict(T=0, q_h=0, o_h=0), 0),
+])
+def test_host_entry_argument_checks_before_any_cuda_call(lib, kw, status):
+    assert call_host(**kw) == status
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
 @pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
     assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1

@@ -254,3 +254,29 @@ def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
     o, lse = run_gpu(q, k, v, True, 1.0 / math.sqrt(d))
     ro, rlse = oracle_full(q, k, v, True, 1.0 / math.sqrt(d))
     check(o.numpy(), lse.numpy(), ro, rlse, "after self-test")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,d,causal,chunks", [
+    (1, 32, 8, 1000, 128, True, 0), (2, 6, 3, 129, 64, True, 4), (3, 4, 2, 77, 128, True, 1),
+    (2, 8, 2, 300, 64, False, 100), (1, 2, 1, 1, 64, True, 0),
+])
+def test_host_pipeline_matches_device_call_bitwise(B, Hq, Hkv, T, d, causal, chunks):
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=21 + T, sigma_qk=2.0)
+    scale = 1.0 / math.sqrt(d)
+    o_ref, lse_ref = run_gpu(q, k, v, causal, scale)
+    qp, kp, vp = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o_h, lse_h = tess.attn_fwd_host(qp, kp, vp, causal=causal, scale=scale, chunks=chunks)
+    slices = B * Hkv
+    want = min(slices, 8) if chunks == 0 else min(chunks, slices)
+    assert tess.tessera_attn_last_launch_count() == want
+    assert tess.tessera_attn_device_error() == 0
+    assert torch.equal(o_h.float(), o_ref) and torch.equal(lse_h, lse_ref)
+
+
+def test_host_pipeline_pageable_inputs_and_no_lse():
+    B, Hq, Hkv, T, d = 2, 4, 2, 260, 128
+    q, k, v = inputs.make_qkv(B, Hq, Hkv, T, d, seed=5)
+    o_ref, _ = run_gpu(q, k, v, True, 0.1)
+    o_h, lse_h = tess.attn_fwd_host(q, k, v, causal=True, scale=0.1, want_lse=False)
+    assert lse_h is None
+    assert torch.equal(o_h.float(), o_ref)
