@@ -89,6 +89,25 @@ def make_qkv(B: int, Hq: int, Hkv: int, T: int, d: int, seed: int,
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
+# The upstream gradient dO of a workload draws from its own generator, seeded
+# with the workload's seed plus this offset, so Q/K/V stay the forward's.
+GRAD_SEED_OFFSET = 1_000_003
+
+
+def make_grad(B: int, Hq: int, T: int, d: int, seed: int):
+    """Draw dO as a bf16 CPU tensor [B,Hq,T,d] of standard normals."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return torch.randn((B, Hq, T, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def workload_grad(w: Workload | str):
+    """dO for a workload: make_grad with the workload's seed + GRAD_SEED_OFFSET."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    return make_grad(w.B, w.Hq, w.T, w.d, w.seed + GRAD_SEED_OFFSET)
+
+
 def workload_inputs(w: Workload | str):
     """Inputs of a named workload (bf16 CPU tensors)."""
     if isinstance(w, str):

@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for causal grouped-query attention (forward).
+"""fp64 CPU oracle for causal grouped-query attention (forward and backward).
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  The product path
@@ -15,6 +15,9 @@ set and its torch fallback"), written out as its definition:
     s_ij = scale * <Q[b,h,i], K[b,h//G,j]>,  j <= i when causal
     O[b,h,i] = sum_j softmax_j(s_i) V[b,h//G,j]
     LSE[b,h,i] = logsumexp_j(s_ij)            (natural log)
+
+and its exact gradient with respect to Q, K and V given dO (the chain rule
+through the row softmax; see the backward section of ``attn_ref.c``).
 """
 from __future__ import annotations
 
@@ -79,6 +82,13 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                           ci, ctypes.c_double, i64p,
                                           ctypes.c_int64, dp, dp]
     lib.oracle_attn_rows_bf16.restype = ci
+    lib.oracle_attn_bwd_f64.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci,
+                                        ci, ctypes.c_double]
+    lib.oracle_attn_bwd_f64.restype = ci
+    lib.oracle_attn_bwd_dq_rows_bf16.argtypes = [u16p, u16p, u16p, u16p, ci, ci, ci, ci,
+                                                 ci, ci, ctypes.c_double, i64p,
+                                                 ctypes.c_int64, dp]
+    lib.oracle_attn_bwd_dq_rows_bf16.restype = ci
     return lib
 
 
@@ -145,3 +155,65 @@ def attn_rows_bf16(q_bits, k_bits, v_bits, rows, causal: bool = True,
     if rc != 0:
         raise ValueError(f"oracle_attn_rows_bf16 failed with code {rc}")
     return o, lse
+
+
+def attn_bwd_f64(q, k, v, dout, causal: bool = True, scale: float | None = None,
+                 lib: ctypes.CDLL | None = None):
+    """Gradients of the attention forward in fp64.
+
+    q, dout: [B,Hq,T,d]; k, v: [B,Hkv,T,d].  Returns (dQ [B,Hq,T,d],
+    dK [B,Hkv,T,d], dV [B,Hkv,T,d]) in float64; dK and dV sum over the query
+    heads of each group.
+    """
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape or dout.shape != q.shape:
+        raise ValueError("k, v must be [B,Hkv,T,d] and dout [B,Hq,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(k.shape, dtype=np.float64)
+    dv = np.zeros(k.shape, dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_bwd_f64(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                                 _ptr(v, ctypes.c_double), _ptr(dout, ctypes.c_double),
+                                 _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                 _ptr(dv, ctypes.c_double), B, Hq, Hkv, T, d,
+                                 int(bool(causal)), float(scale))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_f64 failed with code {rc}")
+    return dq, dk, dv
+
+
+def attn_bwd_dq_rows_bf16(q_bits, k_bits, v_bits, dout_bits, rows, causal: bool = True,
+                          scale: float | None = None, lib: ctypes.CDLL | None = None):
+    """Selected rows of dQ from bf16 inputs given as uint16 bit patterns.
+
+    rows: int64 [n,3] of (b, h, i).  Returns dQ rows [n,d] in fp64.
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    dout_bits = np.ascontiguousarray(dout_bits, dtype=np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    B, Hq, T, d = q_bits.shape
+    Hkv = k_bits.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    n = rows.shape[0]
+    dq = np.zeros((n, d), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_bwd_dq_rows_bf16(_ptr(q_bits, ctypes.c_uint16),
+                                          _ptr(k_bits, ctypes.c_uint16),
+                                          _ptr(v_bits, ctypes.c_uint16),
+                                          _ptr(dout_bits, ctypes.c_uint16), B, Hq, Hkv, T,
+                                          d, int(bool(causal)), float(scale),
+                                          _ptr(rows, ctypes.c_int64), n,
+                                          _ptr(dq, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_dq_rows_bf16 failed with code {rc}")
+    return dq

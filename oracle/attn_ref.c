@@ -25,6 +25,8 @@
  * with no blocking, fusion or reordering.  Layouts are contiguous row-major:
  * Q, O [B,Hq,T,d]; K, V [B,Hkv,T,d]; LSE [B,Hq,T].
  *
+ * The file also holds the backward (dQ, dK, dV given dO), below.
+ *
  * Return codes: 0 ok, 1 invalid argument, 2 out of memory.
  */
 #include <math.h>
@@ -169,5 +171,171 @@ int oracle_attn_rows_bf16(const uint16_t *q, const uint16_t *k,
                        &lse_rows[r]);
     }
     free(kh); free(vh); free(qi); free(s);
+    return 0;
+}
+
+/*
+ * ------------------------------------------------------------------ backward
+ * Gradient of the forward above with respect to Q, K and V, given dO (the
+ * gradient of a loss with respect to O; LSE is treated as saved state, not as
+ * an output that receives a gradient).  The pages list the attention backward
+ * as not yet built; its plain reading is the exact derivative of the forward
+ * definition, which the chain rule through the row softmax gives as
+ *
+ *   P_ij  = exp(s_ij - LSE_i)                  j in J(i)
+ *   dV[b,g,j,:] += P_ij * dO[b,h,i,:]          over h in group g and i
+ *   dP_ij = <dO[b,h,i,:], V[b,g,j,:]>
+ *   D_i   = <dO[b,h,i,:], O[b,h,i,:]>          (= sum_j P_ij dP_ij)
+ *   dS_ij = P_ij * (dP_ij - D_i)
+ *   dQ[b,h,i,:]  = scale * sum_j dS_ij K[b,g,j,:]
+ *   dK[b,g,j,:] += scale * dS_ij * Q[b,h,i,:]  over h in group g and i
+ *
+ * written out one query row at a time, with no blocking or reordering.
+ */
+
+/*
+ * Backward of one query row: recomputes the row's scores, probabilities and
+ * output, then adds its contributions to dk/dv (the key/value head's [T,d]
+ * accumulators) and writes dq[0..d).  s, p: scratch of n_keys doubles;
+ * o: scratch of d doubles.
+ */
+static void backward_one_row(const double *q, const double *dout, const double *kh,
+                             const double *vh, int64_t n_keys, int d, double scale,
+                             double *s, double *p, double *o, double *dq,
+                             double *dkh, double *dvh)
+{
+    double lse;
+    attend_one_row(q, kh, vh, n_keys, d, scale, s, o, &lse);
+    /* attend_one_row leaves exp(s_ij - m) in s; recompute the scores */
+    for (int64_t j = 0; j < n_keys; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+            dot += kh[j * d + c] * q[c];
+        s[j] = dot * scale;
+    }
+    for (int64_t j = 0; j < n_keys; ++j)
+        p[j] = exp(s[j] - lse);
+    double D = 0.0;
+    for (int c = 0; c < d; ++c)
+        D += dout[c] * o[c];
+    for (int c = 0; c < d; ++c)
+        dq[c] = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        double dp = 0.0;
+        for (int c = 0; c < d; ++c)
+            dp += dout[c] * vh[j * d + c];
+        const double ds = p[j] * (dp - D);
+        for (int c = 0; c < d; ++c) {
+            dvh[j * d + c] += p[j] * dout[c];
+            dkh[j * d + c] += scale * ds * q[c];
+            dq[c] += scale * ds * kh[j * d + c];
+        }
+    }
+}
+
+/*
+ * Full backward on fp64 inputs: q, dout [B,Hq,T,d]; k, v [B,Hkv,T,d].
+ * Writes dq [B,Hq,T,d], dk and dv [B,Hkv,T,d].
+ */
+int oracle_attn_bwd_f64(const double *q, const double *k, const double *v,
+                        const double *dout, double *dq, double *dk, double *dv,
+                        int B, int Hq, int Hkv, int T, int d, int causal,
+                        double scale)
+{
+    if (check_shape(B, Hq, Hkv, T, d))
+        return 1;
+    const int64_t nkv = (int64_t)B * Hkv * T * d;
+    for (int64_t e = 0; e < nkv; ++e) {
+        dk[e] = 0.0;
+        dv[e] = 0.0;
+    }
+    if (B == 0 || T == 0)
+        return 0;
+    const int G = Hq / Hkv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    double *p = (double *)malloc(sizeof(double) * (size_t)T);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!s || !p || !o) {
+        free(s); free(p); free(o);
+        return 2;
+    }
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hq; ++h) {
+            const int64_t kv = ((int64_t)b * Hkv + h / G) * T * d;
+            for (int i = 0; i < T; ++i) {
+                const int64_t row = ((int64_t)b * Hq + h) * T + i;
+                const int64_t n_keys = causal ? i + 1 : T; /* keys j <= i */
+                backward_one_row(q + row * d, dout + row * d, k + kv, v + kv, n_keys,
+                                 d, scale, s, p, o, dq + row * d, dk + kv, dv + kv);
+            }
+        }
+    }
+    free(s); free(p); free(o);
+    return 0;
+}
+
+/*
+ * Selected rows of dQ on bf16 inputs (raw bit patterns, widened exactly).
+ * rows: n_rows triples (b, h, i); dq_rows [n_rows, d].  A row of dQ needs only
+ * its own query row and the key/value head, so workloads too large for the
+ * full backward can still be checked row by row.
+ */
+int oracle_attn_bwd_dq_rows_bf16(const uint16_t *q, const uint16_t *k,
+                                 const uint16_t *v, const uint16_t *dout, int B,
+                                 int Hq, int Hkv, int T, int d, int causal,
+                                 double scale, const int64_t *rows, int64_t n_rows,
+                                 double *dq_rows)
+{
+    if (check_shape(B, Hq, Hkv, T, d))
+        return 1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= T)
+            return 1;
+    }
+    if (n_rows == 0)
+        return 0;
+    const int G = Hq / Hkv;
+    const size_t td = (size_t)T * d;
+    double *kh = (double *)malloc(sizeof(double) * td);
+    double *vh = (double *)malloc(sizeof(double) * td);
+    double *dkh = (double *)malloc(sizeof(double) * td); /* discarded */
+    double *dvh = (double *)malloc(sizeof(double) * td); /* discarded */
+    double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+    double *gi = (double *)malloc(sizeof(double) * (size_t)d);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    double *p = (double *)malloc(sizeof(double) * (size_t)T);
+    if (!kh || !vh || !dkh || !dvh || !qi || !gi || !o || !s || !p) {
+        free(kh); free(vh); free(dkh); free(dvh); free(qi); free(gi); free(o);
+        free(s); free(p);
+        return 2;
+    }
+    int64_t cur_b = -1, cur_g = -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        const int64_t g = h / G;
+        if (b != cur_b || g != cur_g) {
+            const int64_t base = (b * Hkv + g) * (int64_t)td;
+            for (int64_t e = 0; e < (int64_t)td; ++e) {
+                kh[e] = bf16_bits_to_f64(k[base + e]);
+                vh[e] = bf16_bits_to_f64(v[base + e]);
+            }
+            cur_b = b;
+            cur_g = g;
+        }
+        const int64_t qrow = (b * Hq + h) * (int64_t)T + i;
+        for (int c = 0; c < d; ++c) {
+            qi[c] = bf16_bits_to_f64(q[qrow * d + c]);
+            gi[c] = bf16_bits_to_f64(dout[qrow * d + c]);
+        }
+        const int64_t n_keys = causal ? i + 1 : (int64_t)T;
+        memset(dkh, 0, sizeof(double) * (size_t)n_keys * d);
+        memset(dvh, 0, sizeof(double) * (size_t)n_keys * d);
+        backward_one_row(qi, gi, kh, vh, n_keys, d, scale, s, p, o, dq_rows + r * d,
+                         dkh, dvh);
+    }
+    free(kh); free(vh); free(dkh); free(dvh); free(qi); free(gi); free(o);
+    free(s); free(p);
     return 0;
 }

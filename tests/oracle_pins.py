@@ -216,5 +216,120 @@ def pin_rows_entry(lib):
         assert np.array_equal(ro, o[b, h, i]) and np.array_equal(rlse, lse[b, h, i])
 
 
+# ------------------------------------------------------------------ backward
+def _torch_grads(q, k, v, dout, causal, scale):
+    """torch CPU float64 autograd of SDPA with K/V heads repeated; the gradients
+    of the repeated heads are summed back onto each K/V head by autograd."""
+    G = q.shape[1] // k.shape[1]
+    qt = torch.tensor(q, requires_grad=True)
+    kt = torch.tensor(k, requires_grad=True)
+    vt = torch.tensor(v, requires_grad=True)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(G, dim=1), vt.repeat_interleave(G, dim=1), is_causal=causal,
+        scale=scale)
+    o.backward(torch.from_numpy(dout))
+    return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+def pin_bwd_library_autograd(lib):
+    shapes = [  # (B, Hq, Hkv, T, d, causal, sigma)
+        (1, 1, 1, 1, 4, True, 1.0),
+        (2, 4, 2, 17, 8, True, 1.0),
+        (1, 6, 3, 33, 16, False, 1.0),
+        (2, 8, 2, 40, 32, True, 3.0),
+        (1, 4, 1, 29, 8, False, 2.0),
+    ]
+    for n, (B, Hq, Hkv, T, d, causal, sigma) in enumerate(shapes):
+        q = _rand((B, Hq, T, d), 40 + n, sigma)
+        k = _rand((B, Hkv, T, d), 50 + n, sigma)
+        v = _rand((B, Hkv, T, d), 60 + n)
+        g = _rand((B, Hq, T, d), 70 + n)
+        scale = 1.0 / math.sqrt(d)
+        dq, dk, dv = oracle.attn_bwd_f64(q, k, v, g, causal=causal, scale=scale, lib=lib)
+        rq, rk, rv = _torch_grads(q, k, v, g, causal, scale)
+        for name, a, r in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+            err = np.max(np.abs(a - r)) / max(1.0, np.max(np.abs(r)))
+            assert err <= 1e-12, (name, n, err)
+
+
+def pin_bwd_finite_differences(lib):
+    """Central differences of L = sum(O * dO), O from the forward entry."""
+    B, Hq, Hkv, T, d = 1, 2, 1, 5, 3
+    scale = 0.7
+    q = _rand((B, Hq, T, d), 81)
+    k = _rand((B, Hkv, T, d), 82)
+    v = _rand((B, Hkv, T, d), 83)
+    g = _rand((B, Hq, T, d), 84)
+    eps = 1e-5
+    for causal in (True, False):
+        grads = oracle.attn_bwd_f64(q, k, v, g, causal=causal, scale=scale, lib=lib)
+        for which, x in enumerate((q, k, v)):
+            for idx in np.ndindex(x.shape):
+                xs = [q.copy(), k.copy(), v.copy()]
+                xs[which][idx] += eps
+                lp = np.sum(oracle.attn_fwd_f64(*xs, causal=causal, scale=scale, lib=lib)[0] * g)
+                xs[which][idx] -= 2 * eps
+                lm = np.sum(oracle.attn_fwd_f64(*xs, causal=causal, scale=scale, lib=lib)[0] * g)
+                fd = (lp - lm) / (2 * eps)
+                assert abs(fd - grads[which][idx]) <= 1e-8, (causal, which, idx, fd,
+                                                             grads[which][idx])
+
+
+def pin_bwd_invariants(lib):
+    B, Hq, Hkv, T, d = 2, 6, 2, 23, 8
+    G = Hq // Hkv
+    scale = 0.4
+    q = _rand((B, Hq, T, d), 91, 2.0)
+    k = _rand((B, Hkv, T, d), 92, 2.0)
+    v = _rand((B, Hkv, T, d), 93)
+    g = _rand((B, Hq, T, d), 94)
+    for causal in (True, False):
+        dq, dk, dv = oracle.attn_bwd_f64(q, k, v, g, causal=causal, scale=scale, lib=lib)
+        # rows of P sum to one: the keys' dV add up to the group's dO
+        want = g.reshape(B, Hkv, G, T, d).sum(axis=(2, 3))
+        assert np.allclose(dv.sum(axis=2), want, rtol=0, atol=1e-12), "sum_j dV != sum dO"
+        # rows of dS sum to zero: the keys' dK add up to zero
+        assert np.allclose(dk.sum(axis=2), 0.0, rtol=0, atol=1e-12), "sum_j dK != 0"
+        # GQA equals MHA with repeated K/V heads, the repeats' gradients summed
+        mq, mk, mv = oracle.attn_bwd_f64(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1), g,
+                                         causal=causal, scale=scale, lib=lib)
+        assert np.array_equal(mq, dq), "GQA dQ != repeated-MHA dQ"
+        assert np.allclose(mk.reshape(B, Hkv, G, T, d).sum(axis=2), dk, rtol=0, atol=1e-13)
+        assert np.allclose(mv.reshape(B, Hkv, G, T, d).sum(axis=2), dv, rtol=0, atol=1e-13)
+        # dS does not depend on how the scale is split between q and scale
+        hq, _, _ = oracle.attn_bwd_f64(2.0 * q, k, v, g, causal=causal, scale=scale / 2.0,
+                                       lib=lib)
+        assert np.allclose(hq, dq / 2.0, rtol=0, atol=1e-13), "dQ scale split"
+        # zero upstream gradient
+        zq, zk, zv = oracle.attn_bwd_f64(q, k, v, np.zeros_like(g), causal=causal,
+                                         scale=scale, lib=lib)
+        assert not zq.any() and not zk.any() and not zv.any()
+    # one key: P = 1, so dS = 0 and dV is the group's dO
+    q1, k1, v1, g1 = q[:, :, :1], k[:, :, :1], v[:, :, :1], g[:, :, :1]
+    dq, dk, dv = oracle.attn_bwd_f64(q1, k1, v1, g1, causal=True, scale=scale, lib=lib)
+    assert np.allclose(dq, 0.0, rtol=0, atol=1e-15) and np.allclose(dk, 0.0, rtol=0, atol=1e-15)
+    assert np.allclose(dv, g1.reshape(B, Hkv, G, 1, d).sum(axis=2), rtol=0, atol=1e-15)
+
+
+def pin_bwd_dq_rows_entry(lib):
+    """The bf16 dQ-row entry agrees bit for bit with the full fp64 backward."""
+    from causal_gqa_attention_03_b200.inputs import make_qkv, bf16_bits, sample_rows
+    B, Hq, Hkv, T, d = 1, 4, 2, 70, 16
+    q, k, v = make_qkv(B, Hq, Hkv, T, d, seed=11, sigma_qk=2.0)
+    gq, _, _ = make_qkv(B, Hq, Hkv, T, d, seed=12)
+    scale = 0.25
+    for causal in (True, False):
+        dq, _, _ = oracle.attn_bwd_f64(q.double().numpy(), k.double().numpy(),
+                                       v.double().numpy(), gq.double().numpy(),
+                                       causal=causal, scale=scale, lib=lib)
+        rows = sample_rows(B, Hq, T, 40, seed=13)
+        rq = oracle.attn_bwd_dq_rows_bf16(bf16_bits(q), bf16_bits(k), bf16_bits(v),
+                                          bf16_bits(gq), rows, causal=causal, scale=scale,
+                                          lib=lib)
+        b, h, i = rows.T
+        assert np.array_equal(rq, dq[b, h, i])
+
+
 ALL_PINS = [pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
-            pin_rows_entry]
+            pin_rows_entry, pin_bwd_library_autograd, pin_bwd_finite_differences,
+            pin_bwd_invariants, pin_bwd_dq_rows_entry]

@@ -63,6 +63,24 @@ MUTATIONS = [
     ("query index off by one head row", "dot += q[c] * kh[j * d + c];",
      "dot += q[(c + 1) % d] * kh[j * d + c];"),
     ("bf16 widened with the wrong shift", "(uint32_t)bits << 16", "(uint32_t)bits << 15"),
+    # backward
+    ("backward drops D", "const double ds = p[j] * (dp - D);", "const double ds = p[j] * dp;"),
+    ("backward adds D", "const double ds = p[j] * (dp - D);",
+     "const double ds = p[j] * (dp + D);"),
+    ("D from Q instead of O", "D += dout[c] * o[c];", "D += dout[c] * q[c];"),
+    ("P not normalised by the LSE", "p[j] = exp(s[j] - lse);", "p[j] = exp(s[j]);"),
+    ("dQ missing the scale", "dq[c] += scale * ds * kh[j * d + c];",
+     "dq[c] += ds * kh[j * d + c];"),
+    ("dK missing the scale", "dkh[j * d + c] += scale * ds * q[c];",
+     "dkh[j * d + c] += ds * q[c];"),
+    ("dK from dO instead of Q", "dkh[j * d + c] += scale * ds * q[c];",
+     "dkh[j * d + c] += scale * ds * dout[c];"),
+    ("dV weighted by dS instead of P", "dvh[j * d + c] += p[j] * dout[c];",
+     "dvh[j * d + c] += ds * dout[c];"),
+    ("backward ignores the causal mask", "const int64_t n_keys = causal ? i + 1 : T;",
+     "const int64_t n_keys = T;"),
+    ("backward group mapping h % Hkv", "((int64_t)b * Hkv + h / G)",
+     "((int64_t)b * Hkv + h % Hkv)"),
 ]
 
 
