@@ -13,6 +13,7 @@ Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
     attn_fwd_host(q, k, v, causal=True, scale=None, out=None, lse=None,
                   staging=None, chunks=0, stream=None)
+    attn_bwd(q, k, v, o, lse, dout, causal=True, scale=None, stream=None)
 """
 from __future__ import annotations
 
@@ -24,7 +25,8 @@ import threading
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_attn.so")
 
 # Symbols declared in include/tessera_attn.h.
-EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_device_error",
+EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
+            "tessera_attn_bwd_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
             "tessera_attn_selftest_timeout")
 
@@ -62,6 +64,12 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci,
                                                   ci, ci, ci, ci, ctypes.c_float, ci, vp]
             lib.tessera_attn_fwd_host.restype = ci
+            lib.tessera_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             ctypes.c_size_t, ci, ci, ci, ci, ci, ci,
+                                             ctypes.c_float, vp]
+            lib.tessera_attn_bwd.restype = ci
+            lib.tessera_attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
+            lib.tessera_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
             lib.tessera_attn_device_error.argtypes = [ctypes.POINTER(ci)]
             lib.tessera_attn_device_error.restype = ci
             lib.tessera_status_str.argtypes = [ci]
@@ -90,6 +98,20 @@ def tessera_attn_fwd_host(q_h: int, k_h: int, v_h: int, o_h: int, lse_h: int | N
     return load_library().tessera_attn_fwd_host(
         q_h, k_h, v_h, o_h, lse_h or None, q_d, k_d, v_d, o_d, lse_d or None, B, Hq, Hkv, T, d,
         int(causal), float(scale), int(chunks), stream or None)
+
+
+def tessera_attn_bwd(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: int, dk: int,
+                     dv: int, workspace: int, workspace_bytes: int, B: int, Hq: int, Hkv: int,
+                     T: int, d: int, causal: int, scale: float, stream: int | None) -> int:
+    """The backward C entry point with integer device pointers; returns the status."""
+    return load_library().tessera_attn_bwd(q, k, v, o, lse or None, dout or None, dq or None,
+                                           dk or None, dv or None, workspace or None,
+                                           int(workspace_bytes), B, Hq, Hkv, T, d,
+                                           int(causal), float(scale), stream or None)
+
+
+def tessera_attn_bwd_workspace_bytes(B: int, Hq: int, T: int, d: int) -> int:
+    return load_library().tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
 
 
 def tessera_attn_device_error() -> int:
@@ -198,3 +220,47 @@ def attn_fwd_host(q, k, v, causal: bool = True, scale: float | None = None, out=
         raise TesseraError(st, "tessera_attn_fwd_host")
     stream.synchronize()
     return out, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = None,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of attn_fwd on CUDA tensors.
+
+    q, o, dout: bf16 [B,Hq,T,d]; k, v: bf16 [B,Hkv,T,d]; lse: fp32 [B,Hq,T]
+    from attn_fwd with the same arguments.  Outputs are bf16 and allocated
+    with torch unless given; the fp32 workspace likewise.  Queued on
+    ``stream`` (default: torch's current stream); does not synchronise.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D tensor [B,H,T,d]")
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, T, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B,Hkv,T,d] matching q")
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must match q")
+    if (not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32 or not lse.is_cuda
+            or tuple(lse.shape) != (B, Hq, T) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous CUDA fp32 tensor [B,Hq,T]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16) + 3) // 4, dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = tessera_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(), B,
+                          Hq, Hkv, T, d, int(bool(causal)), float(scale), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_bwd")
+    return dq, dk, dv

@@ -16,9 +16,12 @@
 
 #include "tessera_attn.h"
 #include "attn_fwd_sm100.cuh"
+#include "attn_bwd_sm100.cuh"
 
 namespace {
 
+using tessera::BwdCfg;
+using tessera::BwdParams;
 using tessera::FwdCfg;
 using tessera::FwdParams;
 
@@ -180,6 +183,90 @@ HostPipe* host_pipe(int dev) {
   return &h;
 }
 
+// Bytes of fp32 workspace the backward needs: the dQ accumulator
+// [B,Hq,T,d] and D [B,Hq,T].
+size_t bwd_workspace_bytes(int B, int Hq, int T, int d) {
+  return static_cast<size_t>(B) * Hq * T * (static_cast<size_t>(d) + 1) * 4;
+}
+
+int sm_count(int dev) {
+  static std::atomic<int> counts[64];
+  int sms = counts[dev].load(std::memory_order_acquire);
+  if (sms == 0) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+      return 0;
+    counts[dev].store(sms, std::memory_order_release);
+  }
+  return sms;
+}
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, float* ws, int B, int Hq, int Hkv,
+               int T, int causal, float scale, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  static std::atomic<int> attr_set[64];
+  if (attr_set[dev].load(std::memory_order_acquire) == 0) {
+    if (cudaFuncSetAttribute(tessera::attn_bwd_dkdv_sm100_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return TESSERA_ERR_CUDA;
+    attr_set[dev].store(1, std::memory_order_release);
+  }
+  const int sms = sm_count(dev);
+  if (sms <= 0) return TESSERA_ERR_CUDA;
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
+      !make_map(&tm_v, v, B * Hkv, T, D) || !make_map(&tm_do, dout, B * Hq, T, D))
+    return TESSERA_ERR_CUDA;
+  const long long rows = static_cast<long long>(B) * Hq * T;
+  float* dq_acc = ws;
+  float* dvec = ws + rows * D;
+  // 1. D = rowsum(dO * O), dQ accumulator = 0
+  const long long prep_blocks = (rows + 7) / 8;  // 8 warps (rows) per block
+  const unsigned pb = static_cast<unsigned>(prep_blocks < 4L * sms * 16 ? prep_blocks : 4L * sms * 16);
+  tessera::attn_bwd_prep_kernel<D><<<pb, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dvec, dq_acc,
+      rows);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  // 2. dK, dV and the dQ partials
+  BwdParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = T;
+  p.G = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.nqb = (T + C::BM - 1) / C::BM;
+  const long long units = static_cast<long long>(B) * Hkv * p.nqb;
+  if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  p.num_units = static_cast<int>(units);
+  p.lse = lse;
+  p.dvec = dvec;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+  tessera::attn_bwd_dkdv_sm100_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+      tm_q, tm_k, tm_v, tm_do, p);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  // 3. dQ = bf16(scale * accumulator)
+  const long long n8 = rows * D / 8;
+  const long long cb = (n8 + 255) / 256;
+  const unsigned cg = static_cast<unsigned>(cb < 4L * sms * 8 ? cb : 4L * sms * 8);
+  tessera::attn_bwd_dq_convert_kernel<<<cg, 256, 0, stream>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  g_last_launches = 3;
+  return TESSERA_OK;
+}
+
 }  // namespace
 
 extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -263,6 +350,48 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
     return TESSERA_ERR_CUDA;
   g_last_launches = launches;
   return TESSERA_OK;
+}
+
+extern "C" size_t tessera_attn_bwd_workspace_bytes(int B, int Hq, int T, int d) {
+  if (B < 0 || Hq < 1 || T < 0 || (d != 64 && d != 128)) return 0;
+  return bwd_workspace_bytes(B, Hq, T, d);
+}
+
+extern "C" int tessera_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                                int T, int d, int causal, float scale, tessera_stream_t stream) {
+  g_last_launches = 0;
+  bool empty = false;
+  // Q/K/V and O: the forward's rules (O plays the output, LSE its LSE).
+  int st = check_args(q, k, v, o, lse, B, Hq, Hkv, T, d, causal, scale, &empty);
+  if (st != TESSERA_OK) return st;
+  if (empty) return TESSERA_OK;
+  if (!lse || !dout || !dq || !dk || !dv || !workspace) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return TESSERA_ERR_MISALIGNED;
+  if (workspace_bytes < bwd_workspace_bytes(B, Hq, T, d)) return TESSERA_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(B) * Hq * T * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * T * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(B) * Hq * T * 4;
+  const size_t ws_bytes = bwd_workspace_bytes(B, Hq, T, d);
+  // outputs and workspace must not overlap any input or each other
+  const void* ins[6] = {q, k, v, o, lse, dout};
+  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, lse_bytes, q_bytes};
+  const void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, ws_bytes};
+  for (int a = 0; a < 4; ++a) {
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(outs[a], out_bytes[a], ins[i], in_bytes[i])) return TESSERA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return TESSERA_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal,
+                                     scale, s);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal, scale, s);
 }
 
 extern "C" int tessera_attn_device_error(int* code) {

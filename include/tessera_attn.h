@@ -22,6 +22,7 @@
 #ifndef TESSERA_ATTN_H
 #define TESSERA_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -69,6 +70,41 @@ typedef enum {
 int tessera_attn_fwd(const void *q, const void *k, const void *v, void *o,
                      float *lse, int B, int Hq, int Hkv, int T, int d,
                      int causal, float scale, tessera_stream_t stream);
+
+/*
+ * Backward of tessera_attn_fwd: the gradients dQ, dK, dV of a loss given
+ * dO = dLoss/dO, treating LSE as saved state.  The pages list the attention
+ * backward as not yet built (it is the first extension after the forward);
+ * the operation is the exact derivative of the forward above:
+ *
+ *   P_ij = exp(s_ij - LSE[b,h,i]),  D_i = <dO[b,h,i,:], O[b,h,i,:]>
+ *   dS_ij = P_ij * (<dO[b,h,i,:], V[b,g,j,:]> - D_i)
+ *   dQ[b,h,i,:] = scale * sum_j dS_ij K[b,g,j,:]
+ *   dK[b,g,j,:] = scale * sum_{h in g, i} dS_ij Q[b,h,i,:]
+ *   dV[b,g,j,:] = sum_{h in g, i} P_ij dO[b,h,i,:]
+ *
+ * q, k, v, o, lse  the forward's inputs and outputs (o and lse as written by
+ *                  tessera_attn_fwd with the same arguments), device memory
+ * dout             bf16 [B, Hq, T, d] device, read only
+ * dq               bf16 [B, Hq, T, d] device, written
+ * dk, dv           bf16 [B, Hkv, T, d] device, written
+ * workspace        device memory of at least
+ *                  tessera_attn_bwd_workspace_bytes(B, Hq, T, d) bytes, 16-byte
+ *                  aligned, owned by the caller; overwritten (no contents need
+ *                  to be set before the call)
+ * other arguments  as in tessera_attn_fwd
+ *
+ * Checks as in tessera_attn_fwd, plus: every pointer non-NULL (lse too) and
+ * 16-byte aligned, a large enough workspace, and no overlap between
+ * dq/dk/dv/workspace and any input or each other.  Queues three kernels on
+ * `stream` (tessera_attn_last_launch_count() = 3); bounded waits as in the
+ * forward.
+ */
+size_t tessera_attn_bwd_workspace_bytes(int B, int Hq, int T, int d);
+int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                     const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                     void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                     int T, int d, int causal, float scale, tessera_stream_t stream);
 
 /*
  * The same operation on host buffers, pipelined over the host link.  (The
@@ -124,8 +160,9 @@ int tessera_attn_selftest_timeout(unsigned int limit_us, tessera_stream_t stream
 const char *tessera_status_str(int status);
 
 /*
- * Kernel launches the last successful tessera_attn_fwd (0 or 1) or
- * tessera_attn_fwd_host (one per chunk) call on this thread queued.  Lets a
+ * Kernel launches the last successful tessera_attn_fwd (0 or 1),
+ * tessera_attn_fwd_host (one per chunk) or tessera_attn_bwd (3) call on this
+ * thread queued.  Lets a
  * caller count the library's own launches.
  */
 int tessera_attn_last_launch_count(void);

@@ -105,6 +105,39 @@ def test_host_entry_argument_checks_before_any_cuda_call(lib, kw, status):
     assert tess.tessera_attn_last_launch_count() == 0
 
 
+def call_bwd(**kw):
+    a = dict(GOOD, dout=ALIGNED + 0x5000000, dq=ALIGNED + 0x6000000, dk=ALIGNED + 0x7000000,
+             dv=ALIGNED + 0x8000000, ws=ALIGNED + 0x9000000, ws_bytes=None)
+    a.update(kw)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = tess.tessera_attn_bwd_workspace_bytes(a["B"], a["Hq"], a["T"], a["d"])
+    return tess.tessera_attn_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"],
+                                 a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["B"], a["Hq"],
+                                 a["Hkv"], a["T"], a["d"], a["causal"], a["scale"], a["stream"])
+
+
+def test_bwd_workspace_bytes(lib):
+    assert tess.tessera_attn_bwd_workspace_bytes(2, 8, 100, 64) == 2 * 8 * 100 * 65 * 4
+    assert tess.tessera_attn_bwd_workspace_bytes(1, 1, 1, 128) == 129 * 4
+    assert tess.tessera_attn_bwd_workspace_bytes(1, 1, 1, 96) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(Hq=6, Hkv=4), 1), (dict(d=96), 2), (dict(scale=0.0), 1),
+    (dict(lse=0), 1), (dict(dout=0), 1), (dict(dq=0), 1), (dict(dk=0), 1), (dict(dv=0), 1),
+    (dict(ws=0), 1), (dict(ws_bytes=16), 1),
+    (dict(dout=ALIGNED + 0x5000008), 3), (dict(ws=ALIGNED + 0x9000004), 3),
+    (dict(dq=ALIGNED + 0x40), 1),            # dQ overlaps Q
+    (dict(dk=ALIGNED + 0x6000000), 1),       # dK overlaps dQ
+    (dict(ws=ALIGNED + 0x5000000), 1),       # workspace overlaps dO
+    (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_bwd_argument_checks_before_any_cuda_call(lib, kw, status):
+    assert call_bwd(**kw) == status
+    if status != 0:
+        assert tess.tessera_attn_last_launch_count() == 0
+
+
 @pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
     assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1
