@@ -232,6 +232,36 @@ def time_kernel(w, q, k, v, steps, warmup, flush, stream, tess, torch):
     return times, launches, o, lse
 
 
+def time_backward(w, q, k, v, g, steps, warmup, flush, stream, tess, torch):
+    """The backward (3 launches: D prep, dK/dV + dQ partials, dQ conversion) on
+    the forward's O and LSE, each step after an L2 flush, CUDA events around
+    the three launches."""
+    o, lse = tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = tess.tessera_attn_bwd_workspace_bytes(w.B, w.Hq, w.T, w.d)
+    ws = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=q.device)
+
+    def call():
+        tess.attn_bwd(q, k, v, o, lse, g, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                      workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        call()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call()
+        launches += tess.tessera_attn_last_launch_count()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
+
+
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
     tessera_attn_fwd_host (copies pipelined with the kernels over key/value-head
@@ -337,19 +367,37 @@ def main():
     e2e_ms = max_over_ranks(e2e_ms, dev)
     e2e_value = w.flops * world / (e2e_ms * 1e-3) / 1e12
 
+    # the backward on the same inputs (dO drawn from its own seeded generator)
+    g = inputs.make_grad(w.B, w.Hq, w.T, w.d,
+                         rank_seed(w.seed, rank) + inputs.GRAD_SEED_OFFSET).to(dev)
+    bwd_steps = max(5, min(args.steps, int(0.5 / max(2.5 * w.flops / 5e14, 1e-6))))
+    bwd_times, bwd_launches, bwd_ws = time_backward(w, q, k, v, g, bwd_steps, 3, flush, stream,
+                                                    tess, torch)
+    bwd_max_ms = max_over_ranks(sum(bwd_times), dev)
+    bwd_value = 2.5 * w.flops * bwd_steps * world / (bwd_max_ms * 1e-3) / 1e12
+    err = tess.tessera_attn_device_error()
+    if err != 0:
+        raise SystemExit(f"device-side wait gave up in the backward (code {err})")
+
     sweep = {}
     if not args.no_sweep and world == 1:
         for name, ws in inputs.WORKLOADS.items():
+            qs, ks, vs = (t.to(dev) for t in inputs.workload_inputs(ws))
             if name == w.name:
                 sweep[name] = {"tflops": round(value, 1), "ms": round(ms_per_step, 4)}
-                continue
-            qs, ks, vs = (t.to(dev) for t in inputs.workload_inputs(ws))
-            n = max(5, min(200, int(0.5 / max(ws.flops / 1.2e15, 1e-6))))
-            ts, _, _, _ = time_kernel(ws, qs, ks, vs, n, 3, flush, stream, tess, torch)
-            ms = statistics.median(ts)
-            sweep[name] = {"tflops": round(ws.flops / (ms * 1e-3) / 1e12, 1),
-                           "ms": round(ms, 4)}
-            del qs, ks, vs
+            else:
+                n = max(5, min(200, int(0.5 / max(ws.flops / 1.2e15, 1e-6))))
+                ts, _, _, _ = time_kernel(ws, qs, ks, vs, n, 3, flush, stream, tess, torch)
+                ms = statistics.median(ts)
+                sweep[name] = {"tflops": round(ws.flops / (ms * 1e-3) / 1e12, 1),
+                               "ms": round(ms, 4)}
+            gs = inputs.workload_grad(ws).to(dev)
+            n = max(5, min(100, int(0.3 / max(2.5 * ws.flops / 5e14, 1e-6))))
+            tb, _, _ = time_backward(ws, qs, ks, vs, gs, n, 3, flush, stream, tess, torch)
+            mb = statistics.median(tb)
+            sweep[name]["bwd_tflops"] = round(2.5 * ws.flops / (mb * 1e-3) / 1e12, 1)
+            sweep[name]["bwd_ms"] = round(mb, 4)
+            del qs, ks, vs, gs
         err = tess.tessera_attn_device_error()
         if err != 0:
             raise SystemExit(f"device-side wait gave up in the sweep (code {err})")
@@ -401,6 +449,14 @@ def main():
                 "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per key/value-head chunk "
                         "(H2D copy, kernel, D2H copy; copies overlap kernels) -> pinned host O/LSE"},
         "gpu_launches": launches,
+        "backward": {"metric": "causal GQA attn bwd TFLOP/s (bf16)", "value": round(bwd_value, 2),
+                     "unit": UNIT, "steps": bwd_steps,
+                     "ms_per_step": round(bwd_max_ms / bwd_steps, 5),
+                     "flops_per_step": 2.5 * w.flops,
+                     "flop_count": "5*B*Hq*T^2*d: five products over the causal triangle, "
+                                   "counted as the forward's 2*B*Hq*T^2*d counts two",
+                     "gpu_launches": bwd_launches, "workspace_bytes": bwd_ws,
+                     "l2": "flushed before every timed step"},
         "clocks": clk,
         "sweep": sweep or None,
     }
