@@ -26,7 +26,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_
 
 # Symbols declared in include/tessera_attn.h.
 EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
-            "tessera_attn_bwd_workspace_bytes", "tessera_attn_device_error",
+            "tessera_attn_bwd_workspace_bytes", "tessera_attn_bwd_noalloc",
+            "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
             "tessera_attn_selftest_timeout")
 
@@ -34,7 +35,8 @@ EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
 DEVICE_ERR_SELFTEST = 9
 
 STATUS = {0: "TESSERA_OK", 1: "TESSERA_ERR_INVALID_ARG", 2: "TESSERA_ERR_UNSUPPORTED",
-          3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT"}
+          3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT",
+          6: "TESSERA_ERR_TOO_LARGE"}
 
 _lock = threading.Lock()
 _lib = None
@@ -70,6 +72,11 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_bwd.restype = ci
             lib.tessera_attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
             lib.tessera_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.tessera_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci,
+                                                     ci, ci, ci, ci, ctypes.c_float, vp]
+            lib.tessera_attn_bwd_noalloc.restype = ci
+            lib.tessera_attn_bwd_noalloc_max_workspace_bytes.argtypes = []
+            lib.tessera_attn_bwd_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
             lib.tessera_attn_device_error.argtypes = [ctypes.POINTER(ci)]
             lib.tessera_attn_device_error.restype = ci
             lib.tessera_status_str.argtypes = [ci]
@@ -112,6 +119,20 @@ def tessera_attn_bwd(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: in
 
 def tessera_attn_bwd_workspace_bytes(B: int, Hq: int, T: int, d: int) -> int:
     return load_library().tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
+
+
+def tessera_attn_bwd_noalloc(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: int,
+                             dk: int, dv: int, B: int, Hq: int, Hkv: int, T: int, d: int,
+                             causal: int, scale: float, stream: int | None) -> int:
+    """The backward entry point with the library's own scratch; returns the status."""
+    return load_library().tessera_attn_bwd_noalloc(q, k, v, o, lse or None, dout or None,
+                                                   dq or None, dk or None, dv or None, B, Hq,
+                                                   Hkv, T, d, int(causal), float(scale),
+                                                   stream or None)
+
+
+def tessera_attn_bwd_noalloc_max_workspace_bytes() -> int:
+    return load_library().tessera_attn_bwd_noalloc_max_workspace_bytes()
 
 
 def tessera_attn_device_error() -> int:
@@ -263,4 +284,27 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = N
                           Hq, Hkv, T, d, int(bool(causal)), float(scale), stream.cuda_stream)
     if st != 0:
         raise TesseraError(st, "tessera_attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = None,
+                     dq=None, dk=None, dv=None, stream=None):
+    """As attn_bwd, through tessera_attn_bwd_noalloc (no workspace argument)."""
+    import torch
+
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = tessera_attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                  dv.data_ptr(), B, Hq, Hkv, T, d, int(bool(causal)),
+                                  float(scale), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_bwd_noalloc")
     return dq, dk, dv

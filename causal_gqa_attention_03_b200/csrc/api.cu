@@ -267,6 +267,61 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return TESSERA_OK;
 }
 
+// Checks of the backward's arguments (before any CUDA call).  With
+// check_ws, also the caller's workspace: non-NULL, 16-byte aligned, large
+// enough, and clear of every other buffer.
+int check_bwd_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, const void* dq, const void* dk, const void* dv,
+                   const void* workspace, size_t workspace_bytes, bool check_ws, int B, int Hq,
+                   int Hkv, int T, int d, int causal, float scale, bool* empty) {
+  // Q/K/V and O: the forward's rules (O plays the output, LSE its LSE).
+  const int st = check_args(q, k, v, o, lse, B, Hq, Hkv, T, d, causal, scale, empty);
+  if (st != TESSERA_OK || *empty) return st;
+  if (!lse || !dout || !dq || !dk || !dv || (check_ws && !workspace))
+    return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (check_ws && !aligned16(workspace)))
+    return TESSERA_ERR_MISALIGNED;
+  const size_t ws_bytes = bwd_workspace_bytes(B, Hq, T, d);
+  if (check_ws && workspace_bytes < ws_bytes) return TESSERA_ERR_INVALID_ARG;
+  const size_t q_bytes = static_cast<size_t>(B) * Hq * T * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * T * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(B) * Hq * T * 4;
+  // outputs (and the workspace) must not overlap any input or each other
+  const void* ins[6] = {q, k, v, o, lse, dout};
+  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, lse_bytes, q_bytes};
+  const void* outs[4] = {dq, dk, dv, check_ws ? workspace : nullptr};
+  const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, ws_bytes};
+  for (int a = 0; a < 4; ++a) {
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(outs[a], out_bytes[a], ins[i], in_bytes[i])) return TESSERA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return TESSERA_ERR_INVALID_ARG;
+  }
+  return TESSERA_OK;
+}
+
+// Workspace of tessera_attn_bwd_noalloc: a device array of the library's own
+// module (one per device, set up when the module loads), so that entry point
+// needs no allocation.  Calls that overlap in time on one device share it.
+constexpr size_t kNoAllocScratchBytes = 272ull << 20;
+__device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+// Address of g_bwd_scratch on the current device (looked up once per device).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  static std::atomic<void*> addr[64];
+  void* a = addr[dev].load(std::memory_order_acquire);
+  if (a == nullptr) {
+    if (cudaGetSymbolAddress(&a, g_bwd_scratch) != cudaSuccess || a == nullptr)
+      return TESSERA_ERR_CUDA;
+    addr[dev].store(a, std::memory_order_release);
+  }
+  *out = a;
+  return TESSERA_OK;
+}
+
 }  // namespace
 
 extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -363,35 +418,39 @@ extern "C" int tessera_attn_bwd(const void* q, const void* k, const void* v, con
                                 int T, int d, int causal, float scale, tessera_stream_t stream) {
   g_last_launches = 0;
   bool empty = false;
-  // Q/K/V and O: the forward's rules (O plays the output, LSE its LSE).
-  int st = check_args(q, k, v, o, lse, B, Hq, Hkv, T, d, causal, scale, &empty);
-  if (st != TESSERA_OK) return st;
-  if (empty) return TESSERA_OK;
-  if (!lse || !dout || !dq || !dk || !dv || !workspace) return TESSERA_ERR_INVALID_ARG;
-  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      !aligned16(workspace))
-    return TESSERA_ERR_MISALIGNED;
-  if (workspace_bytes < bwd_workspace_bytes(B, Hq, T, d)) return TESSERA_ERR_INVALID_ARG;
-  const size_t q_bytes = static_cast<size_t>(B) * Hq * T * d * 2;
-  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * T * d * 2;
-  const size_t lse_bytes = static_cast<size_t>(B) * Hq * T * 4;
-  const size_t ws_bytes = bwd_workspace_bytes(B, Hq, T, d);
-  // outputs and workspace must not overlap any input or each other
-  const void* ins[6] = {q, k, v, o, lse, dout};
-  const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, lse_bytes, q_bytes};
-  const void* outs[4] = {dq, dk, dv, workspace};
-  const size_t out_bytes[4] = {q_bytes, kv_bytes, kv_bytes, ws_bytes};
-  for (int a = 0; a < 4; ++a) {
-    for (int i = 0; i < 6; ++i)
-      if (overlaps(outs[a], out_bytes[a], ins[i], in_bytes[i])) return TESSERA_ERR_INVALID_ARG;
-    for (int b = a + 1; b < 4; ++b)
-      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return TESSERA_ERR_INVALID_ARG;
-  }
+  const int st = check_bwd_args(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                true, B, Hq, Hkv, T, d, causal, scale, &empty);
+  if (st != TESSERA_OK || empty) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
   if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal,
                                      scale, s);
   return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal, scale, s);
+}
+
+extern "C" size_t tessera_attn_bwd_noalloc_max_workspace_bytes(void) {
+  return kNoAllocScratchBytes;
+}
+
+extern "C" int tessera_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                        const void* o, const float* lse, const void* dout,
+                                        void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                        int T, int d, int causal, float scale,
+                                        tessera_stream_t stream) {
+  g_last_launches = 0;
+  bool empty = false;
+  const int st = check_bwd_args(q, k, v, o, lse, dout, dq, dk, dv, nullptr, 0, false, B, Hq, Hkv,
+                                T, d, causal, scale, &empty);
+  if (st != TESSERA_OK || empty) return st;
+  if (bwd_workspace_bytes(B, Hq, T, d) > kNoAllocScratchBytes) return TESSERA_ERR_TOO_LARGE;
+  void* ws = nullptr;
+  const int sst = noalloc_scratch(&ws);
+  if (sst != TESSERA_OK) return sst;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* wsf = static_cast<float*>(ws);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, wsf, B, Hq, Hkv, T,
+                                     causal, scale, s);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, wsf, B, Hq, Hkv, T, causal, scale, s);
 }
 
 extern "C" int tessera_attn_device_error(int* code) {
@@ -424,6 +483,7 @@ extern "C" const char* tessera_status_str(int status) {
     case TESSERA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case TESSERA_ERR_CUDA: return "CUDA runtime error";
     case TESSERA_ERR_TIMEOUT: return "device-side wait timed out";
+    case TESSERA_ERR_TOO_LARGE: return "workspace needed exceeds the static scratch array";
     default: return "unknown status";
   }
 }

@@ -38,7 +38,8 @@ typedef enum {
     TESSERA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128 */
     TESSERA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
     TESSERA_ERR_CUDA = 4,        /* the CUDA runtime reported an error */
-    TESSERA_ERR_TIMEOUT = 5      /* a device-side wait gave up (see below) */
+    TESSERA_ERR_TIMEOUT = 5,     /* a device-side wait gave up (see below) */
+    TESSERA_ERR_TOO_LARGE = 6    /* tessera_attn_bwd_noalloc: problem over its scratch size */
 } tessera_status;
 
 /*
@@ -105,6 +106,26 @@ int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
                      const float *lse, const void *dout, void *dq, void *dk, void *dv,
                      void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
                      int T, int d, int causal, float scale, tessera_stream_t stream);
+
+/*
+ * tessera_attn_bwd without a caller-supplied workspace.  (The pages have no
+ * counterpart: this is an interface of this library.)  The workspace is a
+ * device array in the library itself, of
+ * tessera_attn_bwd_noalloc_max_workspace_bytes() bytes (272 MiB) on every
+ * device the library runs on; the call allocates nothing and calls no
+ * allocating routine.  Nothing in the array needs to start at zero: each call
+ * sets all it reads.  Arguments, checks and results are those of
+ * tessera_attn_bwd; a problem whose workspace
+ * (tessera_attn_bwd_workspace_bytes) exceeds the array returns
+ * TESSERA_ERR_TOO_LARGE before any CUDA call.  Calls whose work overlaps in
+ * time on one device (other streams or threads) share the array and race:
+ * queue them on one stream.
+ */
+size_t tessera_attn_bwd_noalloc_max_workspace_bytes(void);
+int tessera_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                             const float *lse, const void *dout, void *dq, void *dk,
+                             void *dv, int B, int Hq, int Hkv, int T, int d, int causal,
+                             float scale, tessera_stream_t stream);
 
 /*
  * The same operation on host buffers, pipelined over the host link.  (The

@@ -1,0 +1,74 @@
+"""tessera_attn_bwd_noalloc: the backward with the library's own static scratch
+array instead of a caller workspace.
+
+The file is collected last so that it runs after every other test as well as
+alone; its GPU tests compare the entry point with tessera_attn_bwd on two
+calls in a row (different problems, the second reusing the scratch the first
+wrote) and on the largest synthetic workload.
+"""
+import math
+
+import pytest
+import torch
+
+import causal_gqa_attention_03_b200 as tess
+from causal_gqa_attention_03_b200 import inputs
+
+ALIGNED = 0x10000000
+TOO_LARGE = 6
+
+
+def test_noalloc_too_large_is_rejected_before_any_cuda_call():
+    lib = tess.load_library()
+    assert lib is not None
+    cap = tess.tessera_attn_bwd_noalloc_max_workspace_bytes()
+    assert cap == 272 << 20
+    B, Hq, Hkv, T, d = 1, 64, 8, 65536, 128
+    assert tess.tessera_attn_bwd_workspace_bytes(B, Hq, T, d) > cap
+    ptrs = [ALIGNED + i * (1 << 34) for i in range(9)]
+    st = tess.tessera_attn_bwd_noalloc(*ptrs, B, Hq, Hkv, T, d, 1, 0.1, None)
+    assert st == TOO_LARGE
+    assert tess.tessera_status_str(st) != "unknown status"
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
+def _both(q, k, v, g, causal, scale):
+    o, lse = tess.attn_fwd(q, k, v, causal=causal, scale=scale)
+    ref = [t.clone() for t in tess.attn_bwd(q, k, v, o, lse, g, causal=causal, scale=scale)]
+    got = tess.attn_bwd_noalloc(q, k, v, o, lse, g, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert tess.tessera_attn_last_launch_count() == 3
+    assert tess.tessera_attn_device_error() == 0
+    return ref, got
+
+
+def _same(ref, got, what):
+    # dK and dV are summed in a fixed order: bit for bit.  dQ adds partials
+    # with atomics, so only its rounding may differ.
+    assert torch.equal(ref[1], got[1]) and torch.equal(ref[2], got[2]), what
+    assert torch.allclose(ref[0].float(), got[0].float(), rtol=2e-2, atol=1e-3), what
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
+    assert torch.cuda.is_available()
+    dev = torch.device("cuda:0")
+    cases = [(1, 8, 2, 1000, 128, True), (2, 4, 4, 513, 64, True), (1, 6, 3, 300, 128, False)]
+    for n, (B, Hq, Hkv, T, d, causal) in enumerate(cases):
+        q, k, v = (t.to(dev) for t in inputs.make_qkv(B, Hq, Hkv, T, d, seed=60 + n,
+                                                      sigma_qk=1.5))
+        g = inputs.make_grad(B, Hq, T, d, seed=70 + n).to(dev)
+        ref, got = _both(q, k, v, g, causal, 1.0 / math.sqrt(d))
+        _same(ref, got, (B, Hq, Hkv, T, d, causal))
+
+
+@pytest.mark.gpu
+def test_noalloc_largest_workload():
+    dev = torch.device("cuda:0")
+    w = inputs.WORKLOADS[inputs.LARGEST]
+    assert (tess.tessera_attn_bwd_workspace_bytes(w.B, w.Hq, w.T, w.d)
+            <= tess.tessera_attn_bwd_noalloc_max_workspace_bytes())
+    q, k, v = (t.to(dev) for t in inputs.workload_inputs(w))
+    g = inputs.workload_grad(w).to(dev)
+    ref, got = _both(q, k, v, g, True, w.scale)
+    _same(ref, got, w.name)
