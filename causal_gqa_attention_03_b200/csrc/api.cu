@@ -218,12 +218,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   const int sms = sm_count(dev);
   if (sms <= 0) return TESSERA_ERR_CUDA;
+  const long long rows = static_cast<long long>(B) * Hq * T;
+  float* dq_acc = ws;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
   if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
       !make_map(&tm_v, v, B * Hkv, T, D) || !make_map(&tm_do, dout, B * Hq, T, D))
     return TESSERA_ERR_CUDA;
-  const long long rows = static_cast<long long>(B) * Hq * T;
-  float* dq_acc = ws;
   float* dvec = ws + rows * D;
   // 1. D = rowsum(dO * O), dQ accumulator = 0
   const long long prep_blocks = (rows + 7) / 8;  // 8 warps (rows) per block

@@ -19,15 +19,19 @@
 //      its K and V tiles in shared memory and its dK, dV accumulators in
 //      tensor memory while it visits every (query head of the group, 128-row
 //      query block) the keys are visible to; each visit adds its dQ partial
-//      (128 rows x D, fp32) into the accumulator with vector reductions.
+//      (128 rows x D, fp32) into the accumulator with vector reductions,
+//      issued by a warpgroup of their own so that they overlap the next
+//      visits (the reductions are bound by L2 throughput, ~4,000 cycles per
+//      visit, about the time of the rest of a visit).
 //   3. attn_bwd_dq_convert_kernel: dQ = bf16(scale * accumulator).
 //
-// Kernel 2 warp roles (256 threads):
-//   warps 0-3  compute: P^T, dS^T (thread r owns key row r), then the dQ
-//              partial read-out (thread r owns query row r), then dK, dV
-//   warp  4    MMA issue (lane 0) and TMEM allocation
-//   warp  5    TMA producer (lane 0)
-//   warps 6-7  idle
+// Kernel 2 warp roles (384 threads):
+//   warps 0-3   compute: P^T, dS^T (thread r owns key row r), then dK, dV
+//   warp  4     MMA issue (lane 0) and TMEM allocation
+//   warp  5     TMA producer (lane 0)
+//   warps 6-7   idle
+//   warps 8-11  dQ read-out: thread r loads query row r of the dQ partial from
+//               TMEM, frees the columns, then adds it into the accumulator
 // Tensor memory (512 columns):
 //   S^T  [0, 128)      P^T (bf16 pairs) written over its first 64 columns;
 //                      the dQ partial (D columns) written over it afterwards
@@ -38,7 +42,7 @@
 // shared memory, written there by the compute warps in the 128-byte swizzled
 // layout the MMA reads).  tcgen05 MMAs from one thread run in order, so dQp
 // overwrites P^T only after dV has read it; the next visit's S^T waits until
-// the compute warps have read dQp out.
+// the read-out warps have loaded dQp into registers.
 #pragma once
 
 #include "attn_fwd_sm100.cuh"
@@ -81,9 +85,10 @@ struct BwdCfg {
   static constexpr int DPT_COL = 128;
   static constexpr int DV_COL = 256;
   static constexpr int DK_COL = 256 + D;
-  static constexpr int THREADS = 256;
+  static constexpr int THREADS = 384;
   static constexpr int MMA_WARP = 4;
   static constexpr int TMA_WARP = 5;
+  static constexpr int READ_WARP0 = 8;  // warps 8-11: lane quadrant = warp % 4
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DK_COL + D <= 512, "tensor memory budget");
 };
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(p_full, 4);   // one arrival per compute warp
     ptx::mbar_init(dq_full, 1);
-    ptx::mbar_init(dq_free, 4);
+    ptx::mbar_init(dq_free, 4);   // one arrival per read-out warp
     ptx::mbar_init(dkv_full, 1);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
@@ -446,71 +451,51 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           sD[row] = (qr < p.T) ? p.dvec[qrow0 + row] : 0.f;
         }
         ptx::bar_sync_named(1, 128);
+        // A warp whose wait gives up still reaches the read-out's barriers
+        // below (every warp takes the same barrier sequence in each visit).
         ok = warp_wait(s_full, vis & 1, kErrBwdS, p.launch_id);
-        if (!ok) continue;
-        ptx::tc_fence_after();
         const bool diag = p.causal && qb == w.kb;
+        if (ok) {
+          ptx::tc_fence_after();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {  // 32 query columns at a time
-          uint32_t sr[32], gr[32];
-          ptx::tmem_ld32(st_addr + 32 * c4, sr);
-          ptx::tmem_ld32(dpt_addr + 32 * c4, gr);
-          ptx::tmem_ld_wait();
-          ptx::reg_fence(sr);
-          ptx::reg_fence(gr);
-          uint32_t pp[16], dd[16];
+          for (int c4 = 0; c4 < 4; ++c4) {  // 32 query columns at a time
+            uint32_t sr[32], gr[32];
+            ptx::tmem_ld32(st_addr + 32 * c4, sr);
+            ptx::tmem_ld32(dpt_addr + 32 * c4, gr);
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(sr);
+            ptx::reg_fence(gr);
+            uint32_t pp[16], dd[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float pv[2], dv[2];
+            for (int i = 0; i < 16; ++i) {
+              float pv[2], dv[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = 32 * c4 + 2 * i + e;
-              const float x = fmaf(__uint_as_float(sr[2 * i + e]), sl2, -sLse[col]);
-              float pe = ptx::ex2(x);
-              if (!key_ok || (diag && col < row)) pe = 0.f;  // key past T, or key > query
-              pv[e] = pe;
-              dv[e] = pe * (__uint_as_float(gr[2 * i + e]) - sD[col]);
+              for (int e = 0; e < 2; ++e) {
+                const int col = 32 * c4 + 2 * i + e;
+                const float x = fmaf(__uint_as_float(sr[2 * i + e]), sl2, -sLse[col]);
+                float pe = ptx::ex2(x);
+                if (!key_ok || (diag && col < row)) pe = 0.f;  // key past T, or key > query
+                pv[e] = pe;
+                dv[e] = pe * (__uint_as_float(gr[2 * i + e]) - sD[col]);
+              }
+              pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
+              dd[i] = ptx::pack_bf16x2(dv[0], dv[1]);
             }
-            pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
-            dd[i] = ptx::pack_bf16x2(dv[0], dv[1]);
-          }
-          ptx::tmem_st16(st_addr + 16 * c4, pp);
-          ptx::tmem_st16(dpt_addr + 16 * c4, dd);
-          // dS row `row`, queries 32*c4 .. 32*c4+31, into the swizzled tile
+            ptx::tmem_st16(st_addr + 16 * c4, pp);
+            ptx::tmem_st16(dpt_addr + 16 * c4, dd);
+            // dS row `row`, queries 32*c4 .. 32*c4+31, into the swizzled tile
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            ptx::st_shared_v4(ds_base + ds_chunk_offset(row, 32 * c4 + 8 * j), dd[4 * j],
-                              dd[4 * j + 1], dd[4 * j + 2], dd[4 * j + 3]);
+            for (int j = 0; j < 4; ++j)
+              ptx::st_shared_v4(ds_base + ds_chunk_offset(row, 32 * c4 + 8 * j), dd[4 * j],
+                                dd[4 * j + 1], dd[4 * j + 2], dd[4 * j + 3]);
+          }
+          ptx::tmem_st_wait();
+          ptx::fence_proxy_async_smem();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(p_full);
         }
-        ptx::tmem_st_wait();
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(p_full);
 
-        // dQ partial: thread `row` now owns query row qb*128 + row.
-        ok = warp_wait(dq_full, vis & 1, kErrBwdDq, p.launch_id);
-        if (!ok) continue;
-        ptx::tc_fence_after();
-        const bool q_ok = qb * C::BM + row < p.T;
-        float* dst = p.dq_acc + (qrow0 + row) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(st_addr + 32 * c, r);
-          ptx::tmem_ld_wait();
-          ptx::reg_fence(r);
-          if (q_ok) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              ptx::red_add_v4_f32(dst + 32 * c + 4 * i, __uint_as_float(r[4 * i]),
-                                  __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                                  __uint_as_float(r[4 * i + 3]));
-          }
-        }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(dq_free);
       }
       if (stop) break;
       // A warp whose wait gave up skips its work but walks on to the next
@@ -550,6 +535,49 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // dK, dV have been read; the next unit's first P^T arrival (after this
       // fence) is what lets the MMA warp overwrite them.
       ptx::tc_fence_before();
+    }
+  } else if (warp >= C::READ_WARP0) {
+    // ======================= dQ read-out ==================================
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // query row within the visit's block
+    const uint32_t src = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::ST_COL;
+    int vis = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = bwd_unit_of(p, k);
+      if (u < 0) break;
+      const BwdUnit w = decode_bwd_unit(p, u);
+      for (int v = 0; v < w.nvisit; ++v, ++vis) {
+        if (!warp_wait(dq_full, vis & 1, kErrBwdDq, p.launch_id)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        uint32_t r[D / 32][32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(src + 32 * c, r[c]);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) ptx::reg_fence(r[c]);
+        // dQp is in registers: its TMEM columns are free for the next S^T
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(dq_free);
+        int head, qb;
+        bwd_visit(p, w, v, head, qb);
+        if (qb * C::BM + row < p.T) {
+          float* dst =
+              p.dq_acc + ((static_cast<long long>(w.b) * p.Hq + head) * p.T + qb * C::BM + row) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              ptx::red_add_v4_f32(dst + 32 * c + 4 * i, __uint_as_float(r[c][4 * i]),
+                                  __uint_as_float(r[c][4 * i + 1]),
+                                  __uint_as_float(r[c][4 * i + 2]),
+                                  __uint_as_float(r[c][4 * i + 3]));
+        }
+      }
     }
   }
 
