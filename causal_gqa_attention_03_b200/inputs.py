@@ -140,3 +140,30 @@ def sample_rows(B: int, Hq: int, T: int, n: int, seed: int) -> np.ndarray:
     while len(rows) < min(n, total):
         rows.add((int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(T))))
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def make_paged(B: int, Hq: int, Hkv: int, d: int, bs: int, seq_lens, seed: int,
+               spare_blocks: int = 3, sigma_qk: float = 1.0):
+    """A decode step over a paged cache: (q [B,Hq,d], k_cache, v_cache
+    [num_blocks,Hkv,bs,d] bf16, block_table int32 [B,max_blocks], seq_lens int32 [B]).
+
+    Each sequence gets ceil(len/bs) blocks at random physical positions (a
+    random permutation of the pool, which has spare_blocks unused blocks);
+    unused table entries are -1.
+    """
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    need = [(int(n) + bs - 1) // bs for n in seq_lens]
+    max_blocks = max(need + [1])
+    num_blocks = sum(need) + spare_blocks
+    q = torch.randn((B, Hq, d), generator=g, dtype=torch.float32) * sigma_qk
+    k = torch.randn((num_blocks, Hkv, bs, d), generator=g, dtype=torch.float32) * sigma_qk
+    v = torch.randn((num_blocks, Hkv, bs, d), generator=g, dtype=torch.float32)
+    perm = torch.randperm(num_blocks, generator=g).numpy().astype(np.int32)
+    table = np.full((B, max_blocks), -1, dtype=np.int32)
+    pos = 0
+    for b in range(B):
+        table[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), table, seq_lens)

@@ -17,7 +17,8 @@ set and its torch fallback"), written out as its definition:
     LSE[b,h,i] = logsumexp_j(s_ij)            (natural log)
 
 and its exact gradient with respect to Q, K and V given dO (the chain rule
-through the row softmax; see the backward section of ``attn_ref.c``).
+through the row softmax; see the backward section of ``attn_ref.c``), and one
+decoding step over a paged key/value cache (the paged-decode section).
 """
 from __future__ import annotations
 
@@ -89,6 +90,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                                  ci, ci, ctypes.c_double, i64p,
                                                  ctypes.c_int64, dp]
     lib.oracle_attn_bwd_dq_rows_bf16.restype = ci
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.oracle_paged_decode_f64.argtypes = [dp, dp, dp, i32p, i32p, ci, ci, ci, ci, ci, ci, ci,
+                                            ctypes.c_double, dp, dp]
+    lib.oracle_paged_decode_f64.restype = ci
     return lib
 
 
@@ -217,3 +222,34 @@ def attn_bwd_dq_rows_bf16(q_bits, k_bits, v_bits, dout_bits, rows, causal: bool 
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd_dq_rows_bf16 failed with code {rc}")
     return dq
+
+
+def paged_decode_f64(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None,
+                     lib: ctypes.CDLL | None = None):
+    """One decode step over a paged K/V cache, in fp64.
+
+    q: [B,Hq,d]; k_cache, v_cache: [num_blocks,Hkv,bs,d]; block_table: int32
+    [B,max_blocks]; seq_lens: int32 [B].  Returns (O [B,Hq,d], LSE [B,Hq]).
+    """
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k_cache = np.ascontiguousarray(k_cache, dtype=np.float64)
+    v_cache = np.ascontiguousarray(v_cache, dtype=np.float64)
+    block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Hq, d = q.shape
+    num_blocks, Hkv, bs, _ = k_cache.shape
+    max_blocks = block_table.shape[1] if block_table.ndim == 2 else 0
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, Hq, d), dtype=np.float64)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_paged_decode_f64(_ptr(q, ctypes.c_double), _ptr(k_cache, ctypes.c_double),
+                                     _ptr(v_cache, ctypes.c_double),
+                                     _ptr(block_table, ctypes.c_int32),
+                                     _ptr(seq_lens, ctypes.c_int32), B, Hq, Hkv, d, bs,
+                                     max_blocks, num_blocks, float(scale),
+                                     _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_decode_f64 failed with code {rc}")
+    return o, lse

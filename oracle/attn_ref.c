@@ -339,3 +339,77 @@ int oracle_attn_bwd_dq_rows_bf16(const uint16_t *q, const uint16_t *k,
     free(s); free(p);
     return 0;
 }
+
+/*
+ * ------------------------------------------------------------- paged decode
+ * One decoding step of attention over a paged key/value cache (the serving
+ * engine's "paged-KV" that the pages name; they give no layout, so this
+ * library's reading is used): sequence b has seq_lens[b] cached tokens; its
+ * token j lives in physical block block_table[b][j / bs] at row j % bs.
+ *
+ *   q        [B, Hq, d]                         one query row per head
+ *   k_cache  [num_blocks, Hkv, bs, d]           v_cache likewise
+ *   block_table [B, max_blocks] int32, seq_lens [B] int32
+ *   o        [B, Hq, d],  lse [B, Hq]
+ *
+ * Query head h of sequence b attends to all seq_lens[b] tokens of key/value
+ * head g = h / G (no further mask: the newest token is the query's own).
+ * seq_lens[b] = 0 gives o = 0 and lse = -inf.  Written out by gathering the
+ * sequence's keys and values into a contiguous buffer and applying the
+ * forward's definition to the single query row.
+ */
+int oracle_paged_decode_f64(const double *q, const double *k_cache, const double *v_cache,
+                            const int32_t *block_table, const int32_t *seq_lens, int B,
+                            int Hq, int Hkv, int d, int bs, int max_blocks, int num_blocks,
+                            double scale, double *o, double *lse)
+{
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || d < 1 || bs < 1 || max_blocks < 0 ||
+        num_blocks < 0)
+        return 1;
+    const int G = Hq / Hkv;
+    int64_t max_len = 0;
+    for (int b = 0; b < B; ++b) {
+        if (seq_lens[b] < 0 || (int64_t)seq_lens[b] > (int64_t)max_blocks * bs)
+            return 1;
+        for (int64_t j = 0; j < seq_lens[b]; j += bs) {
+            const int32_t blk = block_table[(int64_t)b * max_blocks + j / bs];
+            if (blk < 0 || blk >= num_blocks)
+                return 1;
+        }
+        if (seq_lens[b] > max_len)
+            max_len = seq_lens[b];
+    }
+    double *kh = (double *)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1) * d);
+    double *vh = (double *)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1) * d);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+    if (!kh || !vh || !s) {
+        free(kh); free(vh); free(s);
+        return 2;
+    }
+    for (int b = 0; b < B; ++b) {
+        const int64_t n = seq_lens[b];
+        for (int g = 0; g < Hkv; ++g) {
+            /* gather the sequence's keys and values of head g */
+            for (int64_t j = 0; j < n; ++j) {
+                const int32_t blk = block_table[(int64_t)b * max_blocks + j / bs];
+                const int64_t src = (((int64_t)blk * Hkv + g) * bs + j % bs) * d;
+                for (int c = 0; c < d; ++c) {
+                    kh[j * d + c] = k_cache[src + c];
+                    vh[j * d + c] = v_cache[src + c];
+                }
+            }
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                const int64_t row = (int64_t)b * Hq + h;
+                if (n == 0) {
+                    for (int c = 0; c < d; ++c)
+                        o[row * d + c] = 0.0;
+                    lse[row] = -INFINITY;
+                    continue;
+                }
+                attend_one_row(q + row * d, kh, vh, n, d, scale, s, o + row * d, &lse[row]);
+            }
+        }
+    }
+    free(kh); free(vh); free(s);
+    return 0;
+}

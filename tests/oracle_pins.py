@@ -330,6 +330,87 @@ def pin_bwd_dq_rows_entry(lib):
         assert np.array_equal(rq, dq[b, h, i])
 
 
+# ------------------------------------------------------------- paged decode
+def _gathered(k_cache, tab, b, n):
+    bs = k_cache.shape[2]
+    return np.stack([k_cache[tab[b, j // bs], :, j % bs] for j in range(n)], axis=1)  # [Hkv,n,d]
+
+
+def _paged_case(seed, B, Hq, Hkv, d, bs, lens, sigma=1.0):
+    from causal_gqa_attention_03_b200.inputs import make_paged
+    q, k, v, tab, lens = make_paged(B, Hq, Hkv, d, bs, lens, seed=seed, sigma_qk=sigma)
+    return q.double().numpy(), k.double().numpy(), v.double().numpy(), tab, lens
+
+
+def pin_decode_library(lib):
+    cases = [  # (B, Hq, Hkv, d, bs, lens, sigma)
+        (3, 8, 2, 16, 4, [1, 9, 17], 1.0),
+        (2, 4, 4, 8, 1, [5, 3], 2.0),
+        (2, 6, 1, 32, 16, [40, 16], 3.0),
+    ]
+    for n_case, (B, Hq, Hkv, d, bs, lens, sigma) in enumerate(cases):
+        q, k, v, tab, lens = _paged_case(100 + n_case, B, Hq, Hkv, d, bs, lens, sigma)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.paged_decode_f64(q, k, v, tab, lens, scale=scale, lib=lib)
+        G = Hq // Hkv
+        for b in range(B):
+            n = int(lens[b])
+            kk = torch.from_numpy(_gathered(k, tab, b, n)).repeat_interleave(G, dim=0)
+            vv = torch.from_numpy(_gathered(v, tab, b, n)).repeat_interleave(G, dim=0)
+            qq = torch.from_numpy(q[b])[:, None, :]
+            ro = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)
+            rl = torch.logsumexp(scale * (qq @ kk.transpose(-1, -2)), dim=-1)
+            assert np.max(np.abs(o[b] - ro[:, 0].numpy())) <= 1e-12, (n_case, b)
+            assert np.max(np.abs(lse[b] - rl[:, 0].numpy())) <= 1e-12, (n_case, b)
+
+
+def pin_decode_invariants(lib):
+    B, Hq, Hkv, d, bs = 3, 8, 2, 16, 4
+    q, k, v, tab, lens = _paged_case(7, B, Hq, Hkv, d, bs, [6, 1, 13])
+    scale = 0.3
+    o, lse = oracle.paged_decode_f64(q, k, v, tab, lens, scale=scale, lib=lib)
+    # moving the physical blocks (and the table with them) changes nothing
+    perm = np.random.default_rng(3).permutation(k.shape[0])
+    inv = np.argsort(perm)
+    k2, v2 = k[perm], v[perm]
+    tab2 = np.where(tab >= 0, inv[np.maximum(tab, 0)], -1).astype(np.int32)
+    o2, lse2 = oracle.paged_decode_f64(q, k2, v2, tab2, lens, scale=scale, lib=lib)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2), "block placement"
+    # re-paging the same tokens with blocks of one token changes nothing
+    n_tok = int(lens.sum())
+    k1 = np.zeros((n_tok, Hkv, 1, d)); v1 = np.zeros((n_tok, Hkv, 1, d))
+    tab1 = np.full((B, int(lens.max())), -1, dtype=np.int32)
+    pos = 0
+    for b in range(B):
+        for j in range(int(lens[b])):
+            k1[pos, :, 0] = k[tab[b, j // bs], :, j % bs]
+            v1[pos, :, 0] = v[tab[b, j // bs], :, j % bs]
+            tab1[b, j] = pos
+            pos += 1
+    o1, lse1 = oracle.paged_decode_f64(q, k1, v1, tab1, lens, scale=scale, lib=lib)
+    assert np.array_equal(o, o1) and np.array_equal(lse, lse1), "block size"
+    # one token: the value row itself, LSE = its logit
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        k0 = k[tab[1, 0], g, 0]; v0 = v[tab[1, 0], g, 0]
+        assert np.array_equal(o[1, h], v0)
+        assert abs(lse[1, h] - scale * np.dot(q[1, h], k0)) <= 1e-14
+    # no tokens: zero output, LSE -inf
+    o0, lse0 = oracle.paged_decode_f64(q, k, v, tab, np.array([0, 1, 13], np.int32),
+                                       scale=scale, lib=lib)
+    assert not o0[0].any() and np.all(np.isneginf(lse0[0]))
+    # the decode step equals the last row of a causal forward over the tokens
+    for b in range(B):
+        n = int(lens[b])
+        kk = _gathered(k, tab, b, n)[None]
+        vv = _gathered(v, tab, b, n)[None]
+        qq = np.zeros((1, Hq, n, d)); qq[0, :, n - 1] = q[b]
+        fo, fl = oracle.attn_fwd_f64(qq, kk, vv, causal=True, scale=scale, lib=lib)
+        assert np.array_equal(fo[0, :, n - 1], o[b]) and np.array_equal(fl[0, :, n - 1], lse[b])
+
+
 ALL_PINS = [pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
             pin_rows_entry, pin_bwd_library_autograd, pin_bwd_finite_differences,
-            pin_bwd_invariants, pin_bwd_dq_rows_entry]
+            pin_bwd_invariants, pin_bwd_dq_rows_entry, pin_decode_library,
+            pin_decode_invariants]

@@ -81,6 +81,17 @@ MUTATIONS = [
      "const int64_t n_keys = T;"),
     ("backward group mapping h % Hkv", "((int64_t)b * Hkv + h / G)",
      "((int64_t)b * Hkv + h % Hkv)"),
+    # paged decode
+    ("decode row within the block from j / bs",
+     "(((int64_t)blk * Hkv + g) * bs + j % bs) * d", "(((int64_t)blk * Hkv + g) * bs + (j / bs) % bs) * d"),
+    ("decode cache heads reversed", "(((int64_t)blk * Hkv + g) * bs + j % bs) * d",
+     "(((int64_t)blk * Hkv + (Hkv - 1 - g)) * bs + j % bs) * d"),
+    ("decode gathers V from the K cache", "vh[j * d + c] = v_cache[src + c];",
+     "vh[j * d + c] = k_cache[src + c];"),
+    ("decode group mapping h % Hkv", "for (int h = g * G; h < (g + 1) * G; ++h) {",
+     "for (int h = g; h < Hq; h += Hkv) {"),
+    ("decode drops the last token", "attend_one_row(q + row * d, kh, vh, n, d, scale, s, o + row * d, &lse[row]);",
+     "attend_one_row(q + row * d, kh, vh, n > 1 ? n - 1 : n, d, scale, s, o + row * d, &lse[row]);"),
 ]
 
 
