@@ -262,6 +262,38 @@ def time_backward(w, q, k, v, g, steps, warmup, flush, stream, tess, torch):
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
 
 
+def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
+    """One decode step over the paged cache of ``wd`` (2 launches: the split-KV
+    partial kernel and the merge), each step after an L2 flush, CUDA events
+    around both launches.  Returns (per-step ms list, launches, workspace bytes)."""
+    q, kc, vc, table, lens = inputs.make_paged_device(wd, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
+    nbytes = tess.tessera_attn_decode_workspace_bytes(wd.B, wd.Hq, wd.max_len, wd.d)
+    ws = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        tess.attn_decode(q, kc, vc, table, lens, max_seq_len=wd.max_len, scale=wd.scale, out=o,
+                         lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        call()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call()
+        launches += tess.tessera_attn_last_launch_count()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    del q, kc, vc, table, lens, o, lse, ws
+    return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
+
+
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
     tessera_attn_fwd_host (copies pipelined with the kernels over key/value-head
@@ -379,6 +411,16 @@ def main():
     if err != 0:
         raise SystemExit(f"device-side wait gave up in the backward (code {err})")
 
+    # one decode step over a paged K/V cache (its own synthetic serving batch)
+    wd = inputs.DECODE
+    dec_steps = max(5, min(args.steps, 200))
+    dec_times, dec_launches, dec_ws = time_decode(wd, dec_steps, 3, flush, stream, tess, torch,
+                                                  dev)
+    dec_max_ms = max_over_ranks(sum(dec_times), dev)
+    err = tess.tessera_attn_device_error()
+    if err != 0:
+        raise SystemExit(f"device-side error in the decode step (code {err})")
+
     sweep = {}
     if not args.no_sweep and world == 1:
         for name, ws in inputs.WORKLOADS.items():
@@ -457,11 +499,35 @@ def main():
                                    "counted as the forward's 2*B*Hq*T^2*d counts two",
                      "gpu_launches": bwd_launches, "workspace_bytes": bwd_ws,
                      "l2": "flushed before every timed step"},
+        "decode": decode_line(wd, dec_times, dec_max_ms, dec_steps, dec_launches, dec_ws, world,
+                              peaks, peak_src),
         "clocks": clk,
         "sweep": sweep or None,
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak_src):
+    """The decode step's object of the JSON line: HBM-bound, so GB/s of the
+    bytes a step must move (io_bytes) against the measured copy bandwidth."""
+    nbytes = wd.io_bytes()
+    value = nbytes * steps * world / (max_ms * 1e-3) / 1e9
+    per_step = statistics.mean(times)
+    achieved = nbytes / (per_step * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    return {"metric": "paged-KV GQA decode step GB/s (bf16 cache)", "value": round(value, 1),
+            "unit": "GB/s", "steps": steps, "ms_per_step": round(max_ms / steps, 5),
+            "config": wd.describe(),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "bytes_per_step": nbytes,
+                         "byte_count": "K and V rows of every cached token, q, o, lse, "
+                                       "lengths and the block ids read"},
+            "gpu_launches": launches, "workspace_bytes": ws_bytes,
+            "l2": f"flushed before every timed step; the step reads {nbytes / 1e9:.2f} GB, "
+                  "more than L2 holds"}
 
 
 def kernel_source_sha() -> str:

@@ -8,12 +8,17 @@ There is no fallback: if the library is missing, every call raises.
 Raw C-ABI names (integer pointers, sizes, stream handle):
     tessera_attn_fwd, tessera_attn_fwd_host, tessera_attn_device_error,
     tessera_status_str, tessera_attn_last_launch_count,
-    tessera_attn_selftest_timeout
+    tessera_attn_selftest_timeout, tessera_attn_bwd, tessera_attn_bwd_workspace_bytes,
+    tessera_attn_bwd_noalloc, tessera_attn_bwd_noalloc_max_workspace_bytes,
+    tessera_attn_decode, tessera_attn_decode_workspace_bytes
 Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
     attn_fwd_host(q, k, v, causal=True, scale=None, out=None, lse=None,
                   staging=None, chunks=0, stream=None)
     attn_bwd(q, k, v, o, lse, dout, causal=True, scale=None, stream=None)
+    attn_bwd_noalloc(q, k, v, o, lse, dout, causal=True, scale=None, stream=None)
+    attn_decode(q, k_cache, v_cache, block_table, seq_lens, max_seq_len=None,
+                scale=None, stream=None)
 """
 from __future__ import annotations
 
@@ -29,10 +34,13 @@ EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
             "tessera_attn_bwd_workspace_bytes", "tessera_attn_bwd_noalloc",
             "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
-            "tessera_attn_selftest_timeout")
+            "tessera_attn_selftest_timeout", "tessera_attn_decode",
+            "tessera_attn_decode_workspace_bytes")
 
 # Device error code recorded by tessera_attn_selftest_timeout.
 DEVICE_ERR_SELFTEST = 9
+# Device error code of a decode step given a sequence length or block id out of range.
+DEVICE_ERR_DECODE_INPUT = 20
 
 STATUS = {0: "TESSERA_OK", 1: "TESSERA_ERR_INVALID_ARG", 2: "TESSERA_ERR_UNSUPPORTED",
           3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT",
@@ -85,6 +93,11 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_last_launch_count.restype = ci
             lib.tessera_attn_selftest_timeout.argtypes = [ctypes.c_uint, vp]
             lib.tessera_attn_selftest_timeout.restype = ci
+            lib.tessera_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                ci, ci, ci, ci, ci, ci, ci, ci, ctypes.c_float, vp]
+            lib.tessera_attn_decode.restype = ci
+            lib.tessera_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci]
+            lib.tessera_attn_decode_workspace_bytes.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -133,6 +146,22 @@ def tessera_attn_bwd_noalloc(q: int, k: int, v: int, o: int, lse: int, dout: int
 
 def tessera_attn_bwd_noalloc_max_workspace_bytes() -> int:
     return load_library().tessera_attn_bwd_noalloc_max_workspace_bytes()
+
+
+def tessera_attn_decode(q: int, k_cache: int, v_cache: int, block_table: int, seq_lens: int,
+                        o: int, lse: int | None, workspace: int | None, workspace_bytes: int,
+                        B: int, Hq: int, Hkv: int, d: int, block_size: int, max_blocks: int,
+                        num_blocks: int, max_seq_len: int, scale: float,
+                        stream: int | None) -> int:
+    """The paged-KV decode C entry point with integer device pointers; returns the status."""
+    return load_library().tessera_attn_decode(
+        q, k_cache, v_cache, block_table, seq_lens, o, lse or None, workspace or None,
+        int(workspace_bytes), B, Hq, Hkv, d, block_size, max_blocks, num_blocks, max_seq_len,
+        float(scale), stream or None)
+
+
+def tessera_attn_decode_workspace_bytes(B: int, Hq: int, max_seq_len: int, d: int) -> int:
+    return load_library().tessera_attn_decode_workspace_bytes(B, Hq, max_seq_len, d)
 
 
 def tessera_attn_device_error() -> int:
@@ -308,3 +337,58 @@ def attn_bwd_noalloc(q, k, v, o, lse, dout, causal: bool = True, scale: float | 
     if st != 0:
         raise TesseraError(st, "tessera_attn_bwd_noalloc")
     return dq, dk, dv
+
+
+def attn_decode(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int | None = None,
+                scale: float | None = None, out=None, lse=None, workspace=None, stream=None,
+                want_lse: bool = True):
+    """One decode step over a paged K/V cache, on CUDA tensors.
+
+    q: bf16 [B,Hq,d]; k_cache, v_cache: bf16 [num_blocks,Hkv,bs,d];
+    block_table: int32 [B,max_blocks]; seq_lens: int32 [B] (device);
+    max_seq_len: a host-side bound on seq_lens (default: the table's
+    capacity max_blocks * bs).  Returns (o bf16 [B,Hq,d], lse fp32 [B,Hq]).
+    Queued on ``stream`` (default: torch's current stream); does not synchronise.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for name, t in (("block_table", block_table), ("seq_lens", seq_lens)):
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or not t.is_cuda
+                or not t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous CUDA int32 tensor")
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B,Hq,d] and the caches [num_blocks,Hkv,bs,d]")
+    B, Hq, d = q.shape
+    num_blocks, Hkv, bs, dk = k_cache.shape
+    if dk != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must be [num_blocks,Hkv,bs,d] matching q")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [B,max_blocks] and seq_lens [B]")
+    max_blocks = block_table.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_blocks * bs
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    nbytes = tessera_attn_decode_workspace_bytes(B, Hq, max_seq_len, d)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16) + 3) // 4, dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = tessera_attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                             block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                             lse.data_ptr() if lse is not None else None, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), B, Hq, Hkv, d, bs,
+                             max_blocks, num_blocks, int(max_seq_len), float(scale),
+                             stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_decode")
+    return out, lse

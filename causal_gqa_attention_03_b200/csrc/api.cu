@@ -17,6 +17,7 @@
 #include "tessera_attn.h"
 #include "attn_fwd_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
+#include "paged_decode.cuh"
 
 namespace {
 
@@ -322,6 +323,142 @@ int noalloc_scratch(void** out) {
   return TESSERA_OK;
 }
 
+
+// ------------------------------------------------------------ paged decode
+
+// A paged cache [num_blocks, Hkv, bs, d] bf16 viewed as a 2-D tensor of
+// num_blocks * Hkv * bs rows of d columns; boxes of 64 columns x box_rows
+// rows with the 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, long long rows, int d, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t elem[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+long long decode_chunks(int max_seq_len) {
+  return (static_cast<long long>(max_seq_len) + tessera::kDecodeChunk - 1) / tessera::kDecodeChunk;
+}
+
+// Bytes of fp32 workspace the decode step needs: partial outputs
+// [B*Hq, chunks, d] and (max, sum) pairs [B*Hq, chunks, 2].
+size_t decode_workspace_bytes(int B, int Hq, int max_seq_len, int d) {
+  return static_cast<size_t>(B) * Hq * static_cast<size_t>(decode_chunks(max_seq_len)) *
+         (static_cast<size_t>(d) + 2) * 4;
+}
+
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Checks of the decode step's arguments (before any CUDA call).
+int check_decode_args(const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens, const void* o,
+                      const float* lse, const void* workspace, size_t workspace_bytes, int B,
+                      int Hq, int Hkv, int d, int bs, int max_blocks, int num_blocks,
+                      int max_seq_len, float scale, bool* empty) {
+  *empty = false;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TESSERA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || num_blocks < 1 || max_seq_len < 0) return TESSERA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return TESSERA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TESSERA_ERR_UNSUPPORTED;
+  if (!pow2(bs) || bs < 8) return TESSERA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_seq_len) > static_cast<long long>(max_blocks) * bs)
+    return TESSERA_ERR_INVALID_ARG;
+  // TMA row coordinates are 32-bit
+  if (static_cast<long long>(num_blocks) * Hkv * bs > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  if (B == 0) {
+    *empty = true;
+    return TESSERA_OK;
+  }
+  const long long heads = static_cast<long long>(B) * Hq;
+  const long long nch = decode_chunks(max_seq_len);
+  if (heads * nch > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o) return TESSERA_ERR_INVALID_ARG;
+  const size_t ws_bytes = decode_workspace_bytes(B, Hq, max_seq_len, d);
+  if (ws_bytes > 0 && (!workspace || workspace_bytes < ws_bytes)) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (ws_bytes > 0 && !aligned16(workspace)) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return TESSERA_ERR_MISALIGNED;
+  const size_t q_bytes = static_cast<size_t>(heads) * d * 2;
+  const size_t cache_bytes = static_cast<size_t>(num_blocks) * Hkv * bs * d * 2;
+  const size_t table_bytes = static_cast<size_t>(B) * max_blocks * 4;
+  const size_t lens_bytes = static_cast<size_t>(B) * 4;
+  const size_t lse_bytes = static_cast<size_t>(heads) * 4;
+  const void* ins[5] = {q, k_cache, v_cache, block_table, seq_lens};
+  const size_t in_bytes[5] = {q_bytes, cache_bytes, cache_bytes, table_bytes, lens_bytes};
+  const void* outs[3] = {o, lse, ws_bytes > 0 ? workspace : nullptr};
+  const size_t out_bytes[3] = {q_bytes, lse_bytes, ws_bytes};
+  for (int a = 0; a < 3; ++a) {
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(outs[a], out_bytes[a], ins[i], in_bytes[i])) return TESSERA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 3; ++b)
+      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return TESSERA_ERR_INVALID_ARG;
+  }
+  return TESSERA_OK;
+}
+
+template <int D, int GT>
+int launch_decode(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
+                  cudaStream_t stream) {
+  using C = tessera::DecodeCfg<D, GT>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  static std::atomic<int> attr_set[64];
+  if (attr_set[dev].load(std::memory_order_acquire) == 0) {
+    if (cudaFuncSetAttribute(tessera::paged_decode_partial_kernel<D, GT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return TESSERA_ERR_CUDA;
+    attr_set[dev].store(1, std::memory_order_release);
+  }
+  int launches = 0;
+  if (p.nch > 0) {
+    const long long rows = static_cast<long long>(p.num_blocks) * p.Hkv * p.bs;
+    CUtensorMap tm_k, tm_v;
+    if (!make_cache_map(&tm_k, k_cache, rows, D, p.rows_per_box) ||
+        !make_cache_map(&tm_v, v_cache, rows, D, p.rows_per_box))
+      return TESSERA_ERR_CUDA;
+    const long long ctas = static_cast<long long>(p.B) * p.Hkv * p.zgroups * p.nch;
+    if (ctas > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+    tessera::paged_decode_partial_kernel<D, GT>
+        <<<static_cast<unsigned>(ctas), tessera::kDecodeThreads, C::SMEM, stream>>>(tm_k, tm_v,
+                                                                                    p);
+    if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+    ++launches;
+  }
+  const long long warps = static_cast<long long>(p.B) * p.Hq;
+  tessera::paged_decode_merge_kernel<D><<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  g_last_launches = launches + 1;
+  return TESSERA_OK;
+}
+
+template <int D>
+int launch_decode_d(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
+                    cudaStream_t stream) {
+  const int G = p.G;
+  if (G % 8 == 0) {
+    p.zgroups = G / 8;
+    return launch_decode<D, 8>(k_cache, v_cache, p, stream);
+  }
+  if (G % 4 == 0) {
+    p.zgroups = G / 4;
+    return launch_decode<D, 4>(k_cache, v_cache, p, stream);
+  }
+  if (G % 2 == 0) {
+    p.zgroups = G / 2;
+    return launch_decode<D, 2>(k_cache, v_cache, p, stream);
+  }
+  p.zgroups = G;
+  return launch_decode<D, 1>(k_cache, v_cache, p, stream);
+}
+
 }  // namespace
 
 extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -453,6 +590,50 @@ extern "C" int tessera_attn_bwd_noalloc(const void* q, const void* k, const void
   return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, wsf, B, Hq, Hkv, T, causal, scale, s);
 }
 
+extern "C" size_t tessera_attn_decode_workspace_bytes(int B, int Hq, int max_seq_len, int d) {
+  if (B < 0 || Hq < 1 || max_seq_len < 0 || (d != 64 && d != 128)) return 0;
+  return decode_workspace_bytes(B, Hq, max_seq_len, d);
+}
+
+extern "C" int tessera_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_table, const int32_t* seq_lens, void* o,
+                                   float* lse, void* workspace, size_t workspace_bytes, int B,
+                                   int Hq, int Hkv, int d, int block_size, int max_blocks,
+                                   int num_blocks, int max_seq_len, float scale,
+                                   tessera_stream_t stream) {
+  g_last_launches = 0;
+  bool empty = false;
+  const int st = check_decode_args(q, k_cache, v_cache, block_table, seq_lens, o, lse, workspace,
+                                   workspace_bytes, B, Hq, Hkv, d, block_size, max_blocks,
+                                   num_blocks, max_seq_len, scale, &empty);
+  if (st != TESSERA_OK || empty) return st;
+  tessera::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.bs = block_size;
+  p.rows_per_box = block_size < tessera::kDecodeChunk ? block_size : tessera::kDecodeChunk;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.max_seq_len = max_seq_len;
+  p.nch = static_cast<int>(decode_chunks(max_seq_len));
+  p.zgroups = 1;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  float* ws = static_cast<float*>(workspace);
+  p.part_o = ws;
+  p.part_ml = ws ? ws + static_cast<size_t>(B) * Hq * p.nch * d : nullptr;
+  p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_decode_d<64>(k_cache, v_cache, p, s);
+  return launch_decode_d<128>(k_cache, v_cache, p, s);
+}
+
 extern "C" int tessera_attn_device_error(int* code) {
   if (!code) return TESSERA_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return TESSERA_ERR_CUDA;
@@ -479,7 +660,8 @@ extern "C" const char* tessera_status_str(int status) {
   switch (status) {
     case TESSERA_OK: return "ok";
     case TESSERA_ERR_INVALID_ARG: return "invalid argument";
-    case TESSERA_ERR_UNSUPPORTED: return "unsupported head dimension (64 or 128)";
+    case TESSERA_ERR_UNSUPPORTED:
+      return "unsupported head dimension (64 or 128) or block size (a power of two >= 8)";
     case TESSERA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case TESSERA_ERR_CUDA: return "CUDA runtime error";
     case TESSERA_ERR_TIMEOUT: return "device-side wait timed out";

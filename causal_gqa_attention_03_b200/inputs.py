@@ -167,3 +167,111 @@ def make_paged(B: int, Hq: int, Hkv: int, d: int, bs: int, seq_lens, seed: int,
         table[b, :need[b]] = perm[pos:pos + need[b]]
         pos += need[b]
     return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), table, seq_lens)
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """One decode step of a serving batch over a paged K/V cache.
+
+    Sequence lengths are drawn by a numpy ``default_rng(seed)`` as integers
+    uniform in [1, max_len]; the cache is filled as make_paged does (q, then
+    K, then V standard normal, Q and K times sigma_qk, rounded to bf16; blocks
+    at a random permutation of the pool).
+    """
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    bs: int
+    max_len: int
+    seed: int
+    sigma_qk: float = 1.0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+    def seq_lens(self) -> np.ndarray:
+        rng = np.random.default_rng(self.seed)
+        return rng.integers(1, self.max_len + 1, size=self.B).astype(np.int32)
+
+    def io_bytes(self) -> int:
+        """Bytes one step must move through HBM: the K and V rows of every cached
+        token, q and o (bf16), lse (fp32), the lengths and the block ids used."""
+        lens = self.seq_lens().astype(np.int64)
+        kv = int(lens.sum()) * self.Hkv * self.d * 2 * 2
+        qo = 2 * self.B * self.Hq * self.d * 2
+        blocks = int(((lens + self.bs - 1) // self.bs).sum())
+        return kv + qo + self.B * self.Hq * 4 + self.B * 4 + blocks * 4
+
+    def describe(self) -> dict:
+        out = asdict(self)
+        out["G"] = self.G
+        lens = self.seq_lens()
+        out["tokens"] = int(lens.sum())
+        return out
+
+
+# The decode step measured beside the forward: the headline head configuration
+# (Hq=32, Hkv=8, d=128) serving 64 sequences with contexts up to 16384 tokens.
+DECODE = DecodeWorkload("decode_b64_hq32_hkv8_d128_bs16_len1to16384", B=64, Hq=32, Hkv=8,
+                        d=128, bs=16, max_len=16384, seed=11)
+
+
+def make_paged_device(w: DecodeWorkload, device, spare_blocks: int = 3):
+    """make_paged's recipe for a decode workload, drawn on ``device`` (a CUDA
+    generator seeded with w.seed; the block permutation comes from a CPU
+    generator with the same seed); the table has ceil(max_len / bs) columns.
+    Returns (q, k_cache, v_cache, block_table,
+    seq_lens) as device tensors (table and lengths int32)."""
+    lens = w.seq_lens()
+    need = [(int(n) + w.bs - 1) // w.bs for n in lens]
+    max_blocks = (w.max_len + w.bs - 1) // w.bs  # the table covers the longest context
+    num_blocks = sum(need) + spare_blocks
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.seed))
+    q = (torch.randn((w.B, w.Hq, w.d), generator=g, device=device) * w.sigma_qk).to(torch.bfloat16)
+    caches = []
+    for sigma in (w.sigma_qk, 1.0):
+        c = torch.empty((num_blocks, w.Hkv, w.bs, w.d), dtype=torch.bfloat16, device=device)
+        for i in range(0, num_blocks, 4096):  # in slices, to bound the fp32 temporary
+            j = min(num_blocks, i + 4096)
+            c[i:j] = (torch.randn((j - i, w.Hkv, w.bs, w.d), generator=g, device=device)
+                      * sigma).to(torch.bfloat16)
+        caches.append(c)
+    gc = torch.Generator(device="cpu")
+    gc.manual_seed(int(w.seed))
+    perm = torch.randperm(num_blocks, generator=gc).numpy().astype(np.int32)
+    table = np.full((w.B, max_blocks), -1, dtype=np.int32)
+    pos = 0
+    for b in range(w.B):
+        table[b, :need[b]] = perm[pos:pos + need[b]]
+        pos += need[b]
+    return (q, caches[0], caches[1], torch.from_numpy(table).to(device),
+            torch.from_numpy(lens).to(device))
+
+
+def gather_sequences(table: np.ndarray, seq_lens: np.ndarray, rows, bs: int,
+                     k_cache: torch.Tensor, v_cache: torch.Tensor):
+    """A compact copy of the cache for the sequences ``rows``: their blocks,
+    renumbered 0..n-1 in table order, and the matching table and lengths
+    (host tensors).  Lets the oracle check selected sequences of a cache too
+    large for it."""
+    sub_lens = np.asarray(seq_lens, dtype=np.int32)[list(rows)]
+    ids, sub_rows = [], []
+    for b in rows:
+        n = (int(seq_lens[b]) + bs - 1) // bs
+        sub_rows.append(list(range(len(ids), len(ids) + n)))
+        ids += [int(x) for x in table[b, :n]]
+    max_blocks = max([len(r) for r in sub_rows] + [1])
+    sub_table = np.full((len(rows), max_blocks), -1, dtype=np.int32)
+    for i, r in enumerate(sub_rows):
+        sub_table[i, :len(r)] = r
+    idx = torch.tensor(ids if ids else [0], dtype=torch.long, device=k_cache.device)
+    return (k_cache.index_select(0, idx).cpu(), v_cache.index_select(0, idx).cpu(), sub_table,
+            sub_lens)

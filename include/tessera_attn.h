@@ -35,7 +35,7 @@ typedef struct CUstream_st *tessera_stream_t;
 typedef enum {
     TESSERA_OK = 0,
     TESSERA_ERR_INVALID_ARG = 1, /* bad size, null pointer, aliasing, bad scale */
-    TESSERA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128 */
+    TESSERA_ERR_UNSUPPORTED = 2, /* head dimension not 64/128; decode block size */
     TESSERA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
     TESSERA_ERR_CUDA = 4,        /* the CUDA runtime reported an error */
     TESSERA_ERR_TIMEOUT = 5,     /* a device-side wait gave up (see below) */
@@ -158,6 +158,65 @@ int tessera_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h, voi
                           float scale, int chunks, tessera_stream_t stream);
 
 /*
+ * One decoding step over a block-paged key/value cache.  The pages list a
+ * fused paged-attention decode kernel as not yet built (hysenlabs.com Tessera
+ * review, "The kernel set and its torch fallback"; sourcepulse.org Tessera
+ * page, "Limitations & Caveats") beside the engine's block-paged KV cache
+ * with a ref-counted allocator (Tessera README, "What's in it" / "Serving";
+ * hysenlabs.com review, "Serving: block-paged KV, batch recomposition,
+ * speculation").  They give no formula; the plain reading adopted here is the
+ * forward's attention for one new query row per sequence over all of its
+ * cached tokens, which are found through the block table:
+ *
+ *   n = seq_lens[b]; token j < n sits in block block_table[b][j / bs], row j % bs
+ *   s_j = scale * dot(q[b,h,:], k_cache[blk, g, j % bs, :]),  g = floor(h / G)
+ *   o[b,h,:] = sum_j softmax_j(s) * v_cache[blk, g, j % bs, :]
+ *   lse[b,h] = ln sum_j exp(s_j)
+ *
+ * A sequence with n = 0 gets o = 0 and lse = -infinity.
+ *
+ * q            bf16 [B, Hq, d] device, read only (one query row per sequence)
+ * k_cache,     bf16 [num_blocks, Hkv, block_size, d] device, read only; a block
+ *   v_cache    holds block_size consecutive tokens of one sequence for every
+ *              key/value head
+ * block_table  int32 [B, max_blocks] device, read only; entries past a
+ *              sequence's last block are not read
+ * seq_lens     int32 [B] device, read only; each in 0 .. max_seq_len
+ * o            bf16 [B, Hq, d] device, written
+ * lse          fp32 [B, Hq] device, written; may be NULL
+ * workspace    device memory of at least
+ *              tessera_attn_decode_workspace_bytes(B, Hq, max_seq_len, d)
+ *              bytes (may be NULL when that is 0), 16-byte aligned, owned by
+ *              the caller; overwritten, nothing needs to be set before
+ * B >= 0 (0 launches nothing); Hq, Hkv >= 1 with Hq % Hkv == 0;
+ * d            64 or 128, block_size a power of two >= 8, else
+ *              TESSERA_ERR_UNSUPPORTED
+ * max_blocks, num_blocks >= 1; num_blocks * Hkv * block_size < 2^31
+ * max_seq_len  host-side bound on seq_lens, 0 .. max_blocks * block_size;
+ *              it sizes the launch and the workspace
+ * scale        positive finite multiplier of q.k
+ *
+ * Checks before any CUDA call: sizes as above; q, caches, o, lse and the
+ * workspace 16-byte aligned, the table and lengths 4-byte aligned
+ * (TESSERA_ERR_MISALIGNED); no output (o, lse, workspace) overlapping an
+ * input or another output (TESSERA_ERR_INVALID_ARG).  Device-resident values
+ * are checked by the kernel: a length above max_seq_len (or negative) makes
+ * that sequence empty, a block id outside 0 .. num_blocks-1 among the blocks
+ * a sequence needs drops the 128-token part of the sequence holding it; both
+ * record TESSERA_DEVICE_ERR_DECODE_INPUT for tessera_attn_device_error(), and
+ * no memory outside the buffers above is read.  Queues up to two kernels on
+ * `stream` (tessera_attn_last_launch_count() reports them) and does not
+ * synchronise.
+ */
+#define TESSERA_DEVICE_ERR_DECODE_INPUT 20
+size_t tessera_attn_decode_workspace_bytes(int B, int Hq, int max_seq_len, int d);
+int tessera_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens, void *o,
+                        float *lse, void *workspace, size_t workspace_bytes, int B, int Hq,
+                        int Hkv, int d, int block_size, int max_blocks, int num_blocks,
+                        int max_seq_len, float scale, tessera_stream_t stream);
+
+/*
  * Reads and clears the device-side error word of the current device.  This
  * synchronises the device.  *code receives 0 when no kernel reported a
  * problem since the last call, else a nonzero code naming the wait that gave
@@ -182,9 +241,9 @@ const char *tessera_status_str(int status);
 
 /*
  * Kernel launches the last successful tessera_attn_fwd (0 or 1),
- * tessera_attn_fwd_host (one per chunk) or tessera_attn_bwd (3) call on this
- * thread queued.  Lets a
- * caller count the library's own launches.
+ * tessera_attn_fwd_host (one per chunk), tessera_attn_bwd (3) or
+ * tessera_attn_decode (1 or 2) call on this thread queued.  Lets a caller
+ * count the library's own launches.
  */
 int tessera_attn_last_launch_count(void);
 

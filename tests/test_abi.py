@@ -138,6 +138,52 @@ def test_bwd_argument_checks_before_any_cuda_call(lib, kw, status):
         assert tess.tessera_attn_last_launch_count() == 0
 
 
+DEC = dict(q=ALIGNED, kc=ALIGNED + 0x1000000, vc=ALIGNED + 0x2000000, table=ALIGNED + 0x3000000,
+           lens=ALIGNED + 0x3100000, o=ALIGNED + 0x4000000, lse=ALIGNED + 0x4100000,
+           ws=ALIGNED + 0x5000000, ws_bytes=None, B=4, Hq=8, Hkv=2, d=128, bs=16, max_blocks=8,
+           num_blocks=40, max_seq_len=128, scale=0.125, stream=None)
+
+
+def call_decode(**kw):
+    a = dict(DEC)
+    a.update(kw)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = tess.tessera_attn_decode_workspace_bytes(a["B"], a["Hq"],
+                                                                 a["max_seq_len"], a["d"])
+    return tess.tessera_attn_decode(a["q"], a["kc"], a["vc"], a["table"], a["lens"], a["o"],
+                                    a["lse"], a["ws"], a["ws_bytes"], a["B"], a["Hq"], a["Hkv"],
+                                    a["d"], a["bs"], a["max_blocks"], a["num_blocks"],
+                                    a["max_seq_len"], a["scale"], a["stream"])
+
+
+def test_decode_workspace_bytes(lib):
+    # partial outputs and (max, sum) pairs per (sequence, head, 128-token chunk)
+    assert tess.tessera_attn_decode_workspace_bytes(4, 8, 128, 128) == 4 * 8 * 1 * 130 * 4
+    assert tess.tessera_attn_decode_workspace_bytes(2, 4, 129, 64) == 2 * 4 * 2 * 66 * 4
+    assert tess.tessera_attn_decode_workspace_bytes(3, 4, 0, 64) == 0
+    assert tess.tessera_attn_decode_workspace_bytes(1, 1, 1, 96) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(Hq=6, Hkv=4), 1), (dict(Hkv=0), 1), (dict(d=96), 2),
+    (dict(bs=12), 2), (dict(bs=4), 2), (dict(bs=0), 2), (dict(scale=float("nan")), 1),
+    (dict(max_blocks=0), 1), (dict(num_blocks=0), 1), (dict(max_seq_len=-1), 1),
+    (dict(max_seq_len=8 * 16 + 1), 1),                 # beyond the table's capacity
+    (dict(num_blocks=1 << 26), 1),                     # rows past 32-bit TMA coordinates
+    (dict(q=0), 1), (dict(kc=0), 1), (dict(table=0), 1), (dict(lens=0), 1), (dict(o=0), 1),
+    (dict(ws=0), 1), (dict(ws_bytes=16), 1),
+    (dict(q=ALIGNED + 8), 3), (dict(vc=ALIGNED + 0x2000004), 3),
+    (dict(table=ALIGNED + 0x3000002), 3), (dict(ws=ALIGNED + 0x5000008), 3),
+    (dict(o=ALIGNED + 0x40), 1),                       # o overlaps q
+    (dict(lse=ALIGNED + 0x3000000), 1),                # lse overlaps the block table
+    (dict(ws=ALIGNED + 0x4000000), 1),                 # workspace overlaps o
+    (dict(B=0), 0),
+])
+def test_decode_argument_checks_before_any_cuda_call(lib, kw, status):
+    assert call_decode(**kw) == status
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
 @pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
     assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1
