@@ -346,11 +346,15 @@ long long decode_chunks(int max_seq_len) {
   return (static_cast<long long>(max_seq_len) + tessera::kDecodeChunk - 1) / tessera::kDecodeChunk;
 }
 
-// Bytes of fp32 workspace the decode step needs: partial outputs
-// [B*Hq, chunks, d] and (max, sum) pairs [B*Hq, chunks, 2].
+// Bytes of workspace the decode step needs: fp32 partial outputs
+// [B*Hq, slots, d] and (max, sum) pairs [B*Hq, slots, 2] with one slot per
+// possible 128-token chunk, then an int slot count per item (<= B*Hq items),
+// rounded up to 16 bytes.
 size_t decode_workspace_bytes(int B, int Hq, int max_seq_len, int d) {
-  return static_cast<size_t>(B) * Hq * static_cast<size_t>(decode_chunks(max_seq_len)) *
-         (static_cast<size_t>(d) + 2) * 4;
+  const size_t heads = static_cast<size_t>(B) * Hq;
+  const size_t slots = static_cast<size_t>(decode_chunks(max_seq_len));
+  if (slots == 0) return 0;
+  return heads * slots * (static_cast<size_t>(d) + 2) * 4 + (heads * 4 + 15) / 16 * 16;
 }
 
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -418,22 +422,22 @@ int launch_decode(const void* k_cache, const void* v_cache, tessera::DecodeParam
     attr_set[dev].store(1, std::memory_order_release);
   }
   int launches = 0;
-  if (p.nch > 0) {
+  if (p.nslot > 0) {
     const long long rows = static_cast<long long>(p.num_blocks) * p.Hkv * p.bs;
     CUtensorMap tm_k, tm_v;
     if (!make_cache_map(&tm_k, k_cache, rows, D, p.rows_per_box) ||
         !make_cache_map(&tm_v, v_cache, rows, D, p.rows_per_box))
       return TESSERA_ERR_CUDA;
-    const long long ctas = static_cast<long long>(p.B) * p.Hkv * p.zgroups * p.nch;
-    if (ctas > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+    const int sms = sm_count(dev);
+    if (sms <= 0) return TESSERA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(sms);  // persistent: one CTA per SM
     tessera::paged_decode_partial_kernel<D, GT>
-        <<<static_cast<unsigned>(ctas), tessera::kDecodeThreads, C::SMEM, stream>>>(tm_k, tm_v,
-                                                                                    p);
+        <<<grid, tessera::kDecodeThreads, C::SMEM, stream>>>(tm_k, tm_v, p);
     if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
     ++launches;
   }
-  const long long warps = static_cast<long long>(p.B) * p.Hq;
-  tessera::paged_decode_merge_kernel<D><<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(p);
+  const long long warps = static_cast<long long>(p.B) * p.Hq;  // one merge CTA each
+  tessera::paged_decode_merge_kernel<D><<<static_cast<unsigned>(warps), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = launches + 1;
   return TESSERA_OK;
@@ -622,12 +626,14 @@ extern "C" int tessera_attn_decode(const void* q, const void* k_cache, const voi
   p.max_blocks = max_blocks;
   p.num_blocks = num_blocks;
   p.max_seq_len = max_seq_len;
-  p.nch = static_cast<int>(decode_chunks(max_seq_len));
+  p.nslot = static_cast<int>(decode_chunks(max_seq_len));
   p.zgroups = 1;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   float* ws = static_cast<float*>(workspace);
   p.part_o = ws;
-  p.part_ml = ws ? ws + static_cast<size_t>(B) * Hq * p.nch * d : nullptr;
+  const size_t heads_slots = static_cast<size_t>(B) * Hq * p.nslot;
+  p.part_ml = ws ? ws + heads_slots * d : nullptr;
+  p.slots = ws ? reinterpret_cast<int*>(ws + heads_slots * (d + 2)) : nullptr;
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) return launch_decode_d<64>(k_cache, v_cache, p, s);

@@ -8,23 +8,31 @@
 //   O[b,h,:] = sum_j softmax_j(scale * <q[b,h], k_j>) v_j,  LSE = log-sum-exp.
 //
 // The step reads every cached key and value once and does a few flops per
-// byte, so it is bound by HBM bandwidth and runs on the FP32 pipes.  Split-KV
-// (one CTA per 128-token chunk of one sequence and key/value head, for GT of
-// its G query heads) and a merge:
-//   1. paged_decode_partial_kernel: the pages of the chunk come into shared
-//      memory by TMA (boxes of 64 columns x R rows, R = min(bs, 128), with the
-//      128-byte swizzle, evict-first in L2).  Scores: a thread per token and
-//      column half, reading its swizzled K row without bank conflicts while
-//      q is a shared-memory broadcast.  Per head: the chunk max m and
-//      p = 2^(s - m), l = sum p.  Values: threads over 4-column groups and
-//      token slices, then a sum over the slices.  Writes the unnormalised
-//      partial o, m and l per (b, h, chunk).
-//   2. paged_decode_merge_kernel: a warp per (b, h) combines the chunks:
-//      M = max m_c, L = sum l_c 2^(m_c - M), O = sum o_c 2^(m_c - M) / L.
-// Scores are in log2 units (q is pre-multiplied by scale * log2(e)).
-// A sequence length above the step's maximum, or a block id outside the
-// cache among the pages a chunk needs, sets a device error code; such a
-// sequence (chunk) contributes nothing and nothing outside the cache is read.
+// byte, so it is bound by HBM bandwidth and runs on the FP32 pipes (packed
+// f32x2 FMAs).  An item is one sequence and key/value head, for GT of its G
+// query heads; its tokens form ceil(n / 128) chunks.
+//   1. paged_decode_partial_kernel, persistent (one CTA per SM).  The chunks
+//      of all items, item after item, form one stream; CTA k takes the k-th
+//      of gridDim.x equal contiguous shares of it, so every SM moves the same
+//      number of chunks whatever the lengths.  A producer warp finds its
+//      share from the lengths and fills a ring of NS shared-memory stages by
+//      TMA: a chunk's K and V pages (boxes of 64 columns x R rows, R =
+//      min(bs, 128), 128-byte swizzle, evict-first in L2), plus the q rows at
+//      the first chunk of an item.  Eight consumer warps run an online
+//      softmax over the consecutive chunks of an item (a segment): per chunk,
+//      scores (warp = column slice, lane = tokens, q in registers, swizzled K
+//      rows read without bank conflicts), per head the running max m and sum
+//      l with p = 2^(s - m), and p.V accumulated in registers (warp = column
+//      slice, lanes = token slices x 4-column groups).  At a segment's end the
+//      unnormalised o, m and l go to partial slot (item, k - first CTA of the
+//      item); the CTA that ends an item records its slot count.
+//   2. paged_decode_merge_kernel: a CTA per (b, h) combines the slots:
+//      M = max m_s, L = sum l_s 2^(m_s - M), O = sum o_s 2^(m_s - M) / L.
+// Scores are in log2 units (q is multiplied by scale * log2(e)).
+// A sequence length above the step's maximum (or negative), or a block id
+// outside the cache among the pages a chunk needs, sets a device error code;
+// such a sequence is empty, such a chunk contributes nothing, and nothing
+// outside the cache is read.
 #pragma once
 
 #include <cuda.h>
@@ -36,30 +44,47 @@
 namespace tessera {
 
 constexpr uint32_t kErrDecodeInput = 20;  // a sequence length or block id out of range
-constexpr uint32_t kErrDecodeWait = 21;   // the wait for a chunk's pages gave up
+constexpr uint32_t kErrDecodeWait = 21;   // a wait of the decode pipeline gave up
 
-constexpr int kDecodeChunk = 128;    // tokens per CTA
-constexpr int kDecodeThreads = 256;  // 8 warps
+constexpr int kDecodeChunk = 128;                  // tokens per chunk
+constexpr int kDecodeConsumers = 256;              // 8 consumer warps
+constexpr int kDecodeThreads = 288;                // + the producer warp
+constexpr int kDecodeProducerWarp = 8;
+constexpr int kDecodeMaxBoxes = kDecodeChunk / 8;  // boxes per chunk at the smallest block size
+
+// flags of a ring stage
+constexpr int kStageBad = 1;        // a page of the chunk is not in the cache: skip it
+constexpr int kStageSegFirst = 2;   // first chunk of this CTA's segment of the item (q copied)
+constexpr int kStageSegLast = 4;    // last chunk of the segment: write the partial
+constexpr int kStageItemLast = 8;   // last chunk of the item: record the slot count
 
 template <int D, int GT>
 struct DecodeCfg {
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
-  static_assert(GT == 1 || GT == 2 || GT == 4 || GT == 8, "1, 2, 4 or 8 heads per CTA");
+  static_assert(GT == 1 || GT == 2 || GT == 4 || GT == 8, "1, 2, 4 or 8 heads per item");
   static constexpr int CH = kDecodeChunk;
   static constexpr int NH = D / 64;      // 64-column halves (one TMA box width each)
   static constexpr int HALF = CH * 128;  // bytes of one half-tile [CH rows][64 cols]
-  static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = NH * HALF;
-  static constexpr int Q_OFF = 2 * NH * HALF;             // float [GT][D]
-  static constexpr int SP_OFF = Q_OFF + GT * D * 4;       // float [2][GT][CH] partial scores
-  static constexpr int P_OFF = SP_OFF + 2 * GT * CH * 4;  // float [CH][GT]
-  static constexpr int ML_OFF = P_OFF + CH * GT * 4;      // float m[GT], l[GT]
-  static constexpr int BAR_OFF = ML_OFF + 64;             // 2 mbarriers + a flag
-  static constexpr int BYTES = BAR_OFF + 32;
-  static constexpr int SMEM = BYTES + 1024;               // slack for the 1024-byte alignment
-  // the sums over token slices reuse the K tile: [8 warps][GT][D] floats
-  static_assert(8 * GT * D * 4 <= NH * HALF, "slice sums fit in the K tile");
-  static_assert(GT * D / 4 <= kDecodeThreads, "one output group per thread");
+  static constexpr int KV_BYTES = 2 * NH * HALF;  // K half-tiles, then V half-tiles
+  static constexpr int Q_BYTES = GT * D * 2;      // the item's q rows (bf16)
+  static constexpr int STAGE = (KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
+  static constexpr int CPW = D / 8;               // columns per consumer warp
+  // ring stages: 3 (d = 128) or 6 (d = 64), fewer where the scratch of 8 query
+  // heads leaves no room
+  static constexpr int NS_MAX = D == 128 ? 3 : 6;
+  static constexpr int FIXED = GT * D * 4 + 8 * GT * CH * 4 + CH * GT * 4 + 32 + 48 * NS_MAX;
+  static constexpr int NS_FIT = (232448 - 1024 - FIXED) / STAGE;
+  static constexpr int NS = NS_FIT < NS_MAX ? NS_FIT : NS_MAX;
+  static_assert(NS >= 2, "at least double buffering");
+  static constexpr int SQ_OFF = NS * STAGE;               // float [GT][D]
+  static constexpr int SP_OFF = SQ_OFF + GT * D * 4;      // float [8][GT][CH] partial scores
+  static constexpr int P_OFF = SP_OFF + 8 * GT * CH * 4;  // float [CH][GT]
+  static constexpr int AL_OFF = P_OFF + CH * GT * 4;      // float alpha[GT]
+  static constexpr int META_OFF = AL_OFF + 32;            // int [NS][8]
+  static constexpr int BAR_OFF = META_OFF + 32 * NS;      // full[NS], empty[NS]
+  static constexpr int BYTES = BAR_OFF + 16 * NS;
+  static constexpr int SMEM = BYTES + 1024;  // slack for the 1024-byte alignment
+  static_assert(SMEM <= 232448, "fits the 227 KB a CTA may use");
 };
 
 struct DecodeParams {
@@ -68,9 +93,10 @@ struct DecodeParams {
   const int32_t* seq_lens;     // [B]
   __nv_bfloat16* o;            // [B, Hq, D]
   float* lse;                  // [B, Hq] or null
-  float* part_o;               // [B*Hq, nch, D]  unnormalised partial outputs
-  float* part_ml;              // [B*Hq, nch, 2]  chunk max (log2 units) and sum
-  int B, Hq, Hkv, G, bs, rows_per_box, max_blocks, num_blocks, max_seq_len, nch, zgroups;
+  float* part_o;               // [B*Hq, nslot, D]  unnormalised partial outputs
+  float* part_ml;              // [B*Hq, nslot, 2]  running max (log2 units) and sum
+  int* slots;                  // [B*Hkv*zgroups]   partial slots written per item
+  int B, Hq, Hkv, G, bs, rows_per_box, max_blocks, num_blocks, max_seq_len, nslot, zgroups;
   float scale_log2;  // scale * log2(e)
   unsigned long long launch_id;
 };
@@ -89,6 +115,10 @@ __device__ __forceinline__ int decode_len(const DecodeParams& p, int b) {
   return n;
 }
 
+__device__ __forceinline__ int decode_chunks(int n) {
+  return (n + kDecodeChunk - 1) / kDecodeChunk;
+}
+
 // Bounded wait on an mbarrier phase (no other CTA's state matters here).
 __device__ __forceinline__ bool decode_wait(uint64_t* bar, uint32_t parity) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -99,320 +129,504 @@ __device__ __forceinline__ bool decode_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&f)[8]) {
-  f[0] = __uint_as_float(u.x << 16);
-  f[1] = __uint_as_float(u.x & 0xffff0000u);
-  f[2] = __uint_as_float(u.y << 16);
-  f[3] = __uint_as_float(u.y & 0xffff0000u);
-  f[4] = __uint_as_float(u.z << 16);
-  f[5] = __uint_as_float(u.z & 0xffff0000u);
-  f[6] = __uint_as_float(u.w << 16);
-  f[7] = __uint_as_float(u.w & 0xffff0000u);
-}
-
 // Byte offset, in a [rows][64 cols] bf16 half-tile written by TMA with the
 // 128-byte swizzle (1024-byte aligned), of the 16-byte chunk c of row r.
 __device__ __forceinline__ uint32_t sw128(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int GT>
-__device__ __forceinline__ void decode_empty_partial(const DecodeParams& p, long long head0,
-                                                     int c) {
-  if (threadIdx.x < GT) {
-    float* ml = p.part_ml + ((head0 + threadIdx.x) * p.nch + c) * 2;
-    ml[0] = -INFINITY;
-    ml[1] = 0.f;
+// bf16 pair (low half = lower column) -> fp32 pair
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ long long warp_incl_scan(long long x, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  return x;
+}
+
+// The producer's view of one chunk of the stream.
+struct DecodeCursor {
+  int b, n, nchunks;  // sequence, its length and chunks
+  int gz;             // g * zgroups + z
+  int c;              // chunk within the item
+  long long item0;    // stream position of the item's first chunk
+};
+
+// Producer warp: this CTA's share [lo, hi) of the chunk stream, one ring
+// stage per chunk, block ids of the next chunk read while the current one is
+// issued.  Ends with a sentinel stage (b = -1).
+template <int D, int GT>
+__device__ __forceinline__ void decode_produce(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                               const DecodeParams& p, uint8_t* sm, int* meta,
+                                               uint64_t* full, uint64_t* empty, int lane) {
+  using C = DecodeCfg<D, GT>;
+  const int R = p.rows_per_box;
+  const long long HZ = static_cast<long long>(p.Hkv) * p.zgroups;
+  // total chunks, then this CTA's share
+  long long tot = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    long long ch = b < p.B ? decode_chunks(decode_len(p, b)) : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, off);
+    tot += ch;
+  }
+  const long long total = tot * HZ;
+  const long long per = (total + gridDim.x - 1) / gridDim.x;
+  const long long lo = static_cast<long long>(blockIdx.x) * per;
+  long long hi = min(lo + per, total);
+  uint32_t produced = 0;
+  bool alive = true;
+  if (lo < hi) {
+    // the sequence holding stream position lo
+    DecodeCursor cur{};
+    long long pre = 0;
+    for (int b0 = 0;; b0 += 32) {
+      const int b = b0 + lane;
+      const int n = b < p.B ? decode_len(p, b) : 0;
+      const long long ch = static_cast<long long>(decode_chunks(n)) * HZ;
+      const long long incl = warp_incl_scan(ch, lane) + pre;
+      const unsigned hit = __ballot_sync(0xffffffffu, b < p.B && incl > lo);
+      if (hit) {
+        const int j = __ffs(hit) - 1;
+        cur.b = b0 + j;
+        cur.n = __shfl_sync(0xffffffffu, n, j);
+        const long long start_b = __shfl_sync(0xffffffffu, incl - ch, j);
+        cur.nchunks = decode_chunks(cur.n);
+        const long long r = lo - start_b;
+        cur.gz = static_cast<int>(r / cur.nchunks);
+        cur.c = static_cast<int>(r % cur.nchunks);
+        cur.item0 = start_b + static_cast<long long>(cur.gz) * cur.nchunks;
+        break;
+      }
+      pre = __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const uint64_t pol = ptx::policy_evict_first();
+    // block id of box `lane` of the chunk at `cu` (0 when the lane has none)
+    auto load_ids = [&](const DecodeCursor& cu, int& blk, int& npg) {
+      const int nt = min(C::CH, cu.n - cu.c * C::CH);
+      npg = (nt + R - 1) / R;
+      blk = 0;
+      if (lane < npg)
+        blk = p.block_table[static_cast<long long>(cu.b) * p.max_blocks +
+                            (cu.c * C::CH + lane * R) / p.bs];
+    };
+    int blk, npg;
+    load_ids(cur, blk, npg);
+    for (long long pos = lo; pos < hi; ++pos) {
+      // the next chunk's coordinates and block ids, read while this one is issued
+      DecodeCursor nxt = cur;
+      int nblk = 0, nnpg = 0;
+      if (pos + 1 < hi) {
+        if (++nxt.c == nxt.nchunks) {
+          nxt.c = 0;
+          nxt.item0 += nxt.nchunks;
+          if (++nxt.gz == HZ) {  // next sequence with tokens
+            nxt.gz = 0;
+            do {  // the stream has more chunks, so such a sequence exists before B
+              ++nxt.b;
+              nxt.n = nxt.b < p.B ? decode_len(p, nxt.b) : -1;
+            } while (nxt.n == 0);
+            if (nxt.n < 0) {  // lengths changed under the kernel: stop after this chunk
+              decode_error(p, kErrDecodeInput);
+              nxt.n = 0;
+            }
+            nxt.nchunks = decode_chunks(nxt.n);
+          }
+        }
+        if (nxt.n > 0)
+          load_ids(nxt, nblk, nnpg);
+        else
+          hi = pos + 1;
+      }
+      const bool bad = __any_sync(0xffffffffu, lane < npg && (blk < 0 || blk >= p.num_blocks));
+      const bool seg_first = pos == lo || cur.c == 0;
+      const bool item_last = cur.c == cur.nchunks - 1;
+      const bool seg_last = pos == hi - 1 || item_last;
+      const int flags = (bad ? kStageBad : 0) | (seg_first ? kStageSegFirst : 0) |
+                        (seg_last ? kStageSegLast : 0) | (item_last ? kStageItemLast : 0);
+      const uint32_t s = produced % C::NS;
+      bool ok = true;
+      if (lane == 0) {
+        if (bad) decode_error(p, kErrDecodeInput);
+        ok = decode_wait(&empty[s], ((produced / C::NS) & 1) ^ 1u);
+        if (!ok) decode_error(p, kErrDecodeWait);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        alive = false;
+        break;
+      }
+      const int nt = min(C::CH, cur.n - cur.c * C::CH);
+      const int g = cur.gz / p.zgroups, z = cur.gz % p.zgroups;
+      if (lane == 0) {
+        int* m = meta + 8 * s;
+        m[0] = cur.b;
+        m[1] = cur.gz;
+        m[2] = cur.c;
+        m[3] = nt;
+        m[4] = flags;
+        // partial slot: this CTA's index among the CTAs that share the item
+        m[5] = static_cast<int>(blockIdx.x - cur.item0 / per);
+        const uint32_t qb = seg_first && !bad ? C::Q_BYTES : 0;
+        if (bad)
+          ptx::mbar_arrive(&full[s]);
+        else
+          ptx::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(npg * R * D * 4) + qb);
+        if (qb) {
+          const long long head0 = static_cast<long long>(cur.b) * p.Hq + g * p.G + z * GT;
+          ptx::bulk_load(sm + s * C::STAGE + C::KV_BYTES, p.q + head0 * D, C::Q_BYTES,
+                         &full[s]);
+        }
+      }
+      __syncwarp();
+      if (!bad && lane < npg) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int tok = cur.c * C::CH + lane * R;
+        const int row = (blk * p.Hkv + g) * p.bs + tok % p.bs;
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h)
+          ptx::tma_load_2d_hint(st + h * C::HALF + lane * R * 128, tm_k, &full[s], 64 * h, row,
+                                pol);
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h)
+          ptx::tma_load_2d_hint(st + (C::NH + h) * C::HALF + lane * R * 128, tm_v, &full[s],
+                                64 * h, row, pol);
+      }
+      ++produced;
+      cur = nxt;
+      blk = nblk;
+      npg = nnpg;
+    }
+  }
+  if (alive && lane == 0) {
+    const uint32_t s = produced % C::NS;
+    if (decode_wait(&empty[s], ((produced / C::NS) & 1) ^ 1u)) {
+      meta[8 * s] = -1;
+      ptx::mbar_arrive(&full[s]);
+    } else {
+      decode_error(p, kErrDecodeWait);
+    }
+  }
+}
+
+// The eight consumer warps: the stages in the producer's order.
+template <int D, int GT>
+__device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* sm, int* meta,
+                                               uint64_t* full, uint64_t* empty, int tid) {
+  using C = DecodeCfg<D, GT>;
+  constexpr int CPW = C::CPW;   // columns per warp (16 or 8)
+  constexpr int CGW = CPW / 4;  // 4-column groups per warp (phase 3)
+  constexpr int SL = 32 / CGW;  // token slices (phase 3)
+  float* sq = reinterpret_cast<float*>(sm + C::SQ_OFF);
+  float* sp = reinterpret_cast<float*>(sm + C::SP_OFF);
+  float* spp = reinterpret_cast<float*>(sm + C::P_OFF);
+  float* salpha = reinterpret_cast<float*>(sm + C::AL_OFF);
+  const int warp = tid >> 5, lane = tid & 31;
+  // running max / sum of head `warp` (warps < GT), the same in every lane
+  float m_run = -INFINITY, l_run = 0.f;
+  // p.V accumulators: head gh, columns col0 + {0,1} and + {2,3}
+  float2 acc[GT][2];
+#pragma unroll
+  for (int gh = 0; gh < GT; ++gh) acc[gh][0] = acc[gh][1] = make_float2(0.f, 0.f);
+  const int cg = lane % CGW, slice = lane / CGW;
+  const int col3 = warp * CPW + 4 * cg;  // phase 3 columns col3 .. col3+3
+  for (uint32_t k = 0;; ++k) {
+    const uint32_t s = k % C::NS;
+    bool ok = decode_wait(&full[s], (k / C::NS) & 1);
+    ok = ptx::bar_red_and(1, kDecodeConsumers, ok);
+    if (!ok) {
+      if (tid == 0) decode_error(p, kErrDecodeWait);
+      return;
+    }
+    const int* m = meta + 8 * s;
+    const int b = m[0];
+    if (b < 0) return;  // the producer's sentinel
+    const int gz = m[1], nt = m[3], flags = m[4], slot = m[5];
+    const int g = gz / p.zgroups, z = gz % p.zgroups;
+    const long long head0 = static_cast<long long>(b) * p.Hq + g * p.G + z * GT;
+    const uint8_t* st = sm + s * C::STAGE;
+    if (!(flags & kStageBad)) {
+      if (flags & kStageSegFirst) {
+        const __nv_bfloat16* sqb = reinterpret_cast<const __nv_bfloat16*>(st + C::KV_BYTES);
+        for (int i = tid; i < GT * D; i += kDecodeConsumers)
+          sq[i] = __bfloat162float(sqb[i]) * p.scale_log2;
+        ptx::bar_sync_named(1, kDecodeConsumers);
+      }
+      // 1. partial scores over this warp's CPW columns, tokens lane + 32 r;
+      // heads in groups of up to 4 (q of a group in registers)
+      constexpr int HG = GT < 4 ? GT : 4;
+#pragma unroll
+      for (int h0 = 0; h0 < GT; h0 += HG) {
+        float2 qp[HG][CPW / 2];
+#pragma unroll
+        for (int gh = 0; gh < HG; ++gh)
+#pragma unroll
+          for (int j = 0; j < CPW / 4; ++j) {
+            const float4 x =
+                *reinterpret_cast<const float4*>(sq + (h0 + gh) * D + warp * CPW + 4 * j);
+            qp[gh][2 * j] = make_float2(x.x, x.y);
+            qp[gh][2 * j + 1] = make_float2(x.z, x.w);
+          }
+#pragma unroll
+        for (int r = 0; r < C::CH / 32; ++r) {
+          const int t = lane + 32 * r;
+          if (t < nt) {
+            float2 kp[CPW / 2];
+#pragma unroll
+            for (int j = 0; j < CPW / 8; ++j) {
+              const int gc = warp * (CPW / 8) + j;  // 16-byte chunk (8 columns)
+              const uint4 u =
+                  *reinterpret_cast<const uint4*>(st + (gc >> 3) * C::HALF + sw128(t, gc & 7));
+              kp[4 * j] = bf16x2_to_f2(u.x);
+              kp[4 * j + 1] = bf16x2_to_f2(u.y);
+              kp[4 * j + 2] = bf16x2_to_f2(u.z);
+              kp[4 * j + 3] = bf16x2_to_f2(u.w);
+            }
+#pragma unroll
+            for (int gh = 0; gh < HG; ++gh) {
+              float2 a = __fmul2_rn(kp[0], qp[gh][0]);
+#pragma unroll
+              for (int j = 1; j < CPW / 2; ++j) a = __ffma2_rn(kp[j], qp[gh][j], a);
+              sp[(warp * GT + h0 + gh) * C::CH + t] = a.x + a.y;
+            }
+          }
+        }
+      }
+      ptx::bar_sync_named(1, kDecodeConsumers);
+
+      // 2. per head (warp gh): scores, running max, p = 2^(s - m), running sum
+      if (warp < GT) {
+        const int gh = warp;
+        float sv[C::CH / 32];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < C::CH / 32; ++j) {
+          const int t = lane + 32 * j;
+          float x = -INFINITY;
+          if (t < nt) {
+            x = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) x += sp[(w * GT + gh) * C::CH + t];
+          }
+          sv[j] = x;
+          mx = fmaxf(mx, x);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = ptx::ex2(m_run - m_new);  // 0 at a segment's first chunk
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < C::CH / 32; ++j) {
+          const float e = ptx::ex2(sv[j] - m_new);  // masked tokens: 2^-inf = 0
+          spp[(lane + 32 * j) * GT + gh] = e;
+          sum += e;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        l_run = fmaf(l_run, alpha, sum);
+        m_run = m_new;
+        if (lane == 0) salpha[gh] = alpha;
+      }
+      ptx::bar_sync_named(1, kDecodeConsumers);
+
+      // 3. acc = alpha * acc + sum_i p[i] v_i over this lane's token slice
+      {
+        const int gc = col3 >> 3;
+        const uint8_t* vb = st + (C::NH + (gc >> 3)) * C::HALF + ((col3 & 7) << 1);
+        const int cch = gc & 7;
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh) {
+          const float2 a2 = make_float2(salpha[gh], salpha[gh]);
+          acc[gh][0] = __fmul2_rn(acc[gh][0], a2);
+          acc[gh][1] = __fmul2_rn(acc[gh][1], a2);
+        }
+#pragma unroll 4
+        for (int i = slice; i < nt; i += SL) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vb + sw128(i, cch));
+          const float2 v01 = bf16x2_to_f2(u.x), v23 = bf16x2_to_f2(u.y);
+          float pw[GT];
+          if constexpr (GT >= 4) {
+#pragma unroll
+            for (int q4 = 0; q4 < GT / 4; ++q4) {
+              const float4 x = *reinterpret_cast<const float4*>(spp + i * GT + 4 * q4);
+              pw[4 * q4] = x.x;
+              pw[4 * q4 + 1] = x.y;
+              pw[4 * q4 + 2] = x.z;
+              pw[4 * q4 + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int gh = 0; gh < GT; ++gh) pw[gh] = spp[i * GT + gh];
+          }
+#pragma unroll
+          for (int gh = 0; gh < GT; ++gh) {
+            const float2 pp = make_float2(pw[gh], pw[gh]);
+            acc[gh][0] = __ffma2_rn(v01, pp, acc[gh][0]);
+            acc[gh][1] = __ffma2_rn(v23, pp, acc[gh][1]);
+          }
+        }
+      }
+    }
+    // every read of this stage is done: hand it back to the producer
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[s]);
+
+    if (flags & kStageSegLast) {
+      const long long base = head0 * p.nslot + slot;  // slot of head gh: + gh * nslot
+#pragma unroll
+      for (int msk = CGW; msk < 32; msk <<= 1)
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            acc[gh][e].x += __shfl_xor_sync(0xffffffffu, acc[gh][e].x, msk);
+            acc[gh][e].y += __shfl_xor_sync(0xffffffffu, acc[gh][e].y, msk);
+          }
+      if (slice == 0) {
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh)
+          *reinterpret_cast<float4*>(p.part_o + (base + gh * p.nslot) * D + col3) =
+              make_float4(acc[gh][0].x, acc[gh][0].y, acc[gh][1].x, acc[gh][1].y);
+      }
+#pragma unroll
+      for (int gh = 0; gh < GT; ++gh) acc[gh][0] = acc[gh][1] = make_float2(0.f, 0.f);
+      if (warp < GT) {
+        if (lane == 0) {
+          float* ml = p.part_ml + (base + warp * p.nslot) * 2;
+          ml[0] = m_run;
+          ml[1] = l_run;
+        }
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+      if ((flags & kStageItemLast) && tid == 0)
+        p.slots[static_cast<long long>(b) * p.Hkv * p.zgroups + gz] = slot + 1;
+    }
   }
 }
 
 template <int D, int GT>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, 1)
     paged_decode_partial_kernel(const __grid_constant__ CUtensorMap tm_k,
                                 const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using C = DecodeCfg<D, GT>;
   extern __shared__ uint8_t dsmem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  float* sq = reinterpret_cast<float*>(sm + C::Q_OFF);
-  float* sp = reinterpret_cast<float*>(sm + C::SP_OFF);
-  float* spp = reinterpret_cast<float*>(sm + C::P_OFF);
-  float* sml = reinterpret_cast<float*>(sm + C::ML_OFF);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
-  int* sflag = reinterpret_cast<int*>(sm + C::BAR_OFF + 16);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nch));
-  const int rest = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nch));
-  const int z = rest % p.zgroups;
-  const int bg = rest / p.zgroups;
-  const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int n = decode_len(p, b);
-  const int t0 = c * C::CH;
-  if (t0 >= n) return;  // past the sequence's last chunk: the merge reads nothing here
-  const int nt = min(C::CH, n - t0);
-  const int R = p.rows_per_box;
-  const int npg = (nt + R - 1) / R;  // boxes (pages or parts of one) the chunk needs, <= CH / 8
-  const long long head0 = static_cast<long long>(b) * p.Hq + g * p.G + z * GT;
-
-  // warp 0 reads the chunk's block ids and sets up the barriers
-  int blk = 0;
-  if (warp == 0) {
-    bool bad = false;
-    if (lane < npg) {
-      const int tok = t0 + lane * R;
-      blk = p.block_table[static_cast<long long>(b) * p.max_blocks + tok / p.bs];
-      bad = blk < 0 || blk >= p.num_blocks;
+  int* meta = reinterpret_cast<int*>(sm + C::META_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
+  uint64_t* empty = full + C::NS;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kDecodeConsumers / 32);
     }
-    const bool any_bad = __any_sync(0xffffffffu, bad);
-    if (lane == 0) {
-      *sflag = any_bad ? 1 : 0;
-      if (any_bad) decode_error(p, kErrDecodeInput);
-      ptx::mbar_init(&bar[0], 1);
-      ptx::mbar_init(&bar[1], 1);
-      ptx::fence_mbar_init();
-    }
+    ptx::fence_mbar_init();
   }
   __syncthreads();
-  if (*sflag) {  // a page of this chunk is not in the cache: the chunk contributes nothing
-    decode_empty_partial<GT>(p, head0, c);
-    return;
-  }
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(npg * R * D * 2);
-      ptx::mbar_arrive_expect_tx(&bar[0], bytes);
-      ptx::mbar_arrive_expect_tx(&bar[1], bytes);
-    }
-    __syncwarp();
-    if (lane < npg) {
-      const uint64_t pol = ptx::policy_evict_first();
-      const int tok = t0 + lane * R;
-      const int row = (blk * p.Hkv + g) * p.bs + tok % p.bs;
-#pragma unroll
-      for (int h = 0; h < C::NH; ++h)
-        ptx::tma_load_2d_hint(sm + C::K_OFF + h * C::HALF + lane * R * 128, &tm_k, &bar[0],
-                              64 * h, row, pol);
-#pragma unroll
-      for (int h = 0; h < C::NH; ++h)
-        ptx::tma_load_2d_hint(sm + C::V_OFF + h * C::HALF + lane * R * 128, &tm_v, &bar[1],
-                              64 * h, row, pol);
-    }
-  }
-  // q of the CTA's heads, in log2 units
-  for (int i = tid; i < GT * D; i += kDecodeThreads)
-    sq[i] = __bfloat162float(p.q[head0 * D + i]) * p.scale_log2;
-  __syncthreads();
-
-  bool ok = decode_wait(&bar[0], 0);
-  ok = __syncthreads_and(ok) != 0;
-  if (!ok) {
-    // record, let the copies in flight land (bounded), leave the partial empty
-    if (tid == 0) {
-      decode_error(p, kErrDecodeWait);
-      decode_wait(&bar[0], 0);
-      decode_wait(&bar[1], 0);
-    }
-    decode_empty_partial<GT>(p, head0, c);
-    return;
-  }
-
-  // 1. partial scores: thread = (column half, token)
-  {
-    const int part = warp >> 2;
-    const int t = ((warp & 3) << 5) | lane;
-    float s[GT];
-#pragma unroll
-    for (int gh = 0; gh < GT; ++gh) s[gh] = t < nt ? 0.f : -INFINITY;
-    if (t < nt) {
-#pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        const int gc = part * (D / 16) + j;  // 16-byte chunk of the row (8 columns)
-        const uint4 u = *reinterpret_cast<const uint4*>(sm + C::K_OFF + (gc >> 3) * C::HALF +
-                                                        sw128(t, gc & 7));
-        float kf[8];
-        bf16x8_to_f32(u, kf);
-#pragma unroll
-        for (int gh = 0; gh < GT; ++gh) {
-          const float4 qa = *reinterpret_cast<const float4*>(sq + gh * D + gc * 8);
-          const float4 qb = *reinterpret_cast<const float4*>(sq + gh * D + gc * 8 + 4);
-          s[gh] = fmaf(kf[0], qa.x, s[gh]);
-          s[gh] = fmaf(kf[1], qa.y, s[gh]);
-          s[gh] = fmaf(kf[2], qa.z, s[gh]);
-          s[gh] = fmaf(kf[3], qa.w, s[gh]);
-          s[gh] = fmaf(kf[4], qb.x, s[gh]);
-          s[gh] = fmaf(kf[5], qb.y, s[gh]);
-          s[gh] = fmaf(kf[6], qb.z, s[gh]);
-          s[gh] = fmaf(kf[7], qb.w, s[gh]);
-        }
-      }
-    }
-#pragma unroll
-    for (int gh = 0; gh < GT; ++gh) sp[(part * GT + gh) * C::CH + t] = s[gh];
-  }
-  // V must have landed before step 3; waiting here overlaps it with step 2
-  ok = decode_wait(&bar[1], 0);
-  ok = __syncthreads_and(ok) != 0;
-  if (!ok) {
-    if (tid == 0) decode_error(p, kErrDecodeWait);
-    decode_empty_partial<GT>(p, head0, c);
-    return;
-  }
-
-  // 2. per head (warp gh): chunk max m, p = 2^(s - m), l = sum p
-  if (warp < GT) {
-    const int gh = warp;
-    float sv[C::CH / 32];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < C::CH / 32; ++j) {
-      const int t = lane + 32 * j;
-      sv[j] = sp[gh * C::CH + t] + sp[(GT + gh) * C::CH + t];
-      mx = fmaxf(mx, sv[j]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < C::CH / 32; ++j) {
-      const float e = ptx::ex2(sv[j] - mx);  // masked tokens: 2^-inf = 0
-      spp[(lane + 32 * j) * GT + gh] = e;
-      sum += e;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane == 0) {
-      sml[gh] = mx;
-      sml[GT + gh] = sum;
-    }
-  }
-  __syncthreads();
-
-  // 3. o[gh][4cg .. 4cg+3] = sum_i p[i][gh] v_i: lanes over 4-column groups,
-  // token slices over warps (and lane halves when D = 64)
-  {
-    constexpr int LPR = D / 4;       // lanes per V row
-    constexpr int RPW = 32 / LPR;    // rows per warp step
-    constexpr int STRIDE = 8 * RPW;  // token stride of a slice
-    const int cg = lane % LPR;
-    const int r = lane / LPR;
-    const int gc = cg >> 1;
-    const uint32_t vcol =
-        static_cast<uint32_t>(C::V_OFF + (gc >> 3) * C::HALF + ((cg & 1) << 3));
-    float acc[GT][4];
-#pragma unroll
-    for (int gh = 0; gh < GT; ++gh) acc[gh][0] = acc[gh][1] = acc[gh][2] = acc[gh][3] = 0.f;
-#pragma unroll 4
-    for (int i = warp * RPW + r; i < nt; i += STRIDE) {
-      const uint2 u = *reinterpret_cast<const uint2*>(sm + vcol + sw128(i, gc & 7));
-      const float v0 = __uint_as_float(u.x << 16), v1 = __uint_as_float(u.x & 0xffff0000u);
-      const float v2 = __uint_as_float(u.y << 16), v3 = __uint_as_float(u.y & 0xffff0000u);
-      float pw[GT];
-      if constexpr (GT >= 4) {
-#pragma unroll
-        for (int q4 = 0; q4 < GT / 4; ++q4) {
-          const float4 x = *reinterpret_cast<const float4*>(spp + i * GT + 4 * q4);
-          pw[4 * q4] = x.x;
-          pw[4 * q4 + 1] = x.y;
-          pw[4 * q4 + 2] = x.z;
-          pw[4 * q4 + 3] = x.w;
-        }
-      } else {
-#pragma unroll
-        for (int gh = 0; gh < GT; ++gh) pw[gh] = spp[i * GT + gh];
-      }
-#pragma unroll
-      for (int gh = 0; gh < GT; ++gh) {
-        acc[gh][0] = fmaf(pw[gh], v0, acc[gh][0]);
-        acc[gh][1] = fmaf(pw[gh], v1, acc[gh][1]);
-        acc[gh][2] = fmaf(pw[gh], v2, acc[gh][2]);
-        acc[gh][3] = fmaf(pw[gh], v3, acc[gh][3]);
-      }
-    }
-    if constexpr (RPW == 2) {
-#pragma unroll
-      for (int gh = 0; gh < GT; ++gh)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[gh][e] += __shfl_xor_sync(0xffffffffu, acc[gh][e], 16);
-    }
-    float* red = reinterpret_cast<float*>(sm + C::K_OFF);  // K is no longer read
-    if (r == 0) {
-#pragma unroll
-      for (int gh = 0; gh < GT; ++gh)
-        *reinterpret_cast<float4*>(red + (warp * GT + gh) * D + 4 * cg) =
-            make_float4(acc[gh][0], acc[gh][1], acc[gh][2], acc[gh][3]);
-    }
-    __syncthreads();
-    if (tid < GT * D / 4) {
-      const int gh = tid / (D / 4), col = 4 * (tid % (D / 4));
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const float4 x = *reinterpret_cast<const float4*>(red + (w * GT + gh) * D + col);
-        a.x += x.x;
-        a.y += x.y;
-        a.z += x.z;
-        a.w += x.w;
-      }
-      *reinterpret_cast<float4*>(p.part_o + ((head0 + gh) * p.nch + c) * D + col) = a;
-    }
-    if (tid < GT) {
-      float* ml = p.part_ml + ((head0 + tid) * p.nch + c) * 2;
-      ml[0] = sml[tid];
-      ml[1] = sml[GT + tid];
-    }
-  }
+  if ((tid >> 5) == kDecodeProducerWarp)
+    decode_produce<D, GT>(&tm_k, &tm_v, p, sm, meta, full, empty, tid & 31);
+  else
+    decode_consume<D, GT>(p, sm, meta, full, empty, tid);
 }
 
-// A warp per (b, h): combine the sequence's chunks.  Lanes own D/32 columns.
+// A CTA per (b, h): warp w combines slots w, w + 8, ... (up to 8 at a time,
+// loads issued together), then the warps' sums are added.  Lanes own D/32
+// columns.
 template <int D>
 __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
   constexpr int PER = D / 32;
-  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= static_cast<long long>(p.B) * p.Hq) return;
-  const int b = static_cast<int>(wid / p.Hq);
+  __shared__ float sred[8][D];
+  __shared__ float sw[8];
+  const long long wid = blockIdx.x;  // b * Hq + h
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = static_cast<int>(wid / p.Hq), h = static_cast<int>(wid % p.Hq);
   const int n = decode_len(p, b);
-  const int nc = (n + kDecodeChunk - 1) / kDecodeChunk;
-  const float* ml = p.part_ml + wid * p.nch * 2;
+  int ns = 0;
+  if (n > 0) {
+    const int gt = p.G / p.zgroups;
+    const int gz = (h / p.G) * p.zgroups + (h % p.G) / gt;
+    ns = p.slots[static_cast<long long>(b) * p.Hkv * p.zgroups + gz];
+    if (ns < 1 || ns > p.nslot) {  // not written by this step: cannot happen for valid input
+      if (tid == 0) decode_error(p, kErrDecodeWait);
+      ns = 0;
+    }
+  }
+  const float* ml = p.part_ml + wid * p.nslot * 2;
   float M = -INFINITY;
-  for (int c = lane; c < nc; c += 32) M = fmaxf(M, ml[2 * c]);
+  for (int c = tid; c < ns; c += 256) M = fmaxf(M, ml[2 * c]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) sw[warp] = M;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, sw[w]);
+  __syncthreads();
   float L = 0.f;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  const float* po = p.part_o + wid * p.nch * D + lane * PER;
-  for (int c = 0; c < nc; ++c) {
-    const float m = ml[2 * c];
-    if (m == -INFINITY) continue;  // an empty chunk (its pages were not in the cache)
-    const float w = ptx::ex2(m - M);
-    L = fmaf(w, ml[2 * c + 1], L);
-    if constexpr (PER == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(po + static_cast<long long>(c) * D);
-      acc[0] = fmaf(w, x.x, acc[0]);
-      acc[1] = fmaf(w, x.y, acc[1]);
-      acc[2] = fmaf(w, x.z, acc[2]);
-      acc[3] = fmaf(w, x.w, acc[3]);
-    } else {
-      const float2 x = *reinterpret_cast<const float2*>(po + static_cast<long long>(c) * D);
-      acc[0] = fmaf(w, x.x, acc[0]);
-      acc[1] = fmaf(w, x.y, acc[1]);
+  const float* po = p.part_o + wid * p.nslot * D + lane * PER;
+  for (int c0 = warp; c0 < ns; c0 += 64) {
+    float mm[8], ll[8], x[8][PER];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + 8 * j;
+      mm[j] = -INFINITY;
+      ll[j] = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) x[j][e] = 0.f;
+      if (c < ns) {
+        mm[j] = ml[2 * c];
+        ll[j] = ml[2 * c + 1];
+        if constexpr (PER == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(po + static_cast<long long>(c) * D);
+          x[j][0] = v.x;
+          x[j][1] = v.y;
+          x[j][2] = v.z;
+          x[j][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(po + static_cast<long long>(c) * D);
+          x[j][0] = v.x;
+          x[j][1] = v.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (mm[j] != -INFINITY) {  // -inf: a segment whose chunks were all dropped
+        const float w = ptx::ex2(mm[j] - M);
+        L = fmaf(w, ll[j], L);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, x[j][e], acc[e]);
+      }
     }
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  __nv_bfloat16* dst = p.o + wid * D + lane * PER;
-  if constexpr (PER == 4) {
-    uint2 u;
-    u.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    u.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(dst) = u;
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+#pragma unroll
+  for (int e = 0; e < PER; ++e) sred[warp][lane * PER + e] = acc[e];
+  if (lane == 0) sw[warp] = L;
+  __syncthreads();
+  if (tid < D) {
+    float o = 0.f, Lt = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      o += sred[w][tid];
+      Lt += sw[w];
+    }
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    p.o[wid * D + tid] = __float2bfloat16_rn(o * inv);
+    if (tid == 0 && p.lse != nullptr)
+      p.lse[wid] = Lt > 0.f ? (M + ptx::lg2(Lt)) * 0.69314718055994530942f : -INFINITY;
   }
-  if (lane == 0 && p.lse != nullptr)
-    p.lse[wid] = L > 0.f ? (M + ptx::lg2(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
 }  // namespace tessera

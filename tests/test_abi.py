@@ -157,9 +157,11 @@ def call_decode(**kw):
 
 
 def test_decode_workspace_bytes(lib):
-    # partial outputs and (max, sum) pairs per (sequence, head, 128-token chunk)
-    assert tess.tessera_attn_decode_workspace_bytes(4, 8, 128, 128) == 4 * 8 * 1 * 130 * 4
-    assert tess.tessera_attn_decode_workspace_bytes(2, 4, 129, 64) == 2 * 4 * 2 * 66 * 4
+    # partial outputs and (max, sum) pairs per (sequence, head, 128-token slot),
+    # then an int per item (at most one per head), rounded up to 16 bytes
+    assert tess.tessera_attn_decode_workspace_bytes(4, 8, 128, 128) == 4 * 8 * 1 * 130 * 4 + 128
+    assert tess.tessera_attn_decode_workspace_bytes(2, 4, 129, 64) == 2 * 4 * 2 * 66 * 4 + 32
+    assert tess.tessera_attn_decode_workspace_bytes(1, 3, 1, 64) == 3 * 66 * 4 + 16
     assert tess.tessera_attn_decode_workspace_bytes(3, 4, 0, 64) == 0
     assert tess.tessera_attn_decode_workspace_bytes(1, 1, 1, 96) == 0
 
