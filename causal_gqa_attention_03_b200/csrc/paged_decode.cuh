@@ -330,10 +330,16 @@ __device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* s
   const int warp = tid >> 5, lane = tid & 31;
   // running max / sum of head `warp` (warps < GT), the same in every lane
   float m_run = -INFINITY, l_run = 0.f;
-  // p.V accumulators: head gh, columns col0 + {0,1} and + {2,3}
-  float2 acc[GT][2];
+  // p.V accumulators of columns col3 .. col3+3: one head (GT = 1) as column
+  // pairs acc[0][0..1]; else head pairs acc3[hp][e] = (head 2hp, 2hp+1) of
+  // column col3 + e
+  float2 acc[1][2];
+  float2 acc3[GT / 2 > 0 ? GT / 2 : 1][4];
+  acc[0][0] = acc[0][1] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int gh = 0; gh < GT; ++gh) acc[gh][0] = acc[gh][1] = make_float2(0.f, 0.f);
+  for (int hp = 0; hp < (GT / 2 > 0 ? GT / 2 : 1); ++hp)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc3[hp][e] = make_float2(0.f, 0.f);
   const int cg = lane % CGW, slice = lane / CGW;
   const int col3 = warp * CPW + 4 * cg;  // phase 3 columns col3 .. col3+3
   for (uint32_t k = 0;; ++k) {
@@ -359,30 +365,36 @@ __device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* s
         ptx::bar_sync_named(1, kDecodeConsumers);
       }
       // 1. partial scores over this warp's CPW columns, tokens lane + 32 r;
-      // heads in groups of up to 4 (q of a group in registers)
-      constexpr int HG = GT < 4 ? GT : 4;
+      // heads in groups of up to 4 (q of a group in registers).  Row t's
+      // swizzle phase is t & 7 = lane & 7, so a lane's K offsets are fixed.
+      {
+        constexpr int HG = GT < 4 ? GT : 4;
+        constexpr int KC = CPW / 8;  // 16-byte chunks per row slice
+        uint32_t koff[KC];
 #pragma unroll
-      for (int h0 = 0; h0 < GT; h0 += HG) {
-        float2 qp[HG][CPW / 2];
+        for (int j = 0; j < KC; ++j) {
+          const int gc = warp * KC + j;
+          koff[j] = static_cast<uint32_t>((gc >> 3) * C::HALF + lane * 128 +
+                                          (((gc & 7) ^ (lane & 7)) << 4));
+        }
+        const bool full_chunk = nt == C::CH;
 #pragma unroll
-        for (int gh = 0; gh < HG; ++gh)
+        for (int h0 = 0; h0 < GT; h0 += HG) {
+          float2 qp[HG][CPW / 2];
 #pragma unroll
-          for (int j = 0; j < CPW / 4; ++j) {
-            const float4 x =
-                *reinterpret_cast<const float4*>(sq + (h0 + gh) * D + warp * CPW + 4 * j);
-            qp[gh][2 * j] = make_float2(x.x, x.y);
-            qp[gh][2 * j + 1] = make_float2(x.z, x.w);
-          }
+          for (int gh = 0; gh < HG; ++gh)
 #pragma unroll
-        for (int r = 0; r < C::CH / 32; ++r) {
-          const int t = lane + 32 * r;
-          if (t < nt) {
+            for (int j = 0; j < CPW / 4; ++j) {
+              const float4 x =
+                  *reinterpret_cast<const float4*>(sq + (h0 + gh) * D + warp * CPW + 4 * j);
+              qp[gh][2 * j] = make_float2(x.x, x.y);
+              qp[gh][2 * j + 1] = make_float2(x.z, x.w);
+            }
+          auto token = [&](int r) {
             float2 kp[CPW / 2];
 #pragma unroll
-            for (int j = 0; j < CPW / 8; ++j) {
-              const int gc = warp * (CPW / 8) + j;  // 16-byte chunk (8 columns)
-              const uint4 u =
-                  *reinterpret_cast<const uint4*>(st + (gc >> 3) * C::HALF + sw128(t, gc & 7));
+            for (int j = 0; j < KC; ++j) {
+              const uint4 u = *reinterpret_cast<const uint4*>(st + koff[j] + r * 32 * 128);
               kp[4 * j] = bf16x2_to_f2(u.x);
               kp[4 * j + 1] = bf16x2_to_f2(u.y);
               kp[4 * j + 2] = bf16x2_to_f2(u.z);
@@ -390,11 +402,19 @@ __device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* s
             }
 #pragma unroll
             for (int gh = 0; gh < HG; ++gh) {
-              float2 a = __fmul2_rn(kp[0], qp[gh][0]);
+              float2 acc2 = __fmul2_rn(kp[0], qp[gh][0]);
 #pragma unroll
-              for (int j = 1; j < CPW / 2; ++j) a = __ffma2_rn(kp[j], qp[gh][j], a);
-              sp[(warp * GT + h0 + gh) * C::CH + t] = a.x + a.y;
+              for (int j = 1; j < CPW / 2; ++j) acc2 = __ffma2_rn(kp[j], qp[gh][j], acc2);
+              sp[(warp * GT + h0 + gh) * C::CH + lane + 32 * r] = acc2.x + acc2.y;
             }
+          };
+          if (full_chunk) {
+#pragma unroll
+            for (int r = 0; r < C::CH / 32; ++r) token(r);
+          } else {
+#pragma unroll
+            for (int r = 0; r < C::CH / 32; ++r)
+              if (lane + 32 * r < nt) token(r);
           }
         }
       }
@@ -437,41 +457,52 @@ __device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* s
       }
       ptx::bar_sync_named(1, kDecodeConsumers);
 
-      // 3. acc = alpha * acc + sum_i p[i] v_i over this lane's token slice
+      // 3. acc = alpha * acc + sum_i p[i] v_i over this lane's tokens
+      // i = slice + SL j, whose swizzle phase i & 7 = slice & 7 is fixed
       {
         const int gc = col3 >> 3;
-        const uint8_t* vb = st + (C::NH + (gc >> 3)) * C::HALF + ((col3 & 7) << 1);
-        const int cch = gc & 7;
+        const uint8_t* vl = st + (C::NH + (gc >> 3)) * C::HALF + ((col3 & 7) << 1) +
+                            slice * 128 + (((gc & 7) ^ (slice & 7)) << 4);
+        const float* pl = spp + slice * GT;
+        if constexpr (GT == 1) {
+          const float2 a2 = make_float2(salpha[0], salpha[0]);
+          acc[0][0] = __fmul2_rn(acc[0][0], a2);
+          acc[0][1] = __fmul2_rn(acc[0][1], a2);
+        } else {
 #pragma unroll
-        for (int gh = 0; gh < GT; ++gh) {
-          const float2 a2 = make_float2(salpha[gh], salpha[gh]);
-          acc[gh][0] = __fmul2_rn(acc[gh][0], a2);
-          acc[gh][1] = __fmul2_rn(acc[gh][1], a2);
+          for (int hp = 0; hp < GT / 2; ++hp) {
+            const float2 a2 = *reinterpret_cast<const float2*>(salpha + 2 * hp);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc3[hp][e] = __fmul2_rn(acc3[hp][e], a2);
+          }
         }
-#pragma unroll 4
-        for (int i = slice; i < nt; i += SL) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vb + sw128(i, cch));
-          const float2 v01 = bf16x2_to_f2(u.x), v23 = bf16x2_to_f2(u.y);
-          float pw[GT];
-          if constexpr (GT >= 4) {
-#pragma unroll
-            for (int q4 = 0; q4 < GT / 4; ++q4) {
-              const float4 x = *reinterpret_cast<const float4*>(spp + i * GT + 4 * q4);
-              pw[4 * q4] = x.x;
-              pw[4 * q4 + 1] = x.y;
-              pw[4 * q4 + 2] = x.z;
-              pw[4 * q4 + 3] = x.w;
-            }
+        auto token = [&](int j) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vl + j * SL * 128);
+          const float* pi = pl + j * SL * GT;
+          if constexpr (GT == 1) {
+            // column pairs, p duplicated
+            const float2 pp = make_float2(pi[0], pi[0]);
+            acc[0][0] = __ffma2_rn(bf16x2_to_f2(u.x), pp, acc[0][0]);
+            acc[0][1] = __ffma2_rn(bf16x2_to_f2(u.y), pp, acc[0][1]);
           } else {
+            // head pairs: p of two heads is one load, v duplicated
+            const float v[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u)};
 #pragma unroll
-            for (int gh = 0; gh < GT; ++gh) pw[gh] = spp[i * GT + gh];
-          }
+            for (int hp = 0; hp < GT / 2; ++hp) {
+              const float2 pp = *reinterpret_cast<const float2*>(pi + 2 * hp);
 #pragma unroll
-          for (int gh = 0; gh < GT; ++gh) {
-            const float2 pp = make_float2(pw[gh], pw[gh]);
-            acc[gh][0] = __ffma2_rn(v01, pp, acc[gh][0]);
-            acc[gh][1] = __ffma2_rn(v23, pp, acc[gh][1]);
+              for (int e = 0; e < 4; ++e)
+                acc3[hp][e] = __ffma2_rn(make_float2(v[e], v[e]), pp, acc3[hp][e]);
+            }
           }
+        };
+        if (nt == C::CH) {
+#pragma unroll
+          for (int j = 0; j < C::CH / SL; ++j) token(j);
+        } else {
+#pragma unroll 4
+          for (int j = 0; slice + j * SL < nt; ++j) token(j);
         }
       }
     }
@@ -481,23 +512,35 @@ __device__ __forceinline__ void decode_consume(const DecodeParams& p, uint8_t* s
 
     if (flags & kStageSegLast) {
       const long long base = head0 * p.nslot + slot;  // slot of head gh: + gh * nslot
+      float o4[GT][4];
+      if constexpr (GT == 1) {
+        o4[0][0] = acc[0][0].x;
+        o4[0][1] = acc[0][0].y;
+        o4[0][2] = acc[0][1].x;
+        o4[0][3] = acc[0][1].y;
+        acc[0][0] = acc[0][1] = make_float2(0.f, 0.f);
+      } else {
+#pragma unroll
+        for (int hp = 0; hp < GT / 2; ++hp)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o4[2 * hp][e] = acc3[hp][e].x;
+            o4[2 * hp + 1][e] = acc3[hp][e].y;
+            acc3[hp][e] = make_float2(0.f, 0.f);
+          }
+      }
 #pragma unroll
       for (int msk = CGW; msk < 32; msk <<= 1)
 #pragma unroll
         for (int gh = 0; gh < GT; ++gh)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            acc[gh][e].x += __shfl_xor_sync(0xffffffffu, acc[gh][e].x, msk);
-            acc[gh][e].y += __shfl_xor_sync(0xffffffffu, acc[gh][e].y, msk);
-          }
+          for (int e = 0; e < 4; ++e) o4[gh][e] += __shfl_xor_sync(0xffffffffu, o4[gh][e], msk);
       if (slice == 0) {
 #pragma unroll
         for (int gh = 0; gh < GT; ++gh)
           *reinterpret_cast<float4*>(p.part_o + (base + gh * p.nslot) * D + col3) =
-              make_float4(acc[gh][0].x, acc[gh][0].y, acc[gh][1].x, acc[gh][1].y);
+              make_float4(o4[gh][0], o4[gh][1], o4[gh][2], o4[gh][3]);
       }
-#pragma unroll
-      for (int gh = 0; gh < GT; ++gh) acc[gh][0] = acc[gh][1] = make_float2(0.f, 0.f);
       if (warp < GT) {
         if (lane == 0) {
           float* ml = p.part_ml + (base + warp * p.nslot) * 2;

@@ -199,15 +199,16 @@ def test_decode_bad_lengths_and_block_ids_are_reported():
     o, lse = run_decode(q, kc, vc, table, bad)
     assert tess.tessera_attn_device_error() == tess.DEVICE_ERR_DECODE_INPUT
     assert not o[2].any() and torch.equal(o[0], ref_o[0])
-    # a block id past the cache in sequence 0's second chunk (tokens 128..255)
+    # a block id past the cache among sequence 0's tokens 144..159 (the chunk
+    # holding it is dropped, the rest of the sequence still counts)
     t2 = table.copy()
     t2[0, 9] = kc.shape[0] + 1000
     o, lse = run_decode(q, kc, vc, t2, sl)
     assert tess.tessera_attn_device_error() == tess.DEVICE_ERR_DECODE_INPUT
     assert torch.all(torch.isfinite(o[0])) and torch.equal(o[1], ref_o[1])
-    # ... and a negative one
+    # ... and negative ones for every block of sequence 2 (all of it is dropped)
     t2 = table.copy()
-    t2[2, 0] = -7
+    t2[2, :(lens[2] + bs - 1) // bs] = -7
     o, lse = run_decode(q, kc, vc, t2, sl)
     assert tess.tessera_attn_device_error() == tess.DEVICE_ERR_DECODE_INPUT
     assert not o[2].any() and torch.equal(o[0], ref_o[0])
