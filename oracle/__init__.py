@@ -17,8 +17,10 @@ set and its torch fallback"), written out as its definition:
     LSE[b,h,i] = logsumexp_j(s_ij)            (natural log)
 
 and its exact gradient with respect to Q, K and V given dO (the chain rule
-through the row softmax; see the backward section of ``attn_ref.c``), and one
-decoding step over a paged key/value cache (the paged-decode section).
+through the row softmax; see the backward section of ``attn_ref.c``), one
+decoding step over a paged key/value cache (the paged-decode section), and
+the attention block's prologue: RMSNorm and the rotary embedding of the
+projected queries and keys (the prologue section).
 """
 from __future__ import annotations
 
@@ -94,6 +96,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_paged_decode_f64.argtypes = [dp, dp, dp, i32p, i32p, ci, ci, ci, ci, ci, ci, ci,
                                             ctypes.c_double, dp, dp]
     lib.oracle_paged_decode_f64.restype = ci
+    lib.oracle_rmsnorm_f64.argtypes = [dp, dp, ci, ci, ctypes.c_double, dp]
+    lib.oracle_rmsnorm_f64.restype = ci
+    lib.oracle_rope_qkv_f64.argtypes = [dp, i32p, ci, ci, ci, ci, ci, ctypes.c_double, dp, dp, dp]
+    lib.oracle_rope_qkv_f64.restype = ci
     return lib
 
 
@@ -253,3 +259,50 @@ def paged_decode_f64(q, k_cache, v_cache, block_table, seq_lens, scale: float | 
     if rc != 0:
         raise ValueError(f"oracle_paged_decode_f64 failed with code {rc}")
     return o, lse
+
+
+def rmsnorm_f64(x, w, eps: float = 1e-6, lib: ctypes.CDLL | None = None):
+    """RMSNorm over the last dimension in fp64: x [..., dim], w [dim]."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    dim = x.shape[-1]
+    if w.shape != (dim,):
+        raise ValueError("w must be [dim]")
+    rows = x.size // dim if dim else 0
+    y = np.zeros_like(x)
+    lib = lib or load()
+    rc = lib.oracle_rmsnorm_f64(_ptr(x, ctypes.c_double), _ptr(w, ctypes.c_double), rows, dim,
+                                float(eps), _ptr(y, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_rmsnorm_f64 failed with code {rc}")
+    return y
+
+
+def rope_qkv_f64(qkv, Hq: int, Hkv: int, positions=None, base: float = 10000.0,
+                 lib: ctypes.CDLL | None = None):
+    """Rotary embedding and head split in fp64.
+
+    qkv: [B, T, (Hq + 2 Hkv) * d]; positions: int32 [B, T] or None (p = t).
+    Returns (q [B,Hq,T,d], k [B,Hkv,T,d], v [B,Hkv,T,d]).
+    """
+    qkv = np.ascontiguousarray(qkv, dtype=np.float64)
+    B, T, width = qkv.shape
+    if width % (Hq + 2 * Hkv) != 0:
+        raise ValueError("qkv width must be (Hq + 2 Hkv) * d")
+    d = width // (Hq + 2 * Hkv)
+    pos = None
+    if positions is not None:
+        pos = np.ascontiguousarray(positions, dtype=np.int32)
+        if pos.shape != (B, T):
+            raise ValueError("positions must be [B, T]")
+    q = np.zeros((B, Hq, T, d))
+    k = np.zeros((B, Hkv, T, d))
+    v = np.zeros((B, Hkv, T, d))
+    lib = lib or load()
+    rc = lib.oracle_rope_qkv_f64(_ptr(qkv, ctypes.c_double),
+                                 _ptr(pos, ctypes.c_int32) if pos is not None else None,
+                                 B, T, Hq, Hkv, d, float(base), _ptr(q, ctypes.c_double),
+                                 _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_rope_qkv_f64 failed with code {rc}")
+    return q, k, v

@@ -413,3 +413,82 @@ int oracle_paged_decode_f64(const double *q, const double *k_cache, const double
     free(kh); free(vh); free(s);
     return 0;
 }
+
+/*
+ * ----------------------------------------------------------------------------
+ * Prologue of the attention block: RMSNorm, and the rotary embedding of the
+ * projected queries and keys.
+ *
+ * The pages' decoder is a transformer with "RMSNorm, RoPE, grouped-query
+ * attention and SwiGLU" (Tessera README, "What's in it" / "Training side"),
+ * and its kernels include a fused RMSNorm (README "What's in it" / "Kernels";
+ * hysenlabs.com review, "The kernel set and its torch fallback").  The pages
+ * give no formula; the plain readings written out here are the usual ones:
+ *
+ *   RMSNorm over the last dimension with a learned weight w:
+ *     y[r,c] = x[r,c] / sqrt( (1/dim) sum_c' x[r,c']^2 + eps ) * w[c]
+ *
+ *   Rotary position embedding of a head vector x (length d, even) at
+ *   position p, pairing element i with element i + d/2 (i < d/2):
+ *     theta_i = base^(-2i/d),   a = p * theta_i
+ *     y[i]       = x[i] cos a - x[i + d/2] sin a
+ *     y[i + d/2] = x[i] sin a + x[i + d/2] cos a
+ *
+ * The projection output is token-major: qkv [B, T, (Hq + 2 Hkv) d], per token
+ * the Hq query heads, then the Hkv key heads, then the Hkv value heads, each d
+ * wide.  The prologue writes the attention layout: q [B, Hq, T, d] and
+ * k [B, Hkv, T, d] rotated, v [B, Hkv, T, d] copied.  positions [B, T] gives
+ * each token's position (NULL: p = t).
+ */
+int oracle_rmsnorm_f64(const double *x, const double *w, int rows, int dim, double eps,
+                       double *y)
+{
+    if (rows < 0 || dim < 1 || !(eps >= 0.0)) return 1;
+    for (int r = 0; r < rows; ++r) {
+        const double *xr = x + (int64_t)r * dim;
+        double *yr = y + (int64_t)r * dim;
+        double ss = 0.0;
+        for (int c = 0; c < dim; ++c) ss += xr[c] * xr[c];
+        const double inv = 1.0 / sqrt(ss / dim + eps);
+        for (int c = 0; c < dim; ++c) yr[c] = xr[c] * inv * w[c];
+    }
+    return 0;
+}
+
+/* Rotate one head vector x (length d) at position p into y. */
+static void rope_one_head(const double *x, double p, int d, double base, double *y)
+{
+    const int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        const double theta = pow(base, -2.0 * i / d);
+        const double a = p * theta;
+        const double c = cos(a), s = sin(a);
+        y[i] = x[i] * c - x[i + half] * s;
+        y[i + half] = x[i] * s + x[i + half] * c;
+    }
+}
+
+int oracle_rope_qkv_f64(const double *qkv, const int32_t *positions, int B, int T, int Hq,
+                        int Hkv, int d, double base, double *q, double *k, double *v)
+{
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d < 2 || d % 2 != 0 || !(base > 0.0)) return 1;
+    const int H3 = Hq + 2 * Hkv;
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < T; ++t) {
+            const double *tok = qkv + ((int64_t)b * T + t) * H3 * d;
+            const double p = positions ? (double)positions[(int64_t)b * T + t] : (double)t;
+            for (int h = 0; h < Hq; ++h)
+                rope_one_head(tok + (int64_t)h * d, p, d, base,
+                              q + (((int64_t)b * Hq + h) * T + t) * d);
+            for (int h = 0; h < Hkv; ++h)
+                rope_one_head(tok + (int64_t)(Hq + h) * d, p, d, base,
+                              k + (((int64_t)b * Hkv + h) * T + t) * d);
+            for (int h = 0; h < Hkv; ++h) {
+                const double *src = tok + (int64_t)(Hq + Hkv + h) * d;
+                double *dst = v + (((int64_t)b * Hkv + h) * T + t) * d;
+                for (int c = 0; c < d; ++c) dst[c] = src[c];
+            }
+        }
+    }
+    return 0;
+}

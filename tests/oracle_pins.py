@@ -410,7 +410,109 @@ def pin_decode_invariants(lib):
         assert np.array_equal(fo[0, :, n - 1], o[b]) and np.array_equal(fl[0, :, n - 1], lse[b])
 
 
-ALL_PINS = [pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
+# ---------------------------------------------------------------- prologue
+def pin_rmsnorm_library(lib):
+    """torch's RMSNorm (float64) on random rows and weights, eps large enough
+    to matter."""
+    for seed, (rows, dim, eps, sigma) in enumerate([(5, 64, 1e-6, 1.0), (3, 128, 1e-2, 0.05),
+                                                     (4, 4096, 1e-5, 2.0), (2, 7, 0.5, 0.3)]):
+        x = _rand((rows, dim), 900 + seed, sigma)
+        w = _rand((dim,), 950 + seed)
+        got = oracle.rmsnorm_f64(x, w, eps, lib=lib)
+        want = torch.nn.functional.rms_norm(torch.from_numpy(x), (dim,),
+                                            weight=torch.from_numpy(w), eps=eps).numpy()
+        assert np.allclose(got, want, rtol=1e-13, atol=1e-15), (rows, dim, eps)
+
+
+def pin_rmsnorm_invariants(lib):
+    x = _rand((6, 32), 960)
+    w = _rand((32,), 961)
+    y = oracle.rmsnorm_f64(x, w, 0.0, lib=lib)
+    # scale invariance and oddness (eps = 0)
+    assert np.allclose(oracle.rmsnorm_f64(3.7 * x, w, 0.0, lib=lib), y, rtol=1e-13, atol=0)
+    assert np.array_equal(oracle.rmsnorm_f64(-x, w, 0.0, lib=lib), -y)
+    # unit root-mean-square before the weight
+    ones = oracle.rmsnorm_f64(x, np.ones(32), 0.0, lib=lib)
+    assert np.allclose(np.mean(ones ** 2, axis=1), 1.0, rtol=1e-13)
+    # a constant row c gives sign(c) * w
+    c = np.full((2, 32), -2.5)
+    assert np.allclose(oracle.rmsnorm_f64(c, w, 0.0, lib=lib), -np.tile(w, (2, 1)),
+                       rtol=1e-15, atol=1e-15)
+    # eps: a row of ones over eps = 3 gives 1 / sqrt(1 + 3) = 0.5 times w
+    assert np.allclose(oracle.rmsnorm_f64(np.ones((1, 32)), w, 3.0, lib=lib), 0.5 * w,
+                       rtol=1e-15, atol=0)
+
+
+def _rope_complex(x, pos, base):
+    """Rotary embedding as complex multiplication: z_i = x_i + j x_{i+d/2}
+    times exp(j p theta_i), theta_i = exp(-ln(base) 2i/d)."""
+    d = x.shape[-1]
+    half = d // 2
+    theta = np.exp(-np.log(base) * 2.0 * np.arange(half) / d)
+    z = x[..., :half] + 1j * x[..., half:]
+    r = z * np.exp(1j * pos[..., None] * theta)
+    return np.concatenate([r.real, r.imag], axis=-1)
+
+
+def pin_rope_complex(lib):
+    for seed, (B, T, Hq, Hkv, d, base, big) in enumerate([(2, 5, 4, 2, 8, 10000.0, False),
+                                                           (1, 7, 2, 1, 128, 10000.0, True),
+                                                           (2, 3, 3, 3, 64, 500000.0, True)]):
+        H3 = Hq + 2 * Hkv
+        qkv = _rand((B, T, H3 * d), 970 + seed)
+        pos = None
+        p = np.tile(np.arange(T, dtype=np.float64), (B, 1))
+        if big:
+            pos = np.random.default_rng(980 + seed).integers(0, 200000, size=(B, T)).astype(np.int32)
+            p = pos.astype(np.float64)
+        q, k, v = oracle.rope_qkv_f64(qkv, Hq, Hkv, positions=pos, base=base, lib=lib)
+        heads = qkv.reshape(B, T, H3, d)
+        want_q = _rope_complex(heads[:, :, :Hq], p[:, :, None], base).transpose(0, 2, 1, 3)
+        want_k = _rope_complex(heads[:, :, Hq:Hq + Hkv], p[:, :, None], base).transpose(0, 2, 1, 3)
+        # angles up to 2e5 rad: the two routes differ by the rounding of a * theta
+        tol = 1e-9 if big else 1e-13
+        assert np.allclose(q, want_q, rtol=0, atol=tol), (seed, np.abs(q - want_q).max())
+        assert np.allclose(k, want_k, rtol=0, atol=tol), (seed, np.abs(k - want_k).max())
+        assert np.array_equal(v, heads[:, :, Hq + Hkv:].transpose(0, 2, 1, 3))
+
+
+def pin_rope_invariants(lib):
+    B, T, Hq, Hkv, d = 2, 6, 2, 1, 16
+    qkv = _rand((B, T, (Hq + 2 * Hkv) * d), 990)
+    heads = qkv.reshape(B, T, Hq + 2 * Hkv, d)
+    # position 0 everywhere: the identity, exactly
+    q0, k0, _ = oracle.rope_qkv_f64(qkv, Hq, Hkv, positions=np.zeros((B, T), np.int32), lib=lib)
+    assert np.array_equal(q0, heads[:, :, :Hq].transpose(0, 2, 1, 3))
+    assert np.array_equal(k0, heads[:, :, Hq:Hq + Hkv].transpose(0, 2, 1, 3))
+    # no positions means p = t
+    q1, k1, v1 = oracle.rope_qkv_f64(qkv, Hq, Hkv, lib=lib)
+    pt = np.tile(np.arange(T, dtype=np.int32), (B, 1))
+    q2, k2, v2 = oracle.rope_qkv_f64(qkv, Hq, Hkv, positions=pt, lib=lib)
+    assert np.array_equal(q1, q2) and np.array_equal(k1, k2) and np.array_equal(v1, v2)
+    # each (i, i + d/2) pair keeps its length
+    xin = heads[:, :, :Hq].transpose(0, 2, 1, 3)
+    half = d // 2
+    assert np.allclose(q1[..., :half] ** 2 + q1[..., half:] ** 2,
+                       xin[..., :half] ** 2 + xin[..., half:] ** 2, rtol=1e-13)
+    # q.k depends on the positions only through their difference
+    base_pos = np.array([[3, 11, 40, 41, 100, 7]] * B, np.int32)
+    qa, ka, _ = oracle.rope_qkv_f64(qkv, Hq, Hkv, positions=base_pos, lib=lib)
+    qb, kb, _ = oracle.rope_qkv_f64(qkv, Hq, Hkv, positions=base_pos + 1234, lib=lib)
+    dots_a = np.einsum("bhtd,bsd->bhts", qa, ka[:, 0])
+    dots_b = np.einsum("bhtd,bsd->bhts", qb, kb[:, 0])
+    assert np.allclose(dots_a, dots_b, rtol=1e-9, atol=1e-9)
+    # d = 2: theta_0 = 1, a plain rotation by p radians
+    x = np.array([[[0.3, -1.2, 0.5, 0.25, 2.0, -0.75]]])  # B=1, T=1, Hq=1, Hkv=1, d=2
+    p = 3
+    q, k, v = oracle.rope_qkv_f64(x, 1, 1, positions=np.array([[p]], np.int32), lib=lib)
+    c, s_ = math.cos(p), math.sin(p)
+    assert np.allclose(q[0, 0, 0], [0.3 * c + 1.2 * s_, 0.3 * s_ - 1.2 * c], rtol=0, atol=1e-15)
+    assert np.allclose(k[0, 0, 0], [0.5 * c - 0.25 * s_, 0.5 * s_ + 0.25 * c], rtol=0, atol=1e-15)
+    assert np.array_equal(v[0, 0, 0], [2.0, -0.75])
+
+
+ALL_PINS = [pin_rmsnorm_library, pin_rmsnorm_invariants, pin_rope_complex,
+            pin_rope_invariants, pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
             pin_rows_entry, pin_bwd_library_autograd, pin_bwd_finite_differences,
             pin_bwd_invariants, pin_bwd_dq_rows_entry, pin_decode_library,
             pin_decode_invariants]

@@ -92,6 +92,20 @@ MUTATIONS = [
      "for (int h = g; h < Hq; h += Hkv) {"),
     ("decode drops the last token", "attend_one_row(q + row * d, kh, vh, n, d, scale, s, o + row * d, &lse[row]);",
      "attend_one_row(q + row * d, kh, vh, n > 1 ? n - 1 : n, d, scale, s, o + row * d, &lse[row]);"),
+    # prologue
+    ("RMSNorm without eps", "1.0 / sqrt(ss / dim + eps)", "1.0 / sqrt(ss / dim)"),
+    ("RMSNorm over the sum, not the mean", "1.0 / sqrt(ss / dim + eps)", "1.0 / sqrt(ss + eps)"),
+    ("RMSNorm weight dropped", "yr[c] = xr[c] * inv * w[c];", "yr[c] = xr[c] * inv;"),
+    ("RoPE rotates the other way", "y[i] = x[i] * c - x[i + half] * s;",
+     "y[i] = x[i] * c + x[i + half] * s;"),
+    ("RoPE pairs neighbours instead of halves", "y[i + half] = x[i] * s + x[i + half] * c;",
+     "y[i + half] = x[i] * s + x[i + half] * c; if (i % 2 == 1) { double t_ = y[i]; y[i] = y[i - 1]; y[i - 1] = t_; }"),
+    ("RoPE frequency exponent i / d", "pow(base, -2.0 * i / d)", "pow(base, -1.0 * i / d)"),
+    ("RoPE positions off by one", ": (double)t;", ": (double)t + 1.0;"),
+    ("RoPE leaves the keys unrotated",
+     "rope_one_head(tok + (int64_t)(Hq + h) * d, p, d, base,", "rope_one_head(tok + (int64_t)(Hq + h) * d, 0.0, d, base,"),
+    ("value heads taken from the key slot", "const double *src = tok + (int64_t)(Hq + Hkv + h) * d;",
+     "const double *src = tok + (int64_t)(Hq + h) * d;"),
 ]
 
 
