@@ -294,6 +294,68 @@ def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
 
 
+def time_prologue(w, steps, warmup, flush, stream, tess, torch, dev):
+    """RMSNorm of the hidden states [B*T, Hq*d] and the rotary embedding with
+    head split of the projection output [B, T, (Hq + 2 Hkv) d], at the
+    workload's sizes, each timed alone (one launch per step, L2 flushed
+    before each).  Returns {name: (per-step ms list, bytes per step)}."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 17)
+    dm = w.Hq * w.d
+    rows = w.B * w.T
+    x = torch.randn((rows, dm), generator=g, device=dev).to(torch.bfloat16)
+    wn = torch.randn((dm,), generator=g, device=dev).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    h3 = w.Hq + 2 * w.Hkv
+    qkv = torch.randn((w.B, w.T, h3 * w.d), generator=g, device=dev).to(torch.bfloat16)
+    q = torch.empty((w.B, w.Hq, w.T, w.d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    legs = {
+        "rmsnorm": (lambda: tess.rmsnorm(x, wn, 1e-6, out=y, stream=stream),
+                    2 * rows * dm * 2 + dm * 2),
+        "rope_qkv": (lambda: tess.rope_qkv(qkv, w.Hq, w.Hkv, q=q, k=k, v=v, stream=stream),
+                     2 * w.B * w.T * h3 * w.d * 2),
+    }
+    out = {}
+    for name, (call, nbytes) in legs.items():
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        torch.cuda.synchronize()
+        launches = 0
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            call()
+            launches += tess.tessera_attn_last_launch_count()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        out[name] = ([s_.elapsed_time(e) for s_, e in zip(starts, ends)], nbytes, launches)
+    del x, wn, y, qkv, q, k, v
+    return out
+
+
+def prologue_line(w, res, peaks, peak_src):
+    hbm = float(peaks["hbm_gbs"])
+    line = {"metric": "attention prologue GB/s (bf16): RMSNorm, RoPE + head split",
+            "config": {"rows": w.B * w.T, "hidden": w.Hq * w.d, "B": w.B, "T": w.T, "Hq": w.Hq,
+                       "Hkv": w.Hkv, "d": w.d, "eps": 1e-6, "rope_base": 10000.0,
+                       "positions": "t (none given)"},
+            "l2": "flushed before every timed step"}
+    for name, (times, nbytes, launches) in res.items():
+        ms = statistics.median(times)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        line[name] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 5),
+                      "bytes_per_step": nbytes, "gpu_launches": launches,
+                      "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                   "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                   "peak_source": f"{peak_src} hbm_gbs"}}
+    return line
+
+
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
     tessera_attn_fwd_host (copies pipelined with the kernels over key/value-head
@@ -425,6 +487,9 @@ def main():
     if err != 0:
         raise SystemExit(f"device-side error in the decode step (code {err})")
 
+    # the prologue kernels at the workload's sizes
+    pro = time_prologue(w, max(5, min(args.steps, 100)), 3, flush, stream, tess, torch, dev)
+
     sweep = {}
     if not args.no_sweep and world == 1:
         for name, ws in inputs.WORKLOADS.items():
@@ -505,6 +570,7 @@ def main():
                      "l2": "flushed before every timed step"},
         "decode": decode_line(wd, dec_times, dec_max_ms, dec_steps, dec_launches, dec_ws, world,
                               peaks, peak_src),
+        "prologue": prologue_line(w, pro, peaks, peak_src),
         "clocks": clk,
         "sweep": sweep or None,
     }

@@ -10,7 +10,8 @@ Raw C-ABI names (integer pointers, sizes, stream handle):
     tessera_status_str, tessera_attn_last_launch_count,
     tessera_attn_selftest_timeout, tessera_attn_bwd, tessera_attn_bwd_workspace_bytes,
     tessera_attn_bwd_noalloc, tessera_attn_bwd_noalloc_max_workspace_bytes,
-    tessera_attn_decode, tessera_attn_decode_workspace_bytes
+    tessera_attn_decode, tessera_attn_decode_workspace_bytes, tessera_rmsnorm,
+    tessera_rope_qkv
 Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
     attn_fwd_host(q, k, v, causal=True, scale=None, out=None, lse=None,
@@ -19,6 +20,8 @@ Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_bwd_noalloc(q, k, v, o, lse, dout, causal=True, scale=None, stream=None)
     attn_decode(q, k_cache, v_cache, block_table, seq_lens, max_seq_len=None,
                 scale=None, stream=None)
+    rmsnorm(x, w, eps=1e-6, out=None, stream=None)
+    rope_qkv(qkv, Hq, Hkv, positions=None, base=10000.0, stream=None)
 """
 from __future__ import annotations
 
@@ -35,7 +38,7 @@ EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
             "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
             "tessera_attn_selftest_timeout", "tessera_attn_decode",
-            "tessera_attn_decode_workspace_bytes")
+            "tessera_attn_decode_workspace_bytes", "tessera_rmsnorm", "tessera_rope_qkv")
 
 # Device error code recorded by tessera_attn_selftest_timeout.
 DEVICE_ERR_SELFTEST = 9
@@ -98,6 +101,11 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_decode.restype = ci
             lib.tessera_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci]
             lib.tessera_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+            lib.tessera_rmsnorm.argtypes = [vp, vp, vp, ci, ci, ctypes.c_float, vp]
+            lib.tessera_rmsnorm.restype = ci
+            lib.tessera_rope_qkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                             ctypes.c_float, vp]
+            lib.tessera_rope_qkv.restype = ci
             _lib = lib
     return _lib
 
@@ -162,6 +170,21 @@ def tessera_attn_decode(q: int, k_cache: int, v_cache: int, block_table: int, se
 
 def tessera_attn_decode_workspace_bytes(B: int, Hq: int, max_seq_len: int, d: int) -> int:
     return load_library().tessera_attn_decode_workspace_bytes(B, Hq, max_seq_len, d)
+
+
+def tessera_rmsnorm(x: int, w: int, y: int, rows: int, dim: int, eps: float,
+                    stream: int | None) -> int:
+    """The RMSNorm C entry point with integer device pointers; returns the status."""
+    return load_library().tessera_rmsnorm(x or None, w or None, y or None, rows, dim,
+                                          float(eps), stream or None)
+
+
+def tessera_rope_qkv(qkv: int, positions: int | None, q: int, k: int, v: int, B: int, T: int,
+                     Hq: int, Hkv: int, d: int, base: float, stream: int | None) -> int:
+    """The rotary-embedding C entry point with integer device pointers; returns the status."""
+    return load_library().tessera_rope_qkv(qkv or None, positions or None, q or None, k or None,
+                                           v or None, B, T, Hq, Hkv, d, float(base),
+                                           stream or None)
 
 
 def tessera_attn_device_error() -> int:
@@ -392,3 +415,61 @@ def attn_decode(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int | N
     if st != 0:
         raise TesseraError(st, "tessera_attn_decode")
     return out, lse
+
+
+def rmsnorm(x, w, eps: float = 1e-6, out=None, stream=None):
+    """RMSNorm over the last dimension of a CUDA bf16 tensor x with weight w
+    (bf16 [dim]).  Returns out (allocated unless given; may be x itself)."""
+    import torch
+
+    for name, t in (("x", x), ("w", w)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    dim = x.shape[-1]
+    if tuple(w.shape) != (dim,):
+        raise ValueError("w must be [dim]")
+    if out is None:
+        out = torch.empty_like(x)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    st = tessera_rmsnorm(x.data_ptr(), w.data_ptr(), out.data_ptr(), x.numel() // dim, dim,
+                         float(eps), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_rmsnorm")
+    return out
+
+
+def rope_qkv(qkv, Hq: int, Hkv: int, positions=None, base: float = 10000.0, q=None, k=None,
+             v=None, stream=None):
+    """Rotary embedding and head split of a CUDA bf16 projection output
+    qkv [B, T, (Hq + 2 Hkv) d]; positions int32 [B, T] or None (p = t).
+    Returns (q [B,Hq,T,d], k [B,Hkv,T,d], v [B,Hkv,T,d])."""
+    import torch
+
+    if not isinstance(qkv, torch.Tensor) or qkv.dtype != torch.bfloat16 or not qkv.is_cuda:
+        raise TypeError("qkv must be a CUDA bf16 tensor")
+    if qkv.dim() != 3 or not qkv.is_contiguous():
+        raise ValueError("qkv must be a contiguous [B, T, (Hq + 2 Hkv) d] tensor")
+    B, T, width = qkv.shape
+    if width % (Hq + 2 * Hkv) != 0:
+        raise ValueError("qkv width must be (Hq + 2 Hkv) * d")
+    d = width // (Hq + 2 * Hkv)
+    if positions is not None:
+        if (not isinstance(positions, torch.Tensor) or positions.dtype != torch.int32
+                or not positions.is_cuda or tuple(positions.shape) != (B, T)
+                or not positions.is_contiguous()):
+            raise ValueError("positions must be a contiguous CUDA int32 [B, T] tensor")
+    dev = qkv.device
+    q = torch.empty((B, Hq, T, d), dtype=torch.bfloat16, device=dev) if q is None else q
+    k = torch.empty((B, Hkv, T, d), dtype=torch.bfloat16, device=dev) if k is None else k
+    v = torch.empty((B, Hkv, T, d), dtype=torch.bfloat16, device=dev) if v is None else v
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    st = tessera_rope_qkv(qkv.data_ptr(), positions.data_ptr() if positions is not None else None,
+                          q.data_ptr(), k.data_ptr(), v.data_ptr(), B, T, Hq, Hkv, d,
+                          float(base), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_rope_qkv")
+    return q, k, v

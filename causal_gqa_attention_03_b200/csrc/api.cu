@@ -18,6 +18,7 @@
 #include "attn_fwd_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
 #include "paged_decode.cuh"
+#include "prologue.cuh"
 
 namespace {
 
@@ -638,6 +639,87 @@ extern "C" int tessera_attn_decode(const void* q, const void* k_cache, const voi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) return launch_decode_d<64>(k_cache, v_cache, p, s);
   return launch_decode_d<128>(k_cache, v_cache, p, s);
+}
+
+extern "C" int tessera_rmsnorm(const void* x, const void* w, void* y, int rows, int dim,
+                               float eps, tessera_stream_t stream) {
+  g_last_launches = 0;
+  if (rows < 0 || dim < 1 || !(eps >= 0.f) || !std::isfinite(eps)) return TESSERA_ERR_INVALID_ARG;
+  if (dim % 8 != 0 || dim > tessera::kNormMaxVec * 32 * 8) return TESSERA_ERR_UNSUPPORTED;
+  if (rows == 0) return TESSERA_OK;
+  if (!x || !w || !y) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return TESSERA_ERR_MISALIGNED;
+  const size_t bytes = static_cast<size_t>(rows) * dim * 2;
+  // in place (y == x) is allowed; any other overlap is not
+  if ((y != x && overlaps(y, bytes, x, bytes)) || overlaps(y, bytes, w, static_cast<size_t>(dim) * 2))
+    return TESSERA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  const int sms = sm_count(dev);
+  if (sms <= 0) return TESSERA_ERR_CUDA;
+  const long long blocks = (static_cast<long long>(rows) + 7) / 8;  // a warp per row
+  const long long cap = static_cast<long long>(sms) * 8;           // 8 CTAs of 256 per SM
+  const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* wb = static_cast<const __nv_bfloat16*>(w);
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  const int vpt = (dim / 8 + 31) / 32;  // 16-byte vectors per lane
+  if (vpt <= 4)
+    tessera::rmsnorm_kernel<4><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
+  else if (vpt <= 8)
+    tessera::rmsnorm_kernel<8><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
+  else if (vpt <= 16)
+    tessera::rmsnorm_kernel<16><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
+  else
+    tessera::rmsnorm_kernel<32><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  g_last_launches = 1;
+  return TESSERA_OK;
+}
+
+extern "C" int tessera_rope_qkv(const void* qkv, const int32_t* positions, void* q, void* k,
+                                void* v, int B, int T, int Hq, int Hkv, int d, float base,
+                                tessera_stream_t stream) {
+  g_last_launches = 0;
+  if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TESSERA_ERR_INVALID_ARG;
+  if (!(base > 0.f) || !std::isfinite(base)) return TESSERA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TESSERA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return TESSERA_OK;
+  if (!qkv || !q || !k || !v) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return TESSERA_ERR_MISALIGNED;
+  const long long tokens = static_cast<long long>(B) * T;
+  const long long tiles = (static_cast<long long>(T) + tessera::kRopeTokens - 1) / tessera::kRopeTokens;
+  if (B * tiles > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  const size_t in_bytes = static_cast<size_t>(tokens) * (Hq + 2 * Hkv) * d * 2;
+  const size_t q_bytes = static_cast<size_t>(tokens) * Hq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(tokens) * Hkv * d * 2;
+  const size_t pos_bytes = positions ? static_cast<size_t>(tokens) * 4 : 0;
+  const void* outs[3] = {q, k, v};
+  const size_t out_bytes[3] = {q_bytes, kv_bytes, kv_bytes};
+  for (int a = 0; a < 3; ++a) {
+    if (overlaps(outs[a], out_bytes[a], qkv, in_bytes) ||
+        overlaps(outs[a], out_bytes[a], positions, pos_bytes))
+      return TESSERA_ERR_INVALID_ARG;
+    for (int b2 = a + 1; b2 < 3; ++b2)
+      if (overlaps(outs[a], out_bytes[a], outs[b2], out_bytes[b2])) return TESSERA_ERR_INVALID_ARG;
+  }
+  const double log2_base = std::log2(static_cast<double>(base));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(B * tiles);
+  if (d == 64)
+    tessera::rope_qkv_kernel<64><<<grid, tessera::kRopeThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(qkv), positions, static_cast<__nv_bfloat16*>(q),
+        static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v), B, T, Hq, Hkv, log2_base);
+  else
+    tessera::rope_qkv_kernel<128><<<grid, tessera::kRopeThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(qkv), positions, static_cast<__nv_bfloat16*>(q),
+        static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v), B, T, Hq, Hkv, log2_base);
+  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  g_last_launches = 1;
+  return TESSERA_OK;
 }
 
 extern "C" int tessera_attn_device_error(int* code) {

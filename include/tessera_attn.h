@@ -35,7 +35,7 @@ typedef struct CUstream_st *tessera_stream_t;
 typedef enum {
     TESSERA_OK = 0,
     TESSERA_ERR_INVALID_ARG = 1, /* bad size, null pointer, aliasing, bad scale */
-    TESSERA_ERR_UNSUPPORTED = 2, /* head dimension not 64/128; decode block size */
+    TESSERA_ERR_UNSUPPORTED = 2, /* head dim not 64/128; decode block size; norm width */
     TESSERA_ERR_MISALIGNED = 3,  /* a pointer not 16-byte aligned */
     TESSERA_ERR_CUDA = 4,        /* the CUDA runtime reported an error */
     TESSERA_ERR_TIMEOUT = 5,     /* a device-side wait gave up (see below) */
@@ -217,6 +217,56 @@ int tessera_attn_decode(const void *q, const void *k_cache, const void *v_cache,
                         int max_seq_len, float scale, tessera_stream_t stream);
 
 /*
+ * The attention block's prologue: the steps before attention in the pages'
+ * decoder ("RMSNorm, RoPE, grouped-query attention and SwiGLU", Tessera
+ * README, "What's in it" / "Training side"; its kernels include a fused
+ * RMSNorm, README "What's in it" / "Kernels" and hysenlabs.com review, "The
+ * kernel set and its torch fallback").  The pages give no formula; the plain
+ * readings adopted here:
+ *
+ *   RMSNorm:  y[r,c] = x[r,c] / sqrt(mean_c x[r,c]^2 + eps) * w[c]
+ *   RoPE of a head vector at position p, element i paired with i + d/2:
+ *     theta_i = base^(-2i/d), a = p * theta_i
+ *     y[i] = x[i] cos a - x[i+d/2] sin a,  y[i+d/2] = x[i] sin a + x[i+d/2] cos a
+ *
+ * Between the two runs the Q/K/V projection, a plain GEMM that is not part of
+ * this library.  Both calls are asynchronous on `stream`, launch one kernel
+ * (tessera_attn_last_launch_count() = 1, 0 when there is nothing to do),
+ * allocate nothing, and check their arguments before any CUDA call.
+ *
+ * tessera_rmsnorm
+ *   x    bf16 [rows, dim] device, read only
+ *   w    bf16 [dim] device, read only
+ *   y    bf16 [rows, dim] device, written (rounded to nearest even); may be x
+ *        itself (in place), must not otherwise overlap x or w
+ *   rows >= 0 (0 launches nothing); dim a multiple of 8 up to 8192, else
+ *   TESSERA_ERR_UNSUPPORTED; eps >= 0 and finite.  Pointers 16-byte aligned.
+ *   Sums of squares in fp32.
+ */
+int tessera_rmsnorm(const void *x, const void *w, void *y, int rows, int dim, float eps,
+                    tessera_stream_t stream);
+
+/*
+ * tessera_rope_qkv: rotary embedding of the projected queries and keys, and
+ * the split into the layout tessera_attn_fwd reads.
+ *   qkv        bf16 [B, T, (Hq + 2*Hkv) * d] device, read only: per token the
+ *              Hq query heads, then the Hkv key heads, then the Hkv value
+ *              heads (the projection's output, token-major)
+ *   positions  int32 [B, T] device, each token's position; NULL means p = t
+ *   q          bf16 [B, Hq, T, d] device, written: rotated query heads
+ *   k, v       bf16 [B, Hkv, T, d] device, written: rotated key heads, and the
+ *              value heads copied
+ *   B, T >= 0 (either 0 launches nothing); Hq, Hkv >= 1, Hq % Hkv == 0;
+ *   d 64 or 128, else TESSERA_ERR_UNSUPPORTED; base > 0 and finite (10000 is
+ *   the usual choice).  Pointers 16-byte aligned (positions 4-byte); q, k, v
+ *   must not overlap qkv, positions or each other.  Angles are computed in
+ *   fp64, the rotation in fp32.
+ */
+int tessera_rope_qkv(const void *qkv, const int32_t *positions, void *q, void *k, void *v,
+                     int B, int T, int Hq, int Hkv, int d, float base,
+                     tessera_stream_t stream);
+
+/*
  * Reads and clears the device-side error word of the current device.  This
  * synchronises the device.  *code receives 0 when no kernel reported a
  * problem since the last call, else a nonzero code naming the wait that gave
@@ -241,8 +291,9 @@ const char *tessera_status_str(int status);
 
 /*
  * Kernel launches the last successful tessera_attn_fwd (0 or 1),
- * tessera_attn_fwd_host (one per chunk), tessera_attn_bwd (3) or
- * tessera_attn_decode (1 or 2) call on this thread queued.  Lets a caller
+ * tessera_attn_fwd_host (one per chunk), tessera_attn_bwd (3),
+ * tessera_attn_decode (1 or 2), tessera_rmsnorm or tessera_rope_qkv (1) call
+ * on this thread queued.  Lets a caller
  * count the library's own launches.
  */
 int tessera_attn_last_launch_count(void);

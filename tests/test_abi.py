@@ -186,6 +186,43 @@ def test_decode_argument_checks_before_any_cuda_call(lib, kw, status):
     assert tess.tessera_attn_last_launch_count() == 0
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(rows=-1), 1), (dict(dim=0), 1), (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1),
+    (dict(dim=12), 2), (dict(dim=8200), 2), (dict(dim=16384), 2),
+    (dict(x=0), 1), (dict(w=0), 1), (dict(y=0), 1),
+    (dict(x=ALIGNED + 8), 3), (dict(y=ALIGNED + 0x1000004), 3),
+    (dict(y=ALIGNED + 0x40), 1),                     # y overlaps x (not in place)
+    (dict(w=ALIGNED + 0x1000000 + 64), 1),           # w inside y
+    (dict(rows=0), 0),
+])
+def test_rmsnorm_argument_checks_before_any_cuda_call(lib, kw, status):
+    a = dict(x=ALIGNED, w=ALIGNED + 0x2000000, y=ALIGNED + 0x1000000, rows=16, dim=4096,
+             eps=1e-6)
+    a.update(kw)
+    assert tess.tessera_rmsnorm(a["x"], a["w"], a["y"], a["rows"], a["dim"], a["eps"],
+                                None) == status
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(T=-1), 1), (dict(Hq=6, Hkv=4), 1), (dict(Hkv=0), 1),
+    (dict(d=96), 2), (dict(d=32), 2), (dict(base=0.0), 1), (dict(base=float("nan")), 1),
+    (dict(qkv=0), 1), (dict(q=0), 1), (dict(k=0), 1), (dict(v=0), 1),
+    (dict(qkv=ALIGNED + 4), 3), (dict(k=ALIGNED + 0x2000008), 3), (dict(pos=ALIGNED + 0x5000002), 3),
+    (dict(q=ALIGNED + 0x100), 1),                    # q overlaps qkv
+    (dict(v=ALIGNED + 0x1000000), 1),                # v overlaps q
+    (dict(pos=ALIGNED + 0x2000000), 1),              # positions inside k
+    (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_rope_argument_checks_before_any_cuda_call(lib, kw, status):
+    a = dict(qkv=ALIGNED, pos=ALIGNED + 0x5000000, q=ALIGNED + 0x1000000, k=ALIGNED + 0x2000000,
+             v=ALIGNED + 0x3000000, B=2, T=100, Hq=8, Hkv=2, d=128, base=10000.0)
+    a.update(kw)
+    assert tess.tessera_rope_qkv(a["qkv"], a["pos"], a["q"], a["k"], a["v"], a["B"], a["T"],
+                                 a["Hq"], a["Hkv"], a["d"], a["base"], None) == status
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
 @pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
     assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1
