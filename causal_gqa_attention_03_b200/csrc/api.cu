@@ -658,7 +658,7 @@ extern "C" int tessera_rmsnorm(const void* x, const void* w, void* y, int rows, 
   const int sms = sm_count(dev);
   if (sms <= 0) return TESSERA_ERR_CUDA;
   const long long blocks = (static_cast<long long>(rows) + 7) / 8;  // a warp per row
-  const long long cap = static_cast<long long>(sms) * 8;           // 8 CTAs of 256 per SM
+  const long long cap = static_cast<long long>(sms) * 32;  // beyond residency: the scheduler balances
   const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);

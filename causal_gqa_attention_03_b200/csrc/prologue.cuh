@@ -134,32 +134,46 @@ __global__ void __launch_bounds__(kRopeThreads)
   }
   const int H3 = Hq + 2 * Hkv;
   const __nv_bfloat16* tok = qkv + bt * H3 * D;
-  for (int h = hc; h < H3; h += HS) {
-    const uint4 lo = ld_stream_v4(tok + h * D + 8 * c);
-    const uint4 hi = ld_stream_v4(tok + h * D + D / 2 + 8 * c);
-    __nv_bfloat16* dst;
-    uint4 olo = lo, ohi = hi;
-    if (h < Hq + Hkv) {
-      const uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
-      const uint32_t bb[4] = {hi.x, hi.y, hi.z, hi.w};
-      uint32_t ol[4], oh[4];
+  // the thread's heads in groups of 4, each group's loads issued together
+  for (int h0 = hc; h0 < H3; h0 += 4 * HS) {
+    uint4 lo4[4], hi4[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = bf_lo(a[e]), x1 = bf_hi(a[e]);      // elements i, i+1
-        const float y0 = bf_lo(bb[e]), y1 = bf_hi(bb[e]);    // elements i+D/2, i+1+D/2
-        const float c0 = cs[2 * e], s0 = sn[2 * e], c1 = cs[2 * e + 1], s1 = sn[2 * e + 1];
-        ol[e] = pack_bf2(fmaf(x0, c0, -y0 * s0), fmaf(x1, c1, -y1 * s1));
-        oh[e] = pack_bf2(fmaf(x0, s0, y0 * c0), fmaf(x1, s1, y1 * c1));
+    for (int u = 0; u < 4; ++u) {
+      const int h = h0 + u * HS;
+      if (h < H3) {
+        lo4[u] = ld_stream_v4(tok + h * D + 8 * c);
+        hi4[u] = ld_stream_v4(tok + h * D + D / 2 + 8 * c);
       }
-      olo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-      ohi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-      dst = h < Hq ? q + ((static_cast<long long>(b) * Hq + h) * T + t) * D
-                   : k + ((static_cast<long long>(b) * Hkv + (h - Hq)) * T + t) * D;
-    } else {
-      dst = v + ((static_cast<long long>(b) * Hkv + (h - Hq - Hkv)) * T + t) * D;
     }
-    st_stream_v4(dst + 8 * c, olo);
-    st_stream_v4(dst + D / 2 + 8 * c, ohi);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h = h0 + u * HS;
+      if (h >= H3) break;
+      const uint4 lo = lo4[u], hi = hi4[u];
+      __nv_bfloat16* dst;
+      uint4 olo = lo, ohi = hi;
+      if (h < Hq + Hkv) {
+        const uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
+        const uint32_t bb[4] = {hi.x, hi.y, hi.z, hi.w};
+        uint32_t ol[4], oh[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = bf_lo(a[e]), x1 = bf_hi(a[e]);      // elements i, i+1
+          const float y0 = bf_lo(bb[e]), y1 = bf_hi(bb[e]);    // elements i+D/2, i+1+D/2
+          const float c0 = cs[2 * e], s0 = sn[2 * e], c1 = cs[2 * e + 1], s1 = sn[2 * e + 1];
+          ol[e] = pack_bf2(fmaf(x0, c0, -y0 * s0), fmaf(x1, c1, -y1 * s1));
+          oh[e] = pack_bf2(fmaf(x0, s0, y0 * c0), fmaf(x1, s1, y1 * c1));
+        }
+        olo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        ohi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+        dst = h < Hq ? q + ((static_cast<long long>(b) * Hq + h) * T + t) * D
+                     : k + ((static_cast<long long>(b) * Hkv + (h - Hq)) * T + t) * D;
+      } else {
+        dst = v + ((static_cast<long long>(b) * Hkv + (h - Hq - Hkv)) * T + t) * D;
+      }
+      st_stream_v4(dst + 8 * c, olo);
+      st_stream_v4(dst + D / 2 + 8 * c, ohi);
+    }
   }
 }
 
