@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import itertools
 import json
 import math
 import os
@@ -356,6 +357,58 @@ def prologue_line(w, res, peaks, peak_src):
     return line
 
 
+def time_varlen(wv, steps, warmup, flush, stream, tess, torch, dev):
+    """The packed variable-length forward over ``wv``'s mixed lengths, drawn
+    on the device (CUDA generator seeded with the workload's seed), one
+    launch per step, L2 flushed before each."""
+    lens = wv.lens()
+    total = sum(lens)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wv.seed)
+    q = torch.randn((total, wv.Hq, wv.d), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((total, wv.Hkv, wv.d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((total, wv.Hkv, wv.d), generator=g, device=dev).to(torch.bfloat16)
+    cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wv.Hq, total), dtype=torch.float32, device=dev)
+
+    def call():
+        tess.attn_fwd_varlen(q, k, v, cu, max(lens), causal=True, scale=wv.scale, out=o,
+                             lse=lse, stream=stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        call()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call()
+        launches += tess.tessera_attn_last_launch_count()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    del q, k, v, o, lse
+    return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches
+
+
+def varlen_line(wv, times, launches, peaks, peak_src):
+    ms = statistics.median(times)
+    tf = wv.flops / (ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"metric": "packed variable-length causal GQA attn fwd TFLOP/s (bf16)",
+            "value": round(tf, 2), "unit": UNIT, "ms": round(ms, 5), "steps": len(times),
+            "flops_per_step": wv.flops,
+            "flop_count": "sum over sequences of the metric's 2*Hq*T_b^2*d",
+            "config": wv.describe(), "gpu_launches": launches,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak,
+                         "unit": UNIT, "frac": round(tf / peak, 4),
+                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+            "l2": "flushed before every timed step"}
+
+
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
     tessera_attn_fwd_host (copies pipelined with the kernels over key/value-head
@@ -487,6 +540,10 @@ def main():
     if err != 0:
         raise SystemExit(f"device-side error in the decode step (code {err})")
 
+    # the packed variable-length forward on its mixed-length batch
+    vl_times, vl_launches = time_varlen(inputs.VARLEN, max(5, min(args.steps, 50)), 3, flush,
+                                        stream, tess, torch, dev)
+
     # the prologue kernels at the workload's sizes
     pro = time_prologue(w, max(5, min(args.steps, 100)), 3, flush, stream, tess, torch, dev)
 
@@ -570,6 +627,7 @@ def main():
                      "l2": "flushed before every timed step"},
         "decode": decode_line(wd, dec_times, dec_max_ms, dec_steps, dec_launches, dec_ws, world,
                               peaks, peak_src),
+        "varlen": varlen_line(inputs.VARLEN, vl_times, vl_launches, peaks, peak_src),
         "prologue": prologue_line(w, pro, peaks, peak_src),
         "clocks": clk,
         "sweep": sweep or None,

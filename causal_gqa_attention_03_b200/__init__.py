@@ -11,7 +11,7 @@ Raw C-ABI names (integer pointers, sizes, stream handle):
     tessera_attn_selftest_timeout, tessera_attn_bwd, tessera_attn_bwd_workspace_bytes,
     tessera_attn_bwd_noalloc, tessera_attn_bwd_noalloc_max_workspace_bytes,
     tessera_attn_decode, tessera_attn_decode_workspace_bytes, tessera_rmsnorm,
-    tessera_rope_qkv
+    tessera_rope_qkv, tessera_attn_fwd_varlen
 Tensor convenience wrappers (PyTorch used only for memory and streams):
     attn_fwd(q, k, v, causal=True, scale=None, out=None, lse=None, stream=None)
     attn_fwd_host(q, k, v, causal=True, scale=None, out=None, lse=None,
@@ -22,6 +22,7 @@ Tensor convenience wrappers (PyTorch used only for memory and streams):
                 scale=None, stream=None)
     rmsnorm(x, w, eps=1e-6, out=None, stream=None)
     rope_qkv(qkv, Hq, Hkv, positions=None, base=10000.0, stream=None)
+    attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=True, scale=None, stream=None)
 """
 from __future__ import annotations
 
@@ -38,12 +39,15 @@ EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
             "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
             "tessera_attn_selftest_timeout", "tessera_attn_decode",
-            "tessera_attn_decode_workspace_bytes", "tessera_rmsnorm", "tessera_rope_qkv")
+            "tessera_attn_decode_workspace_bytes", "tessera_rmsnorm", "tessera_rope_qkv",
+            "tessera_attn_fwd_varlen")
 
 # Device error code recorded by tessera_attn_selftest_timeout.
 DEVICE_ERR_SELFTEST = 9
 # Device error code of a decode step given a sequence length or block id out of range.
 DEVICE_ERR_DECODE_INPUT = 20
+# Device error code of a packed forward given sequence offsets out of range.
+DEVICE_ERR_VARLEN_INPUT = 10
 
 STATUS = {0: "TESSERA_OK", 1: "TESSERA_ERR_INVALID_ARG", 2: "TESSERA_ERR_UNSUPPORTED",
           3: "TESSERA_ERR_MISALIGNED", 4: "TESSERA_ERR_CUDA", 5: "TESSERA_ERR_TIMEOUT",
@@ -101,6 +105,9 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_decode.restype = ci
             lib.tessera_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci]
             lib.tessera_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+            lib.tessera_attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                                    ci, ci, ctypes.c_float, vp]
+            lib.tessera_attn_fwd_varlen.restype = ci
             lib.tessera_rmsnorm.argtypes = [vp, vp, vp, ci, ci, ctypes.c_float, vp]
             lib.tessera_rmsnorm.restype = ci
             lib.tessera_rope_qkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
@@ -170,6 +177,16 @@ def tessera_attn_decode(q: int, k_cache: int, v_cache: int, block_table: int, se
 
 def tessera_attn_decode_workspace_bytes(B: int, Hq: int, max_seq_len: int, d: int) -> int:
     return load_library().tessera_attn_decode_workspace_bytes(B, Hq, max_seq_len, d)
+
+
+def tessera_attn_fwd_varlen(q: int, k: int, v: int, o: int, lse: int | None, cu_seqlens: int,
+                            B: int, total: int, max_seqlen: int, Hq: int, Hkv: int, d: int,
+                            causal: int, scale: float, stream: int | None) -> int:
+    """The packed variable-length forward with integer device pointers; returns the status."""
+    return load_library().tessera_attn_fwd_varlen(q or None, k or None, v or None, o or None,
+                                                  lse or None, cu_seqlens or None, B, total,
+                                                  max_seqlen, Hq, Hkv, d, int(causal),
+                                                  float(scale), stream or None)
 
 
 def tessera_rmsnorm(x: int, w: int, y: int, rows: int, dim: int, eps: float,
@@ -473,3 +490,41 @@ def rope_qkv(qkv, Hq: int, Hkv: int, positions=None, base: float = 10000.0, q=No
     if st != 0:
         raise TesseraError(st, "tessera_rope_qkv")
     return q, k, v
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = True,
+                    scale: float | None = None, out=None, lse=None, stream=None,
+                    want_lse: bool = True):
+    """Forward over packed sequences: q [total, Hq, d], k/v [total, Hkv, d]
+    (CUDA bf16), cu_seqlens CUDA int32 [B+1], max_seqlen a host bound on the
+    lengths.  Returns (o [total, Hq, d], lse [Hq, total] fp32 or None)."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [total, H, d] tensor")
+    if (not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dtype != torch.int32
+            or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous()):
+        raise TypeError("cu_seqlens must be a contiguous CUDA int32 [B+1] tensor")
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (total, Hkv, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [total, Hkv, d] matching q")
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = tessera_attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None,
+                                 cu_seqlens.data_ptr(), B, total, int(max_seqlen), Hq, Hkv, d,
+                                 int(bool(causal)), float(scale), stream.cuda_stream)
+    if st != 0:
+        raise TesseraError(st, "tessera_attn_fwd_varlen")
+    return out, lse

@@ -62,6 +62,25 @@ bool make_map(CUtensorMap* map, const void* base, int planes, int T, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// Packed rows [total, H, d] bf16 viewed as a 3-D tensor (d innermost, then
+// head, then row); boxes of 64 columns x 1 head x 128 rows with the 128-byte
+// swizzle, which land in shared memory as the same [128 rows][64] sub-tile.
+// Rows at or past `total` read as zero.
+bool make_map_packed(CUtensorMap* map, const void* base, int total, int H, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(total)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   if (!a || !b || na == 0 || nb == 0) return false;
   const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
@@ -70,9 +89,12 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// One launch of the forward.  With cu_seqlens (device, [B+1]) the B
+// sequences are packed ([total, H, d]) and T is the longest length.
 template <int D>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-           int Hkv, int T, int causal, float scale, cudaStream_t stream) {
+           int Hkv, int T, int causal, float scale, cudaStream_t stream,
+           const int* cu_seqlens = nullptr, int total = 0) {
   using C = FwdCfg<D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TESSERA_ERR_CUDA;
@@ -90,9 +112,14 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
 
   CUtensorMap tm_q, tm_k, tm_v;
-  if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
-      !make_map(&tm_v, v, B * Hkv, T, D))
+  if (cu_seqlens != nullptr) {
+    if (!make_map_packed(&tm_q, q, total, Hq, D) || !make_map_packed(&tm_k, k, total, Hkv, D) ||
+        !make_map_packed(&tm_v, v, total, Hkv, D))
+      return TESSERA_ERR_CUDA;
+  } else if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
+             !make_map(&tm_v, v, B * Hkv, T, D)) {
     return TESSERA_ERR_CUDA;
+  }
 
   FwdParams p;
   p.B = B;
@@ -117,6 +144,8 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
 
   // persistent: one CTA per SM, each walking its share of the units
   const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
@@ -475,6 +504,39 @@ extern "C" int tessera_attn_fwd(const void* q, const void* k, const void* v, voi
   if (st != TESSERA_OK || empty) return st;
   return launch_d(d, q, k, v, o, lse, B, Hq, Hkv, T, causal, scale,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int tessera_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                       float* lse, const int32_t* cu_seqlens, int B, int total,
+                                       int max_seqlen, int Hq, int Hkv, int d, int causal,
+                                       float scale, tessera_stream_t stream) {
+  g_last_launches = 0;
+  if (B < 0 || total < 0 || max_seqlen < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return TESSERA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return TESSERA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TESSERA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TESSERA_ERR_UNSUPPORTED;
+  if (max_seqlen > total) return TESSERA_ERR_INVALID_ARG;
+  if (B == 0 || total == 0 || max_seqlen == 0) return TESSERA_OK;
+  if (!q || !k || !v || !o || !cu_seqlens) return TESSERA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return TESSERA_ERR_MISALIGNED;
+  const size_t q_bytes = static_cast<size_t>(total) * Hq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(total) * Hkv * d * 2;
+  const size_t lse_bytes = static_cast<size_t>(total) * Hq * 4;
+  const size_t cu_bytes = (static_cast<size_t>(B) + 1) * 4;
+  const void* ins[4] = {q, k, v, cu_seqlens};
+  const size_t in_bytes[4] = {q_bytes, kv_bytes, kv_bytes, cu_bytes};
+  for (int i = 0; i < 4; ++i)
+    if (overlaps(o, q_bytes, ins[i], in_bytes[i]) || overlaps(lse, lse_bytes, ins[i], in_bytes[i]))
+      return TESSERA_ERR_INVALID_ARG;
+  if (overlaps(o, q_bytes, lse, lse_bytes)) return TESSERA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int* cu = reinterpret_cast<const int*>(cu_seqlens);
+  if (d == 64)
+    return launch<64>(q, k, v, o, lse, B, Hq, Hkv, max_seqlen, causal, scale, s, cu, total);
+  return launch<128>(q, k, v, o, lse, B, Hq, Hkv, max_seqlen, causal, scale, s, cu, total);
 }
 
 extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,

@@ -59,6 +59,7 @@ enum WaitCode : uint32_t {
   kErrWaitDrain = 7,
   kErrWaitQEmpty = 8,
   kErrSelfTest = 9,  // the deliberate timeout of attn_selftest_timeout_kernel
+  kErrVarlenInput = 10,  // a packed sequence's bounds out of range (that sequence is skipped)
 };
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
@@ -116,14 +117,22 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   unsigned long long launch_id;
+  // Packed sequences: cu_seqlens[b] .. cu_seqlens[b+1] are sequence b's rows
+  // of q [total, Hq, d], k/v [total, Hkv, d], o [total, Hq, d], lse [Hq, total];
+  // T is then the longest length.  Null: fixed length T, layouts [B, H, T, d].
+  const int* cu_seqlens;
+  int total;
 };
 
 // A work unit: batch b, key/value head g, the two tiles' query heads and
-// 128-row blocks, and how many key tiles each visits (0: tile absent).
+// 128-row blocks, and how many key tiles each visits (0: tile absent).  T is
+// the sequence's length and row0 its first row in the packed layout (0 for
+// fixed-length batches).
 struct Unit {
   int b, g;
   int head[2], qblk[2], ntile[2];
   int nmax;
+  int T, row0;
 };
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
@@ -148,9 +157,25 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     w.qblk[0] = 2 * pr;
     w.qblk[1] = 2 * pr + 1;
   }
+  w.T = p.T;
+  w.row0 = 0;
+  if (p.cu_seqlens != nullptr) {
+    const int start = p.cu_seqlens[w.b], end = p.cu_seqlens[w.b + 1];
+    if (start < 0 || end < start || end - start > p.T || end > p.total) {
+      // skip the sequence; recorded under another launch id, so that the
+      // other units' bounded waits carry on
+      atomicCAS(&g_tessera_err, 0ull,
+                (((p.launch_id ^ 0x80000000ull) & 0xffffffffull) << 32) | kErrVarlenInput);
+      w.T = 0;
+    } else {
+      w.T = end - start;
+      w.row0 = start;
+    }
+  }
+  const int nqb = (w.T + 127) / 128;
 #pragma unroll
   for (int t = 0; t < 2; ++t)
-    w.ntile[t] = (w.qblk[t] >= p.nqb) ? 0 : (p.causal ? min(w.qblk[t] + 1, p.nqb) : p.nqb);
+    w.ntile[t] = (w.qblk[t] >= nqb) ? 0 : (p.causal ? min(w.qblk[t] + 1, nqb) : nqb);
   w.nmax = max(w.ntile[0], w.ntile[1]);
   return w;
 }
@@ -334,30 +359,36 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const uint64_t keep = ptx::policy_evict_last();
       const uint64_t once = ptx::policy_evict_first();
       int idx = 0;  // K/V tiles loaded so far (ring position)
-      int k = 0;
+      int kq = 0;   // units with work so far (Q buffer phases)
+      const bool packed = p.cu_seqlens != nullptr;
       bool ok = true;
-      for (; ok; ++k) {
+      for (int k = 0; ok; ++k) {
         const int u = unit_of(p, k);
         if (u < 0) break;
         const Unit w = decode_unit(p, u);
+        if (w.nmax == 0) continue;  // past the end of a short packed sequence
         // Q of this unit, once the previous unit's S products no longer read
-        // the Q buffer.
+        // the Q buffer.  Fixed length: (row, plane b*H + h); packed: the map
+        // is [total][H][d], coordinates (head, row).
         auto load_q = [&]() -> bool {
-          if (!warp_wait(q_empty, (k & 1) ^ 1u, kErrWaitQEmpty, p.launch_id)) return false;
+          if (!warp_wait(q_empty, (kq & 1) ^ 1u, kErrWaitQEmpty, p.launch_id)) return false;
           if (leader) {
             ptx::mbar_arrive_expect_tx(q_full,
                                        ((w.ntile[0] > 0) + (w.ntile[1] > 0)) * C::TILE_BYTES);
             for (int t = 0; t < C::NQ; ++t) {
               if (w.ntile[t] == 0) continue;
+              const int row = w.row0 + w.qblk[t] * C::BM;
+              const int y = packed ? w.head[t] : row;
+              const int z = packed ? row : w.b * p.Hq + w.head[t];
               for (int c = 0; c < C::SUB; ++c)
                 ptx::tma_load_3d_hint(sQ + t * C::TILE_BYTES + c * C::SUB_BYTES, &tm_q, q_full,
-                                      c * 64, w.qblk[t] * C::BM, w.b * p.Hq + w.head[t], once);
+                                      c * 64, y, z, once);
             }
           }
           __syncwarp();
           return true;
         };
-        const int kv_plane = w.b * p.Hkv + w.g;
+        const int kv_plane = packed ? w.g : w.b * p.Hkv + w.g;
         // K_0 and V_0 go first: they do not depend on the Q buffer
         const int q_at = min(2, 2 * w.nmax);
         for (int i = 0; i < 2 * w.nmax; ++i, ++idx) {  // K_0, V_0, K_1, V_1, ...
@@ -374,17 +405,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           if (leader) {
             ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
             const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+            const int row = w.row0 + (i >> 1) * C::BN;
             for (int c = 0; c < C::SUB; ++c)
               ptx::tma_load_3d_hint(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s],
-                                    c * 64, (i >> 1) * C::BN, kv_plane, keep);
+                                    c * 64, packed ? kv_plane : row, packed ? row : kv_plane,
+                                    keep);
           }
           __syncwarp();
         }
         if (ok && q_at == 2 * w.nmax && !load_q()) ok = false;
+        if (ok) ++kq;
       }
       if (!ok) {
         // Gave up: let the copies already in flight land before the CTA exits.
-        if (k > 0) warp_wait(q_full, (k - 1) & 1, kErrWaitQ, p.launch_id);
+        if (kq > 0) warp_wait(q_full, (kq - 1) & 1, kErrWaitQ, p.launch_id);
         for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
           warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrWaitKvFull, p.launch_id);
       }
@@ -401,11 +435,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       int base = 0;           // ring position of the unit's K_0
       int pcnt[2] = {0, 0};   // P tiles consumed per query tile (p_full phases)
       bool ok = true;
+      int kq = 0;  // units with work so far (Q buffer phases)
       for (int k = 0; ok; ++k) {
         const int u = unit_of(p, k);
         if (u < 0) break;
         const Unit w = decode_unit(p, u);
-        if (!warp_wait(q_full, k & 1, kErrWaitQ, p.launch_id)) break;
+        if (w.nmax == 0) continue;  // past the end of a short packed sequence
+        if (!warp_wait(q_full, kq & 1, kErrWaitQ, p.launch_id)) break;
+        ++kq;
         for (int j = 0; ok && j <= w.nmax; ++j) {
           const int kidx = base + 2 * j, vidx = base + 2 * j - 1;
           if (j < w.nmax)
@@ -512,8 +549,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
         const int kv0 = j * C::BN;
-        const bool edge = p.causal ? (kv0 + C::BN - 1 > q_row - row) : (kv0 + C::BN > p.T);
-        const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
+        const bool edge = p.causal ? (kv0 + C::BN - 1 > q_row - row) : (kv0 + C::BN > w.T);
+        const int lim = p.causal ? min(q_row, w.T - 1) : w.T - 1;  // last visible key
         float alpha;
         bool rescale;
         uint32_t pk[2][32];
@@ -548,8 +585,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       ++ocnt;
       ptx::tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool store = q_row < p.T;
-      const int64_t orow = (static_cast<int64_t>(w.b) * p.Hq + w.head[t]) * p.T + q_row;
+      const bool store = q_row < w.T;
+      // O and LSE element offsets of this row: [B,Hq,T,d] / [B,Hq,T], or packed
+      // [total,Hq,d] / [Hq,total]
+      int64_t orow, lrow;
+      if (p.cu_seqlens != nullptr) {
+        const int64_t tok = static_cast<int64_t>(w.row0) + q_row;
+        orow = tok * p.Hq + w.head[t];
+        lrow = static_cast<int64_t>(w.head[t]) * p.total + tok;
+      } else {
+        orow = (static_cast<int64_t>(w.b) * p.Hq + w.head[t]) * p.T + q_row;
+        lrow = orow;
+      }
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -571,7 +618,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
       }
       if (store && p.lse != nullptr)
-        p.lse[orow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[lrow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
       // O_t has been read; the next unit's first P_t arrival (after this
       // fence) is what lets the MMA warp overwrite it.
       ptx::tc_fence_before();

@@ -275,3 +275,58 @@ def gather_sequences(table: np.ndarray, seq_lens: np.ndarray, rows, bs: int,
     idx = torch.tensor(ids if ids else [0], dtype=torch.long, device=k_cache.device)
     return (k_cache.index_select(0, idx).cpu(), v_cache.index_select(0, idx).cpu(), sub_table,
             sub_lens)
+
+
+def make_packed(lens, Hq: int, Hkv: int, d: int, seed: int, sigma_qk: float = 1.0):
+    """Packed sequences for the variable-length forward: (q [total, Hq, d],
+    k, v [total, Hkv, d]) bf16 CPU tensors and cu_seqlens int32 [B+1] (numpy).
+    A torch CPU generator seeded with ``seed`` draws q, then k, then v
+    standard normal in row-major order; q and k are multiplied by sigma_qk."""
+    lens = [int(n) for n in lens]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((total, Hq, d), generator=g) * sigma_qk
+    k = torch.randn((total, Hkv, d), generator=g) * sigma_qk
+    v = torch.randn((total, Hkv, d), generator=g)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), cu
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of mixed-length sequences (lengths uniform in
+    [min_len, max_len] from numpy default_rng(seed)), drawn as make_packed."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    min_len: int
+    max_len: int
+    seed: int
+
+    def lens(self) -> list:
+        rng = np.random.default_rng(self.seed)
+        return [int(x) for x in rng.integers(self.min_len, self.max_len + 1, size=self.B)]
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+    @property
+    def flops(self) -> float:
+        """The metric's causal count per sequence, summed: 2*Hq*T_b^2*d."""
+        return float(sum(2.0 * self.Hq * n * n * self.d for n in self.lens()))
+
+    def describe(self) -> dict:
+        out = asdict(self)
+        lens = self.lens()
+        out["total"] = int(sum(lens))
+        out["longest"] = int(max(lens))
+        return out
+
+
+# Packed mixed lengths with the headline head configuration.
+VARLEN = VarlenWorkload("varlen_b32_hq32_hkv8_d128_len128to8192", B=32, Hq=32, Hkv=8, d=128,
+                        min_len=128, max_len=8192, seed=13)

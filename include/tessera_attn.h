@@ -73,6 +73,40 @@ int tessera_attn_fwd(const void *q, const void *k, const void *v, void *o,
                      int causal, float scale, tessera_stream_t stream);
 
 /*
+ * Variable-length forward: B sequences of different lengths packed into one
+ * batch, each attending only to itself.  The pages' forward has a causal flag
+ * (hysenlabs.com review, "The kernel set and its torch fallback"); running it
+ * over a batch of mixed lengths without padding is the variant adopted here,
+ * with the same per-sequence definition as tessera_attn_fwd:
+ *
+ *   sequence b holds rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of every tensor;
+ *   with T_b its length and i, j rows of sequence b, O and LSE of row i are
+ *   tessera_attn_fwd's over keys j <= i (causal) or all j < T_b.
+ *
+ * q           bf16 [total, Hq, d]  device, read only (token-major, packed)
+ * k, v        bf16 [total, Hkv, d] device, read only
+ * o           bf16 [total, Hq, d]  device, written
+ * lse         fp32 [Hq, total]     device, written; may be NULL
+ * cu_seqlens  int32 [B + 1] device: 0 = cu[0] <= cu[1] <= ... <= cu[B] = total
+ * B >= 0, total >= 0, max_seqlen: a bound on every length, 0 .. total (it
+ *             sizes the launch); B, total or max_seqlen 0 launches nothing
+ * Hq, Hkv, d, causal, scale, stream  as in tessera_attn_fwd
+ *
+ * Checks as in tessera_attn_fwd before any CUDA call, plus cu_seqlens
+ * non-NULL and 4-byte aligned and o/lse clear of every input.  The offsets
+ * live on the device and are checked by the kernel: a sequence whose bounds
+ * are out of order, past `total` or longer than max_seqlen is skipped (its
+ * rows of o and lse are left as they were) and TESSERA_DEVICE_ERR_VARLEN_INPUT
+ * is recorded for tessera_attn_device_error(); the other sequences are
+ * computed as usual and nothing outside the buffers is read.  One launch.
+ */
+#define TESSERA_DEVICE_ERR_VARLEN_INPUT 10
+int tessera_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                            const int32_t *cu_seqlens, int B, int total, int max_seqlen,
+                            int Hq, int Hkv, int d, int causal, float scale,
+                            tessera_stream_t stream);
+
+/*
  * Backward of tessera_attn_fwd: the gradients dQ, dK, dV of a loss given
  * dO = dLoss/dO, treating LSE as saved state.  The pages list the attention
  * backward as not yet built (it is the first extension after the forward);
@@ -290,7 +324,8 @@ int tessera_attn_selftest_timeout(unsigned int limit_us, tessera_stream_t stream
 const char *tessera_status_str(int status);
 
 /*
- * Kernel launches the last successful tessera_attn_fwd (0 or 1),
+ * Kernel launches the last successful tessera_attn_fwd or
+ * tessera_attn_fwd_varlen (0 or 1),
  * tessera_attn_fwd_host (one per chunk), tessera_attn_bwd (3),
  * tessera_attn_decode (1 or 2), tessera_rmsnorm or tessera_rope_qkv (1) call
  * on this thread queued.  Lets a caller

@@ -306,3 +306,32 @@ def rope_qkv_f64(qkv, Hq: int, Hkv: int, positions=None, base: float = 10000.0,
     if rc != 0:
         raise ValueError(f"oracle_rope_qkv_f64 failed with code {rc}")
     return q, k, v
+
+
+def attn_fwd_varlen_f64(q, k, v, cu_seqlens, causal: bool = True, scale: float | None = None,
+                        lib: ctypes.CDLL | None = None):
+    """Packed variable-length attention in fp64: each sequence attends to
+    itself only, with attn_fwd_f64's definition.
+
+    q: [total, Hq, d]; k, v: [total, Hkv, d]; cu_seqlens: [B+1] offsets.
+    Returns (O [total, Hq, d], LSE [Hq, total]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    total, Hq, d = q.shape
+    o = np.zeros((total, Hq, d))
+    lse = np.zeros((Hq, total))
+    for b in range(len(cu) - 1):
+        s, e = cu[b], cu[b + 1]
+        if e < s or s < 0 or e > total:
+            raise ValueError("cu_seqlens out of order or past total")
+        if e == s:
+            continue
+        ob, lb = attn_fwd_f64(q[s:e].transpose(1, 0, 2)[None], k[s:e].transpose(1, 0, 2)[None],
+                              v[s:e].transpose(1, 0, 2)[None], causal=causal, scale=scale,
+                              lib=lib)
+        o[s:e] = ob[0].transpose(1, 0, 2)
+        lse[:, s:e] = lb[0]
+    return o, lse

@@ -511,7 +511,52 @@ def pin_rope_invariants(lib):
     assert np.array_equal(v[0, 0, 0], [2.0, -0.75])
 
 
-ALL_PINS = [pin_rmsnorm_library, pin_rmsnorm_invariants, pin_rope_complex,
+# ---------------------------------------------------------------- varlen
+def pin_varlen_library(lib):
+    """Packed sequences against torch SDPA (float64) over the whole packed
+    batch with a block-diagonal (and causal) mask: no sequence sees another."""
+    for seed, (lens, Hq, Hkv, d, causal) in enumerate([([5, 1, 9, 0, 3], 4, 2, 8, True),
+                                                        ([7, 7, 2], 2, 2, 16, False),
+                                                        ([12, 4], 6, 2, 8, True)]):
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        total = int(cu[-1])
+        q = _rand((total, Hq, d), 1100 + seed)
+        k = _rand((total, Hkv, d), 1110 + seed)
+        v = _rand((total, Hkv, d), 1120 + seed)
+        scale = 0.37
+        o, lse = oracle.attn_fwd_varlen_f64(q, k, v, cu, causal=causal, scale=scale, lib=lib)
+        seq = np.repeat(np.arange(len(lens)), lens)
+        allowed = seq[:, None] == seq[None, :]
+        if causal:
+            allowed &= np.arange(total)[None, :] <= np.arange(total)[:, None]
+        G = Hq // Hkv
+        qt = torch.from_numpy(q).permute(1, 0, 2)
+        kt = torch.from_numpy(k).repeat_interleave(G, dim=1).permute(1, 0, 2)
+        vt = torch.from_numpy(v).repeat_interleave(G, dim=1).permute(1, 0, 2)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, attn_mask=torch.from_numpy(allowed), scale=scale).permute(1, 0, 2)
+        assert np.allclose(o, want.numpy(), rtol=0, atol=1e-12), seed
+        logits = scale * torch.einsum("htd,hsd->hts", qt, kt)
+        logits = logits.masked_fill(~torch.from_numpy(allowed), -math.inf)
+        assert np.allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_varlen_equal_lengths(lib):
+    """Equal lengths: the packed result is the fixed-length batch's, exactly."""
+    B, T, Hq, Hkv, d = 3, 6, 4, 2, 8
+    q = _rand((B, Hq, T, d), 1130)
+    k = _rand((B, Hkv, T, d), 1131)
+    v = _rand((B, Hkv, T, d), 1132)
+    o, lse = oracle.attn_fwd_f64(q, k, v, causal=True, scale=0.5, lib=lib)
+    pack = lambda x: x.transpose(0, 2, 1, 3).reshape(B * T, x.shape[1], d)
+    cu = np.arange(B + 1, dtype=np.int32) * T
+    ov, lv = oracle.attn_fwd_varlen_f64(pack(q), pack(k), pack(v), cu, causal=True, scale=0.5,
+                                        lib=lib)
+    assert np.array_equal(ov, pack(o))
+    assert np.array_equal(lv, lse.transpose(1, 0, 2).reshape(Hq, B * T))
+
+
+ALL_PINS = [pin_varlen_library, pin_varlen_equal_lengths, pin_rmsnorm_library, pin_rmsnorm_invariants, pin_rope_complex,
             pin_rope_invariants, pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
             pin_rows_entry, pin_bwd_library_autograd, pin_bwd_finite_differences,
             pin_bwd_invariants, pin_bwd_dq_rows_entry, pin_decode_library,

@@ -223,6 +223,28 @@ def test_rope_argument_checks_before_any_cuda_call(lib, kw, status):
     assert tess.tessera_attn_last_launch_count() == 0
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(total=-1), 1), (dict(max_seqlen=-1), 1), (dict(Hq=6, Hkv=4), 1),
+    (dict(d=96), 2), (dict(scale=0.0), 1), (dict(causal=2), 1),
+    (dict(max_seqlen=5000), 1),                      # longer than total
+    (dict(q=0), 1), (dict(o=0), 1), (dict(cu=0), 1),
+    (dict(q=ALIGNED + 8), 3), (dict(lse=ALIGNED + 0x4000004), 3), (dict(cu=ALIGNED + 0x5000002), 3),
+    (dict(o=ALIGNED + 0x100), 1),                    # o overlaps q
+    (dict(lse=ALIGNED + 0x5000000), 1),              # lse overlaps cu_seqlens
+    (dict(o=ALIGNED + 0x4000000), 1),                # o overlaps lse
+    (dict(B=0), 0), (dict(total=0, max_seqlen=0), 0), (dict(max_seqlen=0), 0),
+])
+def test_varlen_argument_checks_before_any_cuda_call(lib, kw, status):
+    a = dict(q=ALIGNED, k=ALIGNED + 0x1000000, v=ALIGNED + 0x2000000, o=ALIGNED + 0x3000000,
+             lse=ALIGNED + 0x4000000, cu=ALIGNED + 0x5000000, B=3, total=4000, max_seqlen=2000,
+             Hq=8, Hkv=2, d=128, causal=1, scale=0.1)
+    a.update(kw)
+    assert tess.tessera_attn_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"],
+                                        a["B"], a["total"], a["max_seqlen"], a["Hq"], a["Hkv"],
+                                        a["d"], a["causal"], a["scale"], None) == status
+    assert tess.tessera_attn_last_launch_count() == 0
+
+
 @pytest.mark.parametrize("limit_us", [0, 10_000_001, 2**32 - 1])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(lib, limit_us):
     assert tess.tessera_attn_selftest_timeout(limit_us, None) == 1
