@@ -1,0 +1,608 @@
+// The paged-KV decode step at head dimension 128 on the tensor cores.
+//
+// Same operation, items, chunk stream, partial slots and merge as
+// paged_decode.cuh; here the two contractions of a 128-token chunk run as
+// tcgen05 MMAs with the item's query heads as a narrow N = 16:
+//   S^T[t, h] = K[t, :] . q[h, :]       A = K chunk (M = 128 tokens, K-major),
+//                                        B = q rows (N = 16, K-major, rows >= GT zero)
+//   O^T[c, h] += sum_t V[t, c] P^T[h, t] A = V chunk (M = 128 columns, MN-major),
+//                                        B = P^T (N = 16, K = 128 tokens, K-major)
+// both accumulating in tensor memory.  The FP32 pipes keep only the softmax
+// (a thread per token), so the step stays bound by HBM.
+//
+// Roles (192 threads): warps 0-3 softmax (thread = token for S^T and column
+// for O^T, lanes 32w.. of tensor memory), warp 4 issues the MMAs, warp 5 is
+// the producer.  Rings: K (+ the q rows) in NK stages, released when S^T is
+// done; V in NV stages, released when the chunk's P.V is done.  S^T is double
+// buffered in tensor memory; P^T is one shared-memory tile, rewritten once the
+// previous P.V has finished.  Online softmax across a segment's chunks with a
+// lazy maximum: the running max moves only when a chunk's max exceeds it by
+// more than 2^8, and O^T is rescaled only then.
+#pragma once
+
+#include "paged_decode.cuh"
+
+namespace tessera {
+
+constexpr int kDecTcThreads = 192;
+constexpr int kDecTcMmaWarp = 4;
+constexpr int kDecTcTmaWarp = 5;
+constexpr int kDecTcN = 16;              // N of both products: query heads per item, padded
+constexpr float kDecTcRescale = 8.0f;    // log2 units
+
+struct DecTcCfg {
+  static constexpr int D = 128;
+  static constexpr int CH = kDecodeChunk;       // 128 tokens
+  static constexpr int HALF = CH * 128;         // one [128 rows][64 cols] bf16 sub-tile
+  static constexpr int QHALF = kDecTcN * 128;   // one [16 rows][64 cols] bf16 sub-tile
+  static constexpr int K_BYTES = 2 * HALF;
+  static constexpr int KSTAGE = K_BYTES + 2 * QHALF;  // K, then the q rows
+  static constexpr int VSTAGE = 2 * HALF;
+  static constexpr int NK = 3, NV = 3;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = NK * KSTAGE;
+  static constexpr int P_OFF = V_OFF + NV * VSTAGE;    // P^T: two [16][64] sub-tiles
+  static constexpr int RED_OFF = P_OFF + 2 * QHALF;    // float [2][4][16] chunk maxima
+  static constexpr int LRED_OFF = RED_OFF + 512;       // float [4][16] row-sum partials
+  static constexpr int SMETA_OFF = LRED_OFF + 256;     // int [2][8] (per S^T buffer)
+  static constexpr int KMETA_OFF = SMETA_OFF + 64;     // int [NK][8] (per K stage)
+  static constexpr int BAR_OFF = KMETA_OFF + 32 * NK;
+  // full_k[NK], empty_k[NK], full_v[NV], empty_v[NV], s_full[2], s_free[2],
+  // p_full, pv_done, drain
+  static constexpr int NBAR = 2 * NK + 2 * NV + 7;
+  static constexpr int SLOT_OFF = BAR_OFF + 8 * NBAR;
+  static constexpr int BYTES = SLOT_OFF + 16;
+  static constexpr int SMEM = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 64;
+  static constexpr int S_COL = 0;   // two buffers of 16 columns
+  static constexpr int O_COL = 32;  // 16 columns
+  static_assert(KSTAGE % 1024 == 0 && VSTAGE % 1024 == 0 && P_OFF % 1024 == 0, "alignment");
+  static_assert(SMEM <= 232448, "fits the 227 KB a CTA may use");
+};
+
+// 16-byte units to add to a K-major 128-byte-swizzled descriptor for K step
+// kk (16 elements) when the operand's two 64-column sub-tiles are `sub` bytes
+// apart.
+__device__ __forceinline__ uint32_t kmajor_step(int kk, int sub) {
+  return static_cast<uint32_t>((kk >> 2) * (sub >> 4) + (kk & 3) * 2);
+}
+
+// Producer warp: as decode_produce, with separate K and V rings and the q
+// rows fetched by TMA with every K chunk.
+template <int GT>
+__device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                              const CUtensorMap* tm_q, const DecodeParams& p,
+                                              uint8_t* sm, int* kmeta, uint64_t* full_k,
+                                              uint64_t* empty_k, uint64_t* full_v,
+                                              uint64_t* empty_v, int lane) {
+  using C = DecTcCfg;
+  const int R = p.rows_per_box;
+  const long long HZ = static_cast<long long>(p.Hkv) * p.zgroups;
+  long long tot = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    long long ch = b < p.B ? decode_chunks(decode_len(p, b)) : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ch += __shfl_xor_sync(0xffffffffu, ch, off);
+    tot += ch;
+  }
+  const long long total = tot * HZ;
+  const long long per = (total + gridDim.x - 1) / gridDim.x;
+  const long long lo = static_cast<long long>(blockIdx.x) * per;
+  long long hi = min(lo + per, total);
+  uint32_t produced = 0;
+  bool alive = true;
+  if (lo < hi) {
+    DecodeCursor cur{};
+    long long pre = 0;
+    for (int b0 = 0;; b0 += 32) {
+      const int b = b0 + lane;
+      const int n = b < p.B ? decode_len(p, b) : 0;
+      const long long ch = static_cast<long long>(decode_chunks(n)) * HZ;
+      const long long incl = warp_incl_scan(ch, lane) + pre;
+      const unsigned hit = __ballot_sync(0xffffffffu, b < p.B && incl > lo);
+      if (hit) {
+        const int j = __ffs(hit) - 1;
+        cur.b = b0 + j;
+        cur.n = __shfl_sync(0xffffffffu, n, j);
+        const long long start_b = __shfl_sync(0xffffffffu, incl - ch, j);
+        cur.nchunks = decode_chunks(cur.n);
+        const long long r = lo - start_b;
+        cur.gz = static_cast<int>(r / cur.nchunks);
+        cur.c = static_cast<int>(r % cur.nchunks);
+        cur.item0 = start_b + static_cast<long long>(cur.gz) * cur.nchunks;
+        break;
+      }
+      pre = __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const uint64_t pol = ptx::policy_evict_first();
+    const uint64_t keep = ptx::policy_evict_last();
+    auto load_ids = [&](const DecodeCursor& cu, int& blk, int& npg) {
+      const int nt = min(C::CH, cu.n - cu.c * C::CH);
+      npg = (nt + R - 1) / R;
+      blk = 0;
+      if (lane < npg)
+        blk = p.block_table[static_cast<long long>(cu.b) * p.max_blocks +
+                            (cu.c * C::CH + lane * R) / p.bs];
+    };
+    int blk, npg;
+    load_ids(cur, blk, npg);
+    for (long long pos = lo; pos < hi; ++pos) {
+      DecodeCursor nxt = cur;
+      int nblk = 0, nnpg = 0;
+      if (pos + 1 < hi) {
+        if (++nxt.c == nxt.nchunks) {
+          nxt.c = 0;
+          nxt.item0 += nxt.nchunks;
+          if (++nxt.gz == HZ) {
+            nxt.gz = 0;
+            do {  // the stream has more chunks, so such a sequence exists before B
+              ++nxt.b;
+              nxt.n = nxt.b < p.B ? decode_len(p, nxt.b) : -1;
+            } while (nxt.n == 0);
+            if (nxt.n < 0) {  // lengths changed under the kernel: stop after this chunk
+              decode_error(p, kErrDecodeInput);
+              nxt.n = 0;
+            }
+            nxt.nchunks = decode_chunks(nxt.n);
+          }
+        }
+        if (nxt.n > 0)
+          load_ids(nxt, nblk, nnpg);
+        else
+          hi = pos + 1;
+      }
+      const bool bad = __any_sync(0xffffffffu, lane < npg && (blk < 0 || blk >= p.num_blocks));
+      const bool seg_first = pos == lo || cur.c == 0;
+      const bool item_last = cur.c == cur.nchunks - 1;
+      const bool seg_last = pos == hi - 1 || item_last;
+      const int flags = (bad ? kStageBad : 0) | (seg_first ? kStageSegFirst : 0) |
+                        (seg_last ? kStageSegLast : 0) | (item_last ? kStageItemLast : 0);
+      const int nt = min(C::CH, cur.n - cur.c * C::CH);
+      const int g = cur.gz / p.zgroups, z = cur.gz % p.zgroups;
+      const int tok0 = cur.c * C::CH;
+      // ---- K and the q rows
+      const uint32_t sk = produced % C::NK;
+      bool ok = true;
+      if (lane == 0) {
+        if (bad) decode_error(p, kErrDecodeInput);
+        ok = decode_wait(&empty_k[sk], ((produced / C::NK) & 1) ^ 1u);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) decode_error(p, kErrDecodeWait);
+        alive = false;
+        break;
+      }
+      uint8_t* kst = sm + C::K_OFF + sk * C::KSTAGE;
+      if (lane == 0) {
+        int* m = kmeta + 8 * sk;
+        m[0] = cur.b;
+        m[1] = cur.gz;
+        m[2] = cur.c;
+        m[3] = nt;
+        m[4] = flags;
+        m[5] = static_cast<int>(blockIdx.x - cur.item0 / per);
+        if (bad) {
+          ptx::mbar_arrive(&full_k[sk]);
+        } else {
+          ptx::mbar_arrive_expect_tx(&full_k[sk],
+                                     static_cast<uint32_t>(npg * R * 256 + GT * 256));
+          const int qrow = (cur.b * p.Hq + g * p.G + z * GT);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            ptx::tma_load_2d_hint(kst + C::K_BYTES + h * C::QHALF, tm_q, &full_k[sk], 64 * h,
+                                  qrow, keep);
+        }
+      }
+      __syncwarp();
+      if (!bad && lane < npg) {
+        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          ptx::tma_load_2d_hint(kst + h * C::HALF + lane * R * 128, tm_k, &full_k[sk], 64 * h,
+                                row, pol);
+      }
+      // ---- V
+      const uint32_t sv = produced % C::NV;
+      if (lane == 0) ok = decode_wait(&empty_v[sv], ((produced / C::NV) & 1) ^ 1u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) decode_error(p, kErrDecodeWait);
+        alive = false;
+        break;
+      }
+      uint8_t* vst = sm + C::V_OFF + sv * C::VSTAGE;
+      if (lane == 0) {
+        if (bad)
+          ptx::mbar_arrive(&full_v[sv]);
+        else
+          ptx::mbar_arrive_expect_tx(&full_v[sv], static_cast<uint32_t>(npg * R * 256));
+      }
+      __syncwarp();
+      if (!bad && lane < npg) {
+        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          ptx::tma_load_2d_hint(vst + h * C::HALF + lane * R * 128, tm_v, &full_v[sv], 64 * h,
+                                row, pol);
+      }
+      ++produced;
+      cur = nxt;
+      blk = nblk;
+      npg = nnpg;
+    }
+  }
+  if (alive && lane == 0) {
+    const uint32_t sk = produced % C::NK;
+    if (decode_wait(&empty_k[sk], ((produced / C::NK) & 1) ^ 1u)) {
+      kmeta[8 * sk] = -1;
+      ptx::mbar_arrive(&full_k[sk]);
+    } else {
+      decode_error(p, kErrDecodeWait);
+    }
+  }
+}
+
+template <int GT>
+__global__ void __launch_bounds__(kDecTcThreads, 1)
+    paged_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
+  static_assert(GT == 1 || GT == 2 || GT == 4 || GT == 8 || GT == 16, "heads per item");
+  using C = DecTcCfg;
+  extern __shared__ uint8_t dsmem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  float* red = reinterpret_cast<float*>(sm + C::RED_OFF);
+  float* lred = reinterpret_cast<float*>(sm + C::LRED_OFF);
+  int* smeta = reinterpret_cast<int*>(sm + C::SMETA_OFF);
+  int* kmeta = reinterpret_cast<int*>(sm + C::KMETA_OFF);
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
+  uint64_t* empty_k = full_k + C::NK;
+  uint64_t* full_v = empty_k + C::NK;
+  uint64_t* empty_v = full_v + C::NV;
+  uint64_t* s_full = empty_v + C::NV;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* drain = pv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::SLOT_OFF);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (warp < 4) {
+    // zero the q rows >= GT of every K stage and the P^T tile (never written
+    // again: TMA writes rows < GT, the softmax heads < GT)
+    for (int s = 0; s < C::NK; ++s)
+      for (int i = tid; i < 2 * C::QHALF / 16; i += 128)
+        reinterpret_cast<uint4*>(sm + C::K_OFF + s * C::KSTAGE + C::K_BYTES)[i] =
+            make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < 2 * C::QHALF / 16; i += 128)
+      reinterpret_cast<uint4*>(sm + C::P_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
+    ptx::fence_proxy_async_smem();
+  } else if (warp == kDecTcMmaWarp) {
+    if (lane == 0) {
+      for (int s = 0; s < C::NK; ++s) {
+        ptx::mbar_init(&full_k[s], 1);
+        ptx::mbar_init(&empty_k[s], 1);
+      }
+      for (int s = 0; s < C::NV; ++s) {
+        ptx::mbar_init(&full_v[s], 1);
+        ptx::mbar_init(&empty_v[s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(&s_full[b], 1);
+        ptx::mbar_init(&s_free[b], 128);
+      }
+      ptx::mbar_init(p_full, 128);
+      ptx::mbar_init(pv_done, 1);
+      ptx::mbar_init(drain, 1);
+      ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  } else if (lane == 0) {
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+    ptx::prefetch_tensormap(&tm_q);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kDecTcTmaWarp) {
+    dectc_produce<GT>(&tm_k, &tm_v, &tm_q, p, sm, kmeta, full_k, empty_k, full_v, empty_v,
+                      lane);
+  } else if (warp == kDecTcMmaWarp) {
+    // ======================= MMA issue (lane 0; the warp waits) ===========
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kDecTcN, false, false);
+    constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, kDecTcN, true, false);
+    constexpr uint32_t kHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-byte swizzle
+    const uint32_t k_base = ptx::smem_u32(sm + C::K_OFF);
+    const uint32_t v_base = ptx::smem_u32(sm + C::V_OFF);
+    const uint32_t p_lo = ptx::sdesc_sw128_lo(ptx::smem_u32(sm + C::P_OFF), 16);
+    bool pending = false;   // a good chunk whose P.V is still to issue
+    uint32_t pend_sv = 0, pend_kc = 0, pend_acc = 0;
+    uint32_t npv = 0;       // P.V products issued (p_full / pv_done phases)
+    bool seg_good = false;  // the current segment has had a good chunk
+    bool ok = true;
+    auto issue_pv = [&]() -> bool {
+      bool w_ok = __all_sync(0xffffffffu, decode_wait(p_full, npv & 1));
+      w_ok = w_ok && __all_sync(0xffffffffu,
+                                decode_wait(&full_v[pend_sv], (pend_kc / C::NV) & 1));
+      if (!w_ok) return false;
+      ptx::tc_fence_after();
+      if (leader) {
+        const uint32_t va = ptx::sdesc_sw128_lo(v_base + pend_sv * C::VSTAGE, C::HALF);
+        ptx::mma_ss_lohi_rt(tmem + C::O_COL, va, kHi, p_lo, kHi, kIdescO, pend_acc);
+#pragma unroll
+        for (int kk = 1; kk < C::CH / 16; ++kk)
+          ptx::mma_ss_lohi<1>(tmem + C::O_COL, va + kk * (2048 >> 4), kHi,
+                              p_lo + kmajor_step(kk, C::QHALF), kHi, kIdescO);
+        ptx::tc_commit(&empty_v[pend_sv]);
+        ptx::tc_commit(pv_done);
+      }
+      __syncwarp();
+      ++npv;
+      pending = false;
+      return true;
+    };
+    for (uint32_t kc = 0; ok; ++kc) {
+      const uint32_t sk = kc % C::NK, buf = kc & 1;
+      ok = __all_sync(0xffffffffu, decode_wait(&full_k[sk], (kc / C::NK) & 1));
+      ok = ok && __all_sync(0xffffffffu, decode_wait(&s_free[buf], ((kc >> 1) & 1) ^ 1u));
+      if (!ok) break;
+      int m[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = kmeta[8 * sk + i];
+      if (leader) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) smeta[8 * buf + i] = m[i];
+      }
+      __syncwarp();
+      if (m[0] < 0) {  // sentinel: finish the last P.V, then pass it on
+        if (pending) ok = issue_pv();
+        if (leader) ptx::mbar_arrive(&s_full[buf]);
+        __syncwarp();
+        break;
+      }
+      const bool bad = (m[4] & kStageBad) != 0;
+      if (bad) {
+        // nothing to multiply: hand the stages back in order
+        ok = __all_sync(0xffffffffu, decode_wait(&full_v[kc % C::NV], (kc / C::NV) & 1));
+        if (!ok) break;
+        if (leader) {
+          ptx::mbar_arrive(&empty_k[sk]);
+          ptx::mbar_arrive(&empty_v[kc % C::NV]);
+          ptx::mbar_arrive(&s_full[buf]);
+        }
+        __syncwarp();
+      } else {
+        ptx::tc_fence_after();
+        if (leader) {
+          // S^T = K q^T: A = K (K-major, sub-tiles 16 KB apart), B = q rows
+          // (K-major, sub-tiles 2 KB apart)
+          const uint32_t ka = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE, 16);
+          const uint32_t qb = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE + C::K_BYTES, 16);
+          const uint32_t sd = tmem + C::S_COL + kDecTcN * buf;
+          ptx::mma_ss_lohi<0>(sd, ka, kHi, qb, kHi, kIdescS);
+#pragma unroll
+          for (int kk = 1; kk < C::D / 16; ++kk)
+            ptx::mma_ss_lohi<1>(sd, ka + kmajor_step(kk, C::HALF), kHi,
+                                qb + kmajor_step(kk, C::QHALF), kHi, kIdescS);
+          ptx::tc_commit(&s_full[buf]);
+          ptx::tc_commit(&empty_k[sk]);
+        }
+        __syncwarp();
+      }
+      // the previous good chunk's P.V, now that this chunk's S^T is queued
+      if (pending && !issue_pv()) {
+        ok = false;
+        break;
+      }
+      if (!bad) {
+        pending = true;
+        pend_sv = kc % C::NV;
+        pend_kc = kc;
+        pend_acc = seg_good ? 1u : 0u;
+        seg_good = true;
+      }
+      if (m[4] & kStageSegLast) seg_good = false;
+    }
+    if (!ok) decode_error(p, kErrDecodeWait);
+    // every MMA issued must finish before tensor memory is released
+    if (leader) ptx::tc_commit(drain);
+    __syncwarp();
+    decode_wait(drain, 0);
+    // and the softmax warps are done with it
+    ptx::bar_sync_named(2, 160);
+    ptx::tc_fence_after();
+    __syncwarp();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  } else {
+    // ======================= softmax (warps 0-3, thread = token) ===========
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t o_addr = tmem + lane_base + C::O_COL;
+    const int t = tid;  // token of S^T, column of O^T
+    float m_run[GT], l_w[GT];
+#pragma unroll
+    for (int gh = 0; gh < GT; ++gh) {
+      m_run[gh] = -INFINITY;
+      l_w[gh] = 0.f;
+    }
+    bool seg_good = false;
+    uint32_t ngood = 0;  // good chunks seen (P.V products: pv_done phases)
+    const uint32_t p_base = ptx::smem_u32(sm + C::P_OFF);
+    for (uint32_t kc = 0;; ++kc) {
+      const uint32_t buf = kc & 1;
+      bool ok = decode_wait(&s_full[buf], (kc >> 1) & 1);
+      ok = ptx::bar_red_and(1, 128, ok);
+      if (!ok) {
+        if (tid == 0) decode_error(p, kErrDecodeWait);
+        break;
+      }
+      int m[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = smeta[8 * buf + i];
+      if (m[0] < 0) break;  // sentinel
+      const int flags = m[4], nt = m[3];
+      const bool bad = (flags & kStageBad) != 0;
+      uint32_t sr[16];
+      if (!bad) {
+        ptx::tc_fence_after();
+        ptx::tmem_ld16(tmem + lane_base + C::S_COL + kDecTcN * buf, sr);
+        ptx::tmem_ld_wait();
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&s_free[buf]);
+      const int g = m[1] / p.zgroups, z = m[1] % p.zgroups;
+      const long long head0 = static_cast<long long>(m[0]) * p.Hq + g * p.G + z * GT;
+      if (!bad) {
+        float x[GT];
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh)
+          x[gh] = t < nt ? __uint_as_float(sr[gh]) * p.scale_log2 : -INFINITY;
+        // chunk max per head: warp, then the four warps
+        float* rb = red + buf * 64;
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh) {
+          float mx = x[gh];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          if (lane == 0) rb[warp * 16 + gh] = mx;
+        }
+        ptx::bar_sync_named(1, 128);
+        float alpha[GT];
+        bool rescale = false;
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh) {
+          const float cm = fmaxf(fmaxf(rb[gh], rb[16 + gh]), fmaxf(rb[32 + gh], rb[48 + gh]));
+          float m_new = m_run[gh];
+          if (!seg_good || cm > m_run[gh] + kDecTcRescale) m_new = fmaxf(m_run[gh], cm);
+          alpha[gh] = ptx::ex2(m_run[gh] - m_new);  // 1 when unchanged, 0 at a segment start
+          rescale |= seg_good && m_new != m_run[gh];
+          m_run[gh] = m_new;
+        }
+        float pv[GT];
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh) {
+          pv[gh] = ptx::ex2(x[gh] - m_run[gh]);  // masked tokens: 0
+          float sum = pv[gh];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+          l_w[gh] = fmaf(l_w[gh], alpha[gh], sum);
+        }
+        // the previous P.V must be done: it reads the P^T tile and writes O^T
+        if (ngood > 0) ok = decode_wait(pv_done, (ngood - 1) & 1);
+        ok = ptx::bar_red_and(1, 128, ok);
+        if (!ok) {
+          if (tid == 0) decode_error(p, kErrDecodeWait);
+          break;
+        }
+        ptx::tc_fence_after();
+        // P^T[gh][t] as bf16, K-major with the 128-byte swizzle
+        {
+          const int half = t >> 6, c = t & 63;
+#pragma unroll
+          for (int gh = 0; gh < GT; ++gh) {
+            const uint32_t addr = p_base + half * C::QHALF + gh * 128 +
+                                  ((((c >> 3) ^ (gh & 7))) << 4) + (c & 7) * 2;
+            const __nv_bfloat16 bv = __float2bfloat16_rn(pv[gh]);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr),
+                         "h"(*reinterpret_cast<const unsigned short*>(&bv))
+                         : "memory");
+          }
+        }
+        if (nt < C::CH) {
+          // the P.V product reads all 128 V rows: rows past the chunk's tokens
+          // (stale cache rows or earlier data) become zero, so 0 * row stays 0
+          ok = decode_wait(&full_v[kc % C::NV], (kc / C::NV) & 1);
+          ok = ptx::bar_red_and(1, 128, ok);
+          if (!ok) {
+            if (tid == 0) decode_error(p, kErrDecodeWait);
+            break;
+          }
+          if (t >= nt) {
+            uint4* row = reinterpret_cast<uint4*>(sm + C::V_OFF + (kc % C::NV) * C::VSTAGE) +
+                         t * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              row[i] = make_uint4(0u, 0u, 0u, 0u);                // columns 0..63
+              row[C::HALF / 16 + i] = make_uint4(0u, 0u, 0u, 0u);  // columns 64..127
+            }
+          }
+        }
+        if (rescale) {  // uniform: every thread saw the same maxima
+          uint32_t ov[16];
+          ptx::tmem_ld16(o_addr, ov);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int gh = 0; gh < GT; ++gh) ov[gh] = __float_as_uint(__uint_as_float(ov[gh]) * alpha[gh]);
+          ptx::tmem_st16(o_addr, ov);
+          ptx::tmem_st_wait();
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(p_full);
+        ++ngood;
+        seg_good = true;
+      }
+      if (flags & kStageSegLast) {
+        const long long base = head0 * p.nslot + m[5];  // slot of head gh: + gh * nslot
+        if (seg_good) {
+          ok = decode_wait(pv_done, (ngood - 1) & 1);
+          ok = ptx::bar_red_and(1, 128, ok);
+          if (!ok) {
+            if (tid == 0) decode_error(p, kErrDecodeWait);
+            break;
+          }
+          ptx::tc_fence_after();
+          uint32_t ov[16];
+          ptx::tmem_ld16(o_addr, ov);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int gh = 0; gh < GT; ++gh)
+            p.part_o[(base + gh * p.nslot) * C::D + t] = __uint_as_float(ov[gh]);
+          if (lane == 0) {
+#pragma unroll
+            for (int gh = 0; gh < GT; ++gh) lred[warp * 16 + gh] = l_w[gh];
+          }
+          ptx::bar_sync_named(1, 128);
+          if (t < GT) {
+            float l = 0.f, mm = 0.f;
+#pragma unroll
+            for (int gh = 0; gh < GT; ++gh)
+              if (gh == t) {
+                l = lred[gh] + lred[16 + gh] + lred[32 + gh] + lred[48 + gh];
+                mm = m_run[gh];
+              }
+            float* ml = p.part_ml + (base + t * p.nslot) * 2;
+            ml[0] = mm;
+            ml[1] = l;
+          }
+          ptx::bar_sync_named(1, 128);  // lred is free again
+        } else if (t < GT) {  // every chunk of the segment was dropped
+          float* ml = p.part_ml + (base + t * p.nslot) * 2;
+          ml[0] = -INFINITY;
+          ml[1] = 0.f;
+        }
+        if ((flags & kStageItemLast) && t == 0)
+          p.slots[static_cast<long long>(m[0]) * p.Hkv * p.zgroups + m[1]] = m[5] + 1;
+#pragma unroll
+        for (int gh = 0; gh < GT; ++gh) {
+          m_run[gh] = -INFINITY;
+          l_w[gh] = 0.f;
+        }
+        seg_good = false;
+      }
+    }
+    ptx::tc_fence_before();
+    ptx::bar_arrive_named(2, 160);  // tensor memory may be released
+  }
+}
+
+}  // namespace tessera

@@ -159,6 +159,11 @@ __device__ __forceinline__ void bar_sync_named(int id, int count) {
   asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrive at named barrier `id` (expecting `count` threads) without waiting.
+__device__ __forceinline__ void bar_arrive_named(int id, int count) {
+  asm volatile("barrier.cta.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Named barrier that also returns the AND of every participant's `pred`.
 __device__ __forceinline__ bool bar_red_and(int id, int count, bool pred) {
   uint32_t r;
