@@ -373,6 +373,22 @@ bool make_cache_map(CUtensorMap* map, const void* base, long long rows, int d, i
   return r == CUDA_SUCCESS;
 }
 
+// The same cache as a 4-D tensor of 8-row atoms: (64 columns, 8 rows at 256 B,
+// 2 column halves at 128 B, rows / 8 atoms at 2 KB), 128-byte swizzle; a box
+// of box_rows / 8 atoms lands as [atom][half][8 rows][64 columns].  d = 128.
+bool make_cache_map_atoms(CUtensorMap* map, const void* base, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, 8, 2, static_cast<cuuint64_t>(rows / 8)};
+  cuuint64_t strides[3] = {256, 128, 2048};
+  cuuint32_t box[4] = {64, 8, 2, static_cast<cuuint32_t>(box_rows / 8)};
+  cuuint32_t elem[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                  strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 long long decode_chunks(int max_seq_len) {
   return (static_cast<long long>(max_seq_len) + tessera::kDecodeChunk - 1) / tessera::kDecodeChunk;
 }
@@ -494,8 +510,8 @@ int launch_decode_tc(const void* k_cache, const void* v_cache, tessera::DecodePa
   if (p.nslot > 0) {
     const long long rows = static_cast<long long>(p.num_blocks) * p.Hkv * p.bs;
     CUtensorMap tm_k, tm_v, tm_q;
-    if (!make_cache_map(&tm_k, k_cache, rows, 128, p.rows_per_box) ||
-        !make_cache_map(&tm_v, v_cache, rows, 128, p.rows_per_box) ||
+    if (!make_cache_map_atoms(&tm_k, k_cache, rows, p.rows_per_box) ||
+        !make_cache_map_atoms(&tm_v, v_cache, rows, p.rows_per_box) ||
         !make_cache_map(&tm_q, p.q, static_cast<long long>(p.B) * p.Hq, 128, GT))
       return TESSERA_ERR_CUDA;
     const int sms = sm_count(dev);

@@ -10,6 +10,13 @@
 // both accumulating in tensor memory.  The FP32 pipes keep only the softmax
 // (a thread per token), so the step stays bound by HBM.
 //
+// Layout of a K or V chunk in shared memory: 16 atoms of 8 tokens, each atom
+// [columns 0-63: 8 rows x 128 B][columns 64-127: 8 rows x 128 B] (2 KB, the
+// 128-byte swizzle inside each 1 KB half).  One 4-D TMA box (64 columns x 8
+// rows x 2 halves x R/8 atoms, the tensor viewed with row stride 256 B, half
+// stride 128 B and atom stride 2 KB) brings a whole page of R tokens, and the
+// MMA descriptors read it with an 8-row stride of 2 KB.
+//
 // Roles (192 threads): warps 0-3 softmax (thread = token for S^T and column
 // for O^T, lanes 32w.. of tensor memory), warp 4 issues the MMAs, warp 5 is
 // the producer.  Rings: K (+ the q rows) in NK stages, released when S^T is
@@ -33,11 +40,11 @@ constexpr float kDecTcRescale = 8.0f;    // log2 units
 struct DecTcCfg {
   static constexpr int D = 128;
   static constexpr int CH = kDecodeChunk;       // 128 tokens
-  static constexpr int HALF = CH * 128;         // one [128 rows][64 cols] bf16 sub-tile
+  static constexpr int ATOM = 2048;             // 8 tokens x 128 columns, halves 1 KB apart
   static constexpr int QHALF = kDecTcN * 128;   // one [16 rows][64 cols] bf16 sub-tile
-  static constexpr int K_BYTES = 2 * HALF;
+  static constexpr int K_BYTES = (CH / 8) * ATOM;
   static constexpr int KSTAGE = K_BYTES + 2 * QHALF;  // K, then the q rows
-  static constexpr int VSTAGE = 2 * HALF;
+  static constexpr int VSTAGE = (CH / 8) * ATOM;
   static constexpr int NK = 3, NV = 3;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NK * KSTAGE;
@@ -197,11 +204,8 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
       }
       __syncwarp();
       if (!bad && lane < npg) {
-        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          ptx::tma_load_2d_hint(kst + h * C::HALF + lane * R * 128, tm_k, &full_k[sk], 64 * h,
-                                row, pol);
+        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
+        ptx::tma_load_4d_hint(kst + lane * R * 256, tm_k, &full_k[sk], 0, 0, 0, row >> 3, pol);
       }
       // ---- V
       const uint32_t sv = produced % C::NV;
@@ -221,11 +225,8 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
       }
       __syncwarp();
       if (!bad && lane < npg) {
-        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          ptx::tma_load_2d_hint(vst + h * C::HALF + lane * R * 128, tm_v, &full_v[sv], 64 * h,
-                                row, pol);
+        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
+        ptx::tma_load_4d_hint(vst + lane * R * 256, tm_v, &full_v[sv], 0, 0, 0, row >> 3, pol);
       }
       ++produced;
       cur = nxt;
@@ -320,7 +321,8 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
     const bool leader = lane == 0;
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kDecTcN, false, false);
     constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, kDecTcN, true, false);
-    constexpr uint32_t kHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-byte swizzle
+    constexpr uint32_t kHi = ptx::sdesc_sw128_hi(1024);      // q, P^T: 8-row groups 1 KB apart
+    constexpr uint32_t kHiKV = ptx::sdesc_sw128_hi(C::ATOM); // K, V: 8-token atoms 2 KB apart
     const uint32_t k_base = ptx::smem_u32(sm + C::K_OFF);
     const uint32_t v_base = ptx::smem_u32(sm + C::V_OFF);
     const uint32_t p_lo = ptx::sdesc_sw128_lo(ptx::smem_u32(sm + C::P_OFF), 16);
@@ -336,11 +338,13 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
       if (!w_ok) return false;
       ptx::tc_fence_after();
       if (leader) {
-        const uint32_t va = ptx::sdesc_sw128_lo(v_base + pend_sv * C::VSTAGE, C::HALF);
-        ptx::mma_ss_lohi_rt(tmem + C::O_COL, va, kHi, p_lo, kHi, kIdescO, pend_acc);
+        // A = V (MN-major): the two 64-column halves 1 KB apart (LBO), 8-token
+        // atoms 2 KB apart (SBO); K step kk = 16 tokens = two atoms
+        const uint32_t va = ptx::sdesc_sw128_lo(v_base + pend_sv * C::VSTAGE, C::ATOM / 2);
+        ptx::mma_ss_lohi_rt(tmem + C::O_COL, va, kHiKV, p_lo, kHi, kIdescO, pend_acc);
 #pragma unroll
         for (int kk = 1; kk < C::CH / 16; ++kk)
-          ptx::mma_ss_lohi<1>(tmem + C::O_COL, va + kk * (2048 >> 4), kHi,
+          ptx::mma_ss_lohi<1>(tmem + C::O_COL, va + kk * ((2 * C::ATOM) >> 4), kHiKV,
                               p_lo + kmajor_step(kk, C::QHALF), kHi, kIdescO);
         ptx::tc_commit(&empty_v[pend_sv]);
         ptx::tc_commit(pv_done);
@@ -383,15 +387,15 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
       } else {
         ptx::tc_fence_after();
         if (leader) {
-          // S^T = K q^T: A = K (K-major, sub-tiles 16 KB apart), B = q rows
-          // (K-major, sub-tiles 2 KB apart)
+          // S^T = K q^T: A = K (K-major, column halves 1 KB apart, atoms 2 KB
+          // apart), B = q rows (K-major, column halves 2 KB apart)
           const uint32_t ka = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE, 16);
           const uint32_t qb = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE + C::K_BYTES, 16);
           const uint32_t sd = tmem + C::S_COL + kDecTcN * buf;
-          ptx::mma_ss_lohi<0>(sd, ka, kHi, qb, kHi, kIdescS);
+          ptx::mma_ss_lohi<0>(sd, ka, kHiKV, qb, kHi, kIdescS);
 #pragma unroll
           for (int kk = 1; kk < C::D / 16; ++kk)
-            ptx::mma_ss_lohi<1>(sd, ka + kmajor_step(kk, C::HALF), kHi,
+            ptx::mma_ss_lohi<1>(sd, ka + kmajor_step(kk, C::ATOM / 2), kHiKV,
                                 qb + kmajor_step(kk, C::QHALF), kHi, kIdescS);
           ptx::tc_commit(&s_full[buf]);
           ptx::tc_commit(&empty_k[sk]);
@@ -527,12 +531,12 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
             break;
           }
           if (t >= nt) {
-            uint4* row = reinterpret_cast<uint4*>(sm + C::V_OFF + (kc % C::NV) * C::VSTAGE) +
-                         t * 8;
+            uint4* row = reinterpret_cast<uint4*>(sm + C::V_OFF + (kc % C::NV) * C::VSTAGE +
+                                                  (t >> 3) * C::ATOM + (t & 7) * 128);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              row[i] = make_uint4(0u, 0u, 0u, 0u);                // columns 0..63
-              row[C::HALF / 16 + i] = make_uint4(0u, 0u, 0u, 0u);  // columns 64..127
+              row[i] = make_uint4(0u, 0u, 0u, 0u);                    // columns 0..63
+              row[C::ATOM / 32 + i] = make_uint4(0u, 0u, 0u, 0u);      // columns 64..127
             }
           }
         }
