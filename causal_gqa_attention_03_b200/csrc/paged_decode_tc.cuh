@@ -74,8 +74,8 @@ __device__ __forceinline__ uint32_t kmajor_step(int kk, int sub) {
   return static_cast<uint32_t>((kk >> 2) * (sub >> 4) + (kk & 3) * 2);
 }
 
-// Producer warp: as decode_produce, with separate K and V rings and the q
-// rows fetched by TMA with every K chunk.
+// Producer warp: as decode_produce, with separate K and V rings (V one chunk
+// behind K) and the q rows fetched by TMA with every K chunk.
 template <int GT>
 __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const CUtensorMap* tm_q, const DecodeParams& p,
@@ -134,6 +134,32 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
     };
     int blk, npg;
     load_ids(cur, blk, npg);
+    // the chunk whose V is still to issue
+    bool pv_bad = false;
+    int pv_npg = 0, pv_blk = 0, pv_row0 = 0, pv_tok0 = 0;
+    auto issue_v = [&](uint32_t idx) -> bool {
+      const uint32_t sv = idx % C::NV;
+      bool ok_v = true;
+      if (lane == 0) ok_v = decode_wait(&empty_v[sv], ((idx / C::NV) & 1) ^ 1u);
+      ok_v = __shfl_sync(0xffffffffu, ok_v, 0);
+      if (!ok_v) {
+        if (lane == 0) decode_error(p, kErrDecodeWait);
+        return false;
+      }
+      uint8_t* vst = sm + C::V_OFF + sv * C::VSTAGE;
+      if (lane == 0) {
+        if (pv_bad)
+          ptx::mbar_arrive(&full_v[sv]);
+        else
+          ptx::mbar_arrive_expect_tx(&full_v[sv], static_cast<uint32_t>(pv_npg * R * 256));
+      }
+      __syncwarp();
+      if (!pv_bad && lane < pv_npg) {
+        const int row = pv_row0 + (pv_tok0 + lane * R) % p.bs;  // a multiple of 8
+        ptx::tma_load_4d_hint(vst + lane * R * 256, tm_v, &full_v[sv], 0, 0, 0, row >> 3, pol);
+      }
+      return true;
+    };
     for (long long pos = lo; pos < hi; ++pos) {
       DecodeCursor nxt = cur;
       int nblk = 0, nnpg = 0;
@@ -207,32 +233,23 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
         const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
         ptx::tma_load_4d_hint(kst + lane * R * 256, tm_k, &full_k[sk], 0, 0, 0, row >> 3, pol);
       }
-      // ---- V
-      const uint32_t sv = produced % C::NV;
-      if (lane == 0) ok = decode_wait(&empty_v[sv], ((produced / C::NV) & 1) ^ 1u);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) decode_error(p, kErrDecodeWait);
+      // ---- V of the previous chunk (K runs one chunk ahead of V: V is needed
+      // later, and its stages are held until the chunk's P.V is done)
+      if (produced > 0 && !issue_v(produced - 1)) {
         alive = false;
         break;
       }
-      uint8_t* vst = sm + C::V_OFF + sv * C::VSTAGE;
-      if (lane == 0) {
-        if (bad)
-          ptx::mbar_arrive(&full_v[sv]);
-        else
-          ptx::mbar_arrive_expect_tx(&full_v[sv], static_cast<uint32_t>(npg * R * 256));
-      }
-      __syncwarp();
-      if (!bad && lane < npg) {
-        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
-        ptx::tma_load_4d_hint(vst + lane * R * 256, tm_v, &full_v[sv], 0, 0, 0, row >> 3, pol);
-      }
+      pv_bad = bad;
+      pv_npg = npg;
+      pv_blk = blk;
+      pv_row0 = (blk * p.Hkv + g) * p.bs;
+      pv_tok0 = tok0;
       ++produced;
       cur = nxt;
       blk = nblk;
       npg = nnpg;
     }
+    if (alive && produced > 0 && !issue_v(produced - 1)) alive = false;
   }
   if (alive && lane == 0) {
     const uint32_t sk = produced % C::NK;
@@ -331,80 +348,91 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
     uint32_t npv = 0;       // P.V products issued (p_full / pv_done phases)
     bool seg_good = false;  // the current segment has had a good chunk
     bool ok = true;
-    auto issue_pv = [&]() -> bool {
-      bool w_ok = __all_sync(0xffffffffu, decode_wait(p_full, npv & 1));
-      w_ok = w_ok && __all_sync(0xffffffffu,
-                                decode_wait(&full_v[pend_sv], (pend_kc / C::NV) & 1));
-      if (!w_ok) return false;
-      ptx::tc_fence_after();
-      if (leader) {
-        // A = V (MN-major): the two 64-column halves 1 KB apart (LBO), 8-token
-        // atoms 2 KB apart (SBO); K step kk = 16 tokens = two atoms
-        const uint32_t va = ptx::sdesc_sw128_lo(v_base + pend_sv * C::VSTAGE, C::ATOM / 2);
-        ptx::mma_ss_lohi_rt(tmem + C::O_COL, va, kHiKV, p_lo, kHi, kIdescO, pend_acc);
-#pragma unroll
-        for (int kk = 1; kk < C::CH / 16; ++kk)
-          ptx::mma_ss_lohi<1>(tmem + C::O_COL, va + kk * ((2 * C::ATOM) >> 4), kHiKV,
-                              p_lo + kmajor_step(kk, C::QHALF), kHi, kIdescO);
-        ptx::tc_commit(&empty_v[pend_sv]);
-        ptx::tc_commit(pv_done);
-      }
-      __syncwarp();
-      ++npv;
-      pending = false;
-      return true;
+    // Each step handles chunk kc (its S^T, or nothing for a dropped chunk) and
+    // the previous good chunk's P.V, in whichever order their inputs arrive,
+    // so a late K chunk does not hold back the P.V that frees a V stage.
+    auto ready = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, ptx::mbar_test_wait(bar, parity));
     };
     for (uint32_t kc = 0; ok; ++kc) {
       const uint32_t sk = kc % C::NK, buf = kc & 1;
-      ok = __all_sync(0xffffffffu, decode_wait(&full_k[sk], (kc / C::NK) & 1));
-      ok = ok && __all_sync(0xffffffffu, decode_wait(&s_free[buf], ((kc >> 1) & 1) ^ 1u));
-      if (!ok) break;
+      bool s_done = false, sentinel = false, bad = false;
       int m[8];
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!s_done || pending) {
+        bool progressed = false;
+        if (pending && ready(p_full, npv & 1) &&
+            ready(&full_v[pend_sv], (pend_kc / C::NV) & 1)) {
+          ptx::tc_fence_after();
+          if (leader) {
+            // A = V (MN-major): the two 64-column halves 1 KB apart (LBO),
+            // 8-token atoms 2 KB apart (SBO); K step kk = 16 tokens = two atoms
+            const uint32_t va = ptx::sdesc_sw128_lo(v_base + pend_sv * C::VSTAGE, C::ATOM / 2);
+            ptx::mma_ss_lohi_rt(tmem + C::O_COL, va, kHiKV, p_lo, kHi, kIdescO, pend_acc);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = kmeta[8 * sk + i];
-      if (leader) {
+            for (int kk = 1; kk < C::CH / 16; ++kk)
+              ptx::mma_ss_lohi<1>(tmem + C::O_COL, va + kk * ((2 * C::ATOM) >> 4), kHiKV,
+                                  p_lo + kmajor_step(kk, C::QHALF), kHi, kIdescO);
+            ptx::tc_commit(&empty_v[pend_sv]);
+            ptx::tc_commit(pv_done);
+          }
+          __syncwarp();
+          ++npv;
+          pending = false;
+          progressed = true;
+        }
+        if (!s_done && ready(&full_k[sk], (kc / C::NK) & 1) &&
+            ready(&s_free[buf], ((kc >> 1) & 1) ^ 1u)) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) smeta[8 * buf + i] = m[i];
+          for (int i = 0; i < 8; ++i) m[i] = kmeta[8 * sk + i];
+          if (leader) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) smeta[8 * buf + i] = m[i];
+          }
+          __syncwarp();
+          s_done = true;
+          progressed = true;
+          if (m[0] < 0) {
+            sentinel = true;  // passed on once the last P.V is issued
+          } else if (m[4] & kStageBad) {
+            bad = true;
+            // nothing to multiply: hand the stages back in order
+            ok = __all_sync(0xffffffffu, decode_wait(&full_v[kc % C::NV], (kc / C::NV) & 1));
+            if (!ok) break;
+            if (leader) {
+              ptx::mbar_arrive(&empty_k[sk]);
+              ptx::mbar_arrive(&empty_v[kc % C::NV]);
+              ptx::mbar_arrive(&s_full[buf]);
+            }
+            __syncwarp();
+          } else {
+            ptx::tc_fence_after();
+            if (leader) {
+              // S^T = K q^T: A = K (K-major, column halves 1 KB apart, atoms 2 KB
+              // apart), B = q rows (K-major, column halves 2 KB apart)
+              const uint32_t ka = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE, 16);
+              const uint32_t qb = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE + C::K_BYTES, 16);
+              const uint32_t sd = tmem + C::S_COL + kDecTcN * buf;
+              ptx::mma_ss_lohi<0>(sd, ka, kHiKV, qb, kHi, kIdescS);
+#pragma unroll
+              for (int kk = 1; kk < C::D / 16; ++kk)
+                ptx::mma_ss_lohi<1>(sd, ka + kmajor_step(kk, C::ATOM / 2), kHiKV,
+                                    qb + kmajor_step(kk, C::QHALF), kHi, kIdescS);
+              ptx::tc_commit(&s_full[buf]);
+              ptx::tc_commit(&empty_k[sk]);
+            }
+            __syncwarp();
+          }
+        }
+        if (!progressed && ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+          ok = false;
+          break;
+        }
       }
-      __syncwarp();
-      if (m[0] < 0) {  // sentinel: finish the last P.V, then pass it on
-        if (pending) ok = issue_pv();
+      if (!ok) break;
+      if (sentinel) {
         if (leader) ptx::mbar_arrive(&s_full[buf]);
         __syncwarp();
-        break;
-      }
-      const bool bad = (m[4] & kStageBad) != 0;
-      if (bad) {
-        // nothing to multiply: hand the stages back in order
-        ok = __all_sync(0xffffffffu, decode_wait(&full_v[kc % C::NV], (kc / C::NV) & 1));
-        if (!ok) break;
-        if (leader) {
-          ptx::mbar_arrive(&empty_k[sk]);
-          ptx::mbar_arrive(&empty_v[kc % C::NV]);
-          ptx::mbar_arrive(&s_full[buf]);
-        }
-        __syncwarp();
-      } else {
-        ptx::tc_fence_after();
-        if (leader) {
-          // S^T = K q^T: A = K (K-major, column halves 1 KB apart, atoms 2 KB
-          // apart), B = q rows (K-major, column halves 2 KB apart)
-          const uint32_t ka = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE, 16);
-          const uint32_t qb = ptx::sdesc_sw128_lo(k_base + sk * C::KSTAGE + C::K_BYTES, 16);
-          const uint32_t sd = tmem + C::S_COL + kDecTcN * buf;
-          ptx::mma_ss_lohi<0>(sd, ka, kHiKV, qb, kHi, kIdescS);
-#pragma unroll
-          for (int kk = 1; kk < C::D / 16; ++kk)
-            ptx::mma_ss_lohi<1>(sd, ka + kmajor_step(kk, C::ATOM / 2), kHiKV,
-                                qb + kmajor_step(kk, C::QHALF), kHi, kIdescS);
-          ptx::tc_commit(&s_full[buf]);
-          ptx::tc_commit(&empty_k[sk]);
-        }
-        __syncwarp();
-      }
-      // the previous good chunk's P.V, now that this chunk's S^T is queued
-      if (pending && !issue_pv()) {
-        ok = false;
         break;
       }
       if (!bad) {
