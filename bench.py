@@ -452,8 +452,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--decode-only", action="store_true",
-                    help="time only the paged-KV decode step (for profiling it alone)")
+    ap.add_argument("--only", choices=["decode", "prologue", "varlen"],
+                    help="time one extra leg alone and print its object (for profiling it)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -476,8 +476,8 @@ def main():
         dist.init_process_group("nccl", device_id=dev,
                                 timeout=datetime.timedelta(seconds=120))
     tess.load_library()
-    if args.decode_only:
-        return decode_only(args, tess, torch, dev, world, rank, local)
+    if args.only:
+        return one_leg(args, tess, torch, dev, world, rank, local)
 
     q_h, k_h, v_h = inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
                                     rank_seed(w.seed, rank), w.sigma_qk)
@@ -636,23 +636,31 @@ def main():
     return 0
 
 
-def decode_only(args, tess, torch, dev, world, rank, local):
-    """--decode-only: the decode step alone, one JSON line with its object."""
+def one_leg(args, tess, torch, dev, world, rank, local):
+    """--only LEG: one of the extra legs alone, one JSON line with its object."""
     import torch.distributed as dist
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    wd = inputs.DECODE
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     t0 = time.time()
-    times, launches, ws = time_decode(wd, args.steps, args.warmup, flush, stream, tess, torch, dev)
+    if args.only == "decode":
+        wd = inputs.DECODE
+        times, launches, ws = time_decode(wd, args.steps, args.warmup, flush, stream, tess, torch,
+                                          dev)
+        max_ms = max_over_ranks(sum(times), dev)
+    elif args.only == "varlen":
+        times, launches = time_varlen(inputs.VARLEN, args.steps, args.warmup, flush, stream, tess,
+                                      torch, dev)
+    else:
+        pro = time_prologue(inputs.WORKLOADS[args.workload], args.steps, args.warmup, flush,
+                            stream, tess, torch, dev)
     t1 = time.time()
     clocks.mark(t0, t1)
-    max_ms = max_over_ranks(sum(times), dev)
     err = tess.tessera_attn_device_error()
     if err != 0:
-        raise SystemExit(f"device-side error in the decode step (code {err})")
+        raise SystemExit(f"device-side error in the {args.only} leg (code {err})")
     clocks.stop()
     if world > 1:
         dist.barrier()
@@ -660,7 +668,12 @@ def decode_only(args, tess, torch, dev, world, rank, local):
     if rank != 0:
         return 0
     peaks, peak_src = load_peaks()
-    line = decode_line(wd, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
+    if args.only == "decode":
+        line = decode_line(wd, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
+    elif args.only == "varlen":
+        line = varlen_line(inputs.VARLEN, times, launches, peaks, peak_src)
+    else:
+        line = prologue_line(inputs.WORKLOADS[args.workload], pro, peaks, peak_src)
     line.update({"n_gpus": world, "warmup": args.warmup, "higher_is_better": True,
                  "scaling": "weak", "dtype": "bf16", "data": "synthetic",
                  "clocks": clocks.summary()})
