@@ -791,10 +791,8 @@ extern "C" int tessera_rmsnorm(const void* x, const void* w, void* y, int rows, 
     tessera::rmsnorm_kernel<4><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
   else if (vpt <= 8)
     tessera::rmsnorm_kernel<8><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
-  else if (vpt <= 16)
-    tessera::rmsnorm_kernel<16><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
-  else
-    tessera::rmsnorm_kernel<32><<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
+  else  // wider rows: two passes, the second from L2
+    tessera::rmsnorm_2pass_kernel<<<grid, 256, 0, s>>>(xb, wb, yb, rows, dim, eps);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = 1;
   return TESSERA_OK;

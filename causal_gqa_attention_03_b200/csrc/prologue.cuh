@@ -96,6 +96,70 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const __nv_bfloat16* __res
   }
 }
 
+// Wide rows: a warp per row in two passes, 4 vectors per lane in flight per
+// step: the sum of squares, then the scaled write from a second read, which
+// the row's recent first read leaves in L2.  64 registers (4 CTAs, 32 warps
+// per SM) instead of the 104 a 4096-wide row held in registers takes.
+__global__ void __launch_bounds__(256, 4) rmsnorm_2pass_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const __nv_bfloat16* __restrict__ w,
+                                                            __nv_bfloat16* y, long long rows,
+                                                            int dim, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int nvec = dim / 8;
+  const float inv_dim = 1.f / static_cast<float>(dim);
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < rows; r += warps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * dim);
+    float ss = 0.f;
+    for (int v0 = lane; v0 < nvec; v0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (v0 + 32 * j < nvec) v[j] = xr[v0 + 32 * j];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (v0 + 32 * j < nvec) {
+          const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = bf_lo(u[e]), b = bf_hi(u[e]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = rsqrtf(fmaf(ss, inv_dim, eps));
+    uint4* yr = reinterpret_cast<uint4*>(y + r * dim);
+    const uint4* wv = reinterpret_cast<const uint4*>(w);
+    for (int v0 = lane; v0 < nvec; v0 += 128) {
+      uint4 v[4], g[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (v0 + 32 * j < nvec) {
+          v[j] = ld_stream_v4(xr + v0 + 32 * j);  // the last read of x: evict first
+          g[j] = wv[v0 + 32 * j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (v0 + 32 * j < nvec) {
+          const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+          const uint32_t gw[4] = {g[j].x, g[j].y, g[j].z, g[j].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[e] = pack_bf2(bf_lo(u[e]) * inv * bf_lo(gw[e]), bf_hi(u[e]) * inv * bf_hi(gw[e]));
+          st_stream_v4(yr + v0 + 32 * j, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+  }
+}
+
 constexpr int kRopeTokens = 16;  // tokens per CTA
 constexpr int kRopeThreads = 256;
 
