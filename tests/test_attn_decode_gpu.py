@@ -74,6 +74,9 @@ CASES = [
     (2, 4, 2, 128, 256, [700, 256]),       # blocks larger than a chunk
     (1, 12, 4, 64, 128, [1025]),           # G = 3, d = 64
     (5, 4, 4, 128, 8, [5, 0, 131, 2048, 64]),
+    (2, 16, 2, 128, 64, [1000, 77]),       # G = 8: eight heads per item
+    (1, 32, 1, 128, 16, [300]),            # G = 32: two items of 16 heads
+    (2, 6, 2, 64, 16, [0, 0]),             # every sequence empty
 ]
 
 
