@@ -17,9 +17,9 @@
 // stride 128 B and atom stride 2 KB) brings a whole page of R tokens, and the
 // MMA descriptors read it with an 8-row stride of 2 KB.
 //
-// Roles (192 threads): warps 0-3 softmax (thread = token for S^T and column
-// for O^T, lanes 32w.. of tensor memory), warp 4 issues the MMAs, warp 5 is
-// the producer.  Rings: K (+ the q rows) in NK stages, released when S^T is
+// Roles (224 threads): warps 0-3 softmax (thread = token for S^T and column
+// for O^T, lanes 32w.. of tensor memory), warp 4 issues the MMAs, warps 5 and
+// 6 produce the K and the V ring.  Rings: K (+ the q rows) in NK stages, released when S^T is
 // done; V in NV stages, released when the chunk's P.V is done.  S^T is double
 // buffered in tensor memory; P^T is one shared-memory tile, rewritten once the
 // previous P.V has finished.  Online softmax across a segment's chunks with a
@@ -31,9 +31,9 @@
 
 namespace tessera {
 
-constexpr int kDecTcThreads = 192;
+constexpr int kDecTcThreads = 224;
 constexpr int kDecTcMmaWarp = 4;
-constexpr int kDecTcTmaWarp = 5;
+constexpr int kDecTcTmaWarp = 5;   // K (and q) producer; warp 6 produces V
 constexpr int kDecTcN = 16;              // N of both products: query heads per item, padded
 constexpr float kDecTcRescale = 8.0f;    // log2 units
 
@@ -74,14 +74,16 @@ __device__ __forceinline__ uint32_t kmajor_step(int kk, int sub) {
   return static_cast<uint32_t>((kk >> 2) * (sub >> 4) + (kk & 3) * 2);
 }
 
-// Producer warp: as decode_produce, with separate K and V rings (V one chunk
-// behind K) and the q rows fetched by TMA with every K chunk.
+// Producer warps: as decode_produce, one per ring.  Both walk the same chunk
+// stream; the K warp (is_v false) fills the K ring, with the q rows fetched by
+// TMA with every K chunk, and ends it with the sentinel; the V warp fills the
+// V ring.
 template <int GT>
 __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                               const CUtensorMap* tm_q, const DecodeParams& p,
                                               uint8_t* sm, int* kmeta, uint64_t* full_k,
                                               uint64_t* empty_k, uint64_t* full_v,
-                                              uint64_t* empty_v, int lane) {
+                                              uint64_t* empty_v, int lane, bool is_v) {
   using C = DecTcCfg;
   const int R = p.rows_per_box;
   const long long HZ = static_cast<long long>(p.Hkv) * p.zgroups;
@@ -134,32 +136,6 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
     };
     int blk, npg;
     load_ids(cur, blk, npg);
-    // the chunk whose V is still to issue
-    bool pv_bad = false;
-    int pv_npg = 0, pv_blk = 0, pv_row0 = 0, pv_tok0 = 0;
-    auto issue_v = [&](uint32_t idx) -> bool {
-      const uint32_t sv = idx % C::NV;
-      bool ok_v = true;
-      if (lane == 0) ok_v = decode_wait(&empty_v[sv], ((idx / C::NV) & 1) ^ 1u);
-      ok_v = __shfl_sync(0xffffffffu, ok_v, 0);
-      if (!ok_v) {
-        if (lane == 0) decode_error(p, kErrDecodeWait);
-        return false;
-      }
-      uint8_t* vst = sm + C::V_OFF + sv * C::VSTAGE;
-      if (lane == 0) {
-        if (pv_bad)
-          ptx::mbar_arrive(&full_v[sv]);
-        else
-          ptx::mbar_arrive_expect_tx(&full_v[sv], static_cast<uint32_t>(pv_npg * R * 256));
-      }
-      __syncwarp();
-      if (!pv_bad && lane < pv_npg) {
-        const int row = pv_row0 + (pv_tok0 + lane * R) % p.bs;  // a multiple of 8
-        ptx::tma_load_4d_hint(vst + lane * R * 256, tm_v, &full_v[sv], 0, 0, 0, row >> 3, pol);
-      }
-      return true;
-    };
     for (long long pos = lo; pos < hi; ++pos) {
       DecodeCursor nxt = cur;
       int nblk = 0, nnpg = 0;
@@ -194,64 +170,77 @@ __device__ __forceinline__ void dectc_produce(const CUtensorMap* tm_k, const CUt
       const int nt = min(C::CH, cur.n - cur.c * C::CH);
       const int g = cur.gz / p.zgroups, z = cur.gz % p.zgroups;
       const int tok0 = cur.c * C::CH;
-      // ---- K and the q rows
-      const uint32_t sk = produced % C::NK;
-      bool ok = true;
-      if (lane == 0) {
-        if (bad) decode_error(p, kErrDecodeInput);
-        ok = decode_wait(&empty_k[sk], ((produced / C::NK) & 1) ^ 1u);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) decode_error(p, kErrDecodeWait);
-        alive = false;
-        break;
-      }
-      uint8_t* kst = sm + C::K_OFF + sk * C::KSTAGE;
-      if (lane == 0) {
-        int* m = kmeta + 8 * sk;
-        m[0] = cur.b;
-        m[1] = cur.gz;
-        m[2] = cur.c;
-        m[3] = nt;
-        m[4] = flags;
-        m[5] = static_cast<int>(blockIdx.x - cur.item0 / per);
-        if (bad) {
-          ptx::mbar_arrive(&full_k[sk]);
-        } else {
-          ptx::mbar_arrive_expect_tx(&full_k[sk],
-                                     static_cast<uint32_t>(npg * R * 256 + GT * 256));
-          const int qrow = (cur.b * p.Hq + g * p.G + z * GT);
+      if (!is_v) {
+        // ---- K and the q rows
+        const uint32_t sk = produced % C::NK;
+        bool ok = true;
+        if (lane == 0) {
+          if (bad) decode_error(p, kErrDecodeInput);
+          ok = decode_wait(&empty_k[sk], ((produced / C::NK) & 1) ^ 1u);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) decode_error(p, kErrDecodeWait);
+          alive = false;
+          break;
+        }
+        uint8_t* kst = sm + C::K_OFF + sk * C::KSTAGE;
+        if (lane == 0) {
+          int* m = kmeta + 8 * sk;
+          m[0] = cur.b;
+          m[1] = cur.gz;
+          m[2] = cur.c;
+          m[3] = nt;
+          m[4] = flags;
+          m[5] = static_cast<int>(blockIdx.x - cur.item0 / per);
+          if (bad) {
+            ptx::mbar_arrive(&full_k[sk]);
+          } else {
+            ptx::mbar_arrive_expect_tx(&full_k[sk],
+                                       static_cast<uint32_t>(npg * R * 256 + GT * 256));
+            const int qrow = (cur.b * p.Hq + g * p.G + z * GT);
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            ptx::tma_load_2d_hint(kst + C::K_BYTES + h * C::QHALF, tm_q, &full_k[sk], 64 * h,
-                                  qrow, keep);
+            for (int h = 0; h < 2; ++h)
+              ptx::tma_load_2d_hint(kst + C::K_BYTES + h * C::QHALF, tm_q, &full_k[sk], 64 * h,
+                                    qrow, keep);
+          }
+        }
+        __syncwarp();
+        if (!bad && lane < npg) {
+          const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
+          ptx::tma_load_4d_hint(kst + lane * R * 256, tm_k, &full_k[sk], 0, 0, 0, row >> 3, pol);
+        }
+      } else {
+        // ---- V
+        const uint32_t sv = produced % C::NV;
+        bool ok = true;
+        if (lane == 0) ok = decode_wait(&empty_v[sv], ((produced / C::NV) & 1) ^ 1u);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) decode_error(p, kErrDecodeWait);
+          alive = false;
+          break;
+        }
+        uint8_t* vst = sm + C::V_OFF + sv * C::VSTAGE;
+        if (lane == 0) {
+          if (bad)
+            ptx::mbar_arrive(&full_v[sv]);
+          else
+            ptx::mbar_arrive_expect_tx(&full_v[sv], static_cast<uint32_t>(npg * R * 256));
+        }
+        __syncwarp();
+        if (!bad && lane < npg) {
+          const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
+          ptx::tma_load_4d_hint(vst + lane * R * 256, tm_v, &full_v[sv], 0, 0, 0, row >> 3, pol);
         }
       }
-      __syncwarp();
-      if (!bad && lane < npg) {
-        const int row = (blk * p.Hkv + g) * p.bs + (tok0 + lane * R) % p.bs;  // multiple of 8
-        ptx::tma_load_4d_hint(kst + lane * R * 256, tm_k, &full_k[sk], 0, 0, 0, row >> 3, pol);
-      }
-      // ---- V of the previous chunk (K runs one chunk ahead of V: V is needed
-      // later, and its stages are held until the chunk's P.V is done)
-      if (produced > 0 && !issue_v(produced - 1)) {
-        alive = false;
-        break;
-      }
-      pv_bad = bad;
-      pv_npg = npg;
-      pv_blk = blk;
-      pv_row0 = (blk * p.Hkv + g) * p.bs;
-      pv_tok0 = tok0;
       ++produced;
       cur = nxt;
       blk = nblk;
       npg = nnpg;
     }
-    if (alive && produced > 0 && !issue_v(produced - 1)) alive = false;
   }
-  if (alive && lane == 0) {
+  if (alive && !is_v && lane == 0) {
     const uint32_t sk = produced % C::NK;
     if (decode_wait(&empty_k[sk], ((produced / C::NK) & 1) ^ 1u)) {
       kmeta[8 * sk] = -1;
@@ -330,9 +319,9 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kDecTcTmaWarp) {
+  if (warp == kDecTcTmaWarp || warp == kDecTcTmaWarp + 1) {
     dectc_produce<GT>(&tm_k, &tm_v, &tm_q, p, sm, kmeta, full_k, empty_k, full_v, empty_v,
-                      lane);
+                      lane, warp == kDecTcTmaWarp + 1);
   } else if (warp == kDecTcMmaWarp) {
     // ======================= MMA issue (lane 0; the warp waits) ===========
     const bool leader = lane == 0;
