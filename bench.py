@@ -177,6 +177,87 @@ def oracle_rows_rate(w, q, k, v, seconds: float, seed: int, max_rows: int | None
     return flops / el / 1e12, rows_done, flops, el
 
 
+# Host copies of small parts of the extra legs' inputs, kept for the oracle's
+# timing (filled by the time_* functions).
+SAMPLES = {}
+
+
+def leg_cpu_baselines(w, q_h, k_h, v_h, seconds: float):
+    """The fp64 oracle timed on bounded samples of each extra leg's own
+    workload (single thread), in each leg's unit."""
+    import numpy as np
+    import oracle
+    out = {}
+
+    def timed(fn):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return n, el
+
+    # backward: random dQ rows of the headline workload (6*d*(i+1) flops each:
+    # the score row, the dP row and the dQ row)
+    g_h = inputs.make_grad(w.B, w.Hq, w.T, w.d, w.seed + inputs.GRAD_SEED_OFFSET)
+    qb, kb, vb, gb = (inputs.bf16_bits(t) for t in (q_h, k_h, v_h, g_h))
+    rng = np.random.default_rng(2)
+    fl = [0.0]
+
+    def bwd_rows():
+        rows = np.stack([rng.integers(0, w.B, 8), rng.integers(0, w.Hq, 8),
+                         rng.integers(0, w.T, 8)], axis=1).astype(np.int64)
+        rows = rows[np.lexsort((rows[:, 2], rows[:, 1], rows[:, 0]))]
+        oracle.attn_bwd_dq_rows_bf16(qb, kb, vb, gb, rows, causal=True, scale=w.scale)
+        fl[0] += float(np.sum(6.0 * w.d * (rows[:, 2] + 1)))
+
+    n, el = timed(bwd_rows)
+    out["backward"] = {"value": fl[0] / el / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+                       "sample": f"{8 * n} random dQ rows of {w.name} in {el:.1f}s "
+                                 "(6*d*(i+1) flops per row), fp64, single thread"}
+    if "decode" in SAMPLES:
+        qd, sk, sv, st_, sn = SAMPLES["decode"]
+        qn, skn, svn = qd.double().numpy(), sk.double().numpy(), sv.double().numpy()
+        wd = inputs.DECODE
+        nbytes = float(int(sn.sum()) * wd.Hkv * wd.d * 4 + 2 * len(sn) * wd.Hq * wd.d * 2)
+        n, el = timed(lambda: oracle.paged_decode_f64(qn, skn, svn, st_, sn, scale=wd.scale))
+        out["decode"] = {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": 1,
+                         "kind": "oracle",
+                         "sample": f"{len(sn)} sequences ({int(sn.sum())} tokens) of {wd.name}, "
+                                   f"{n} steps in {el:.1f}s, fp64, single thread"}
+    if "varlen" in SAMPLES:
+        qv, kv, vv = (inputs.bf16_bits(t) for t in SAMPLES["varlen"])
+        T = qv.shape[2]
+        wv = inputs.VARLEN
+        fl = [0.0]
+
+        def vrows():
+            rows = np.stack([np.zeros(8, np.int64), rng.integers(0, wv.Hq, 8),
+                             rng.integers(0, T, 8)], axis=1).astype(np.int64)
+            rows = rows[np.lexsort((rows[:, 2], rows[:, 1], rows[:, 0]))]
+            oracle.attn_rows_bf16(qv, kv, vv, rows, causal=True, scale=wv.scale)
+            fl[0] += float(np.sum(4.0 * wv.d * (rows[:, 2] + 1)))
+
+        n, el = timed(vrows)
+        out["varlen"] = {"value": fl[0] / el / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{8 * n} random rows of the longest sequence ({T} tokens) of "
+                                   f"{wv.name} in {el:.1f}s, fp64, single thread"}
+    if "prologue" in SAMPLES:
+        x, wn, qkv = SAMPLES["prologue"]
+        xn, wnn, qkvn = x.double().numpy(), wn.double().numpy(), qkv.double().numpy()
+        n, el = timed(lambda: oracle.rmsnorm_f64(xn, wnn, 1e-6))
+        rms = {"value": (4.0 * x.numel()) * n / el / 1e9, "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "sample": f"{x.shape[0]} rows of {x.shape[1]}, {n} times in "
+                                           f"{el:.1f}s, fp64, single thread"}
+        n, el = timed(lambda: oracle.rope_qkv_f64(qkvn, w.Hq, w.Hkv))
+        rope = {"value": (4.0 * qkv.numel()) * n / el / 1e9, "unit": "GB/s", "cores": 1,
+                "kind": "oracle", "sample": f"{qkv.shape[1]} tokens x {w.Hq + 2 * w.Hkv} heads, "
+                                            f"{n} times in {el:.1f}s, fp64, single thread"}
+        out["prologue"] = {"rmsnorm": rms, "rope_qkv": rope}
+    return out
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -291,6 +372,11 @@ def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
+    # two sequences of the batch, copied to the host, for the oracle's timing
+    tab_h, lens_h = table.cpu().numpy(), lens.cpu().numpy()
+    pick = [int(lens_h.argmax()), int(len(lens_h) // 2)]
+    sk, sv, st_, sn = inputs.gather_sequences(tab_h, lens_h, pick, wd.bs, kc, vc)
+    SAMPLES["decode"] = (q[pick].cpu(), sk, sv, st_, sn)
     del q, kc, vc, table, lens, o, lse, ws
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
 
@@ -335,6 +421,7 @@ def time_prologue(w, steps, warmup, flush, stream, tess, torch, dev):
             ends[i].record(stream)
         torch.cuda.synchronize()
         out[name] = ([s_.elapsed_time(e) for s_, e in zip(starts, ends)], nbytes, launches)
+    SAMPLES["prologue"] = (x[:64].cpu(), wn.cpu(), qkv[:, :16].contiguous().cpu())
     del x, wn, y, qkv, q, k, v
     return out
 
@@ -390,6 +477,10 @@ def time_varlen(wv, steps, warmup, flush, stream, tess, torch, dev):
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
+    b = max(range(len(lens)), key=lambda i: lens[i])
+    s0 = sum(lens[:b])
+    SAMPLES["varlen"] = tuple(t[s0:s0 + lens[b]].permute(1, 0, 2).contiguous()[None].cpu()
+                              for t in (q, k, v))
     del q, k, v, o, lse
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches
 
@@ -595,11 +686,13 @@ def main():
                 "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes}
 
     cpu = None
+    leg_cpu = {}
     if not args.no_cpu_baseline and world == 1:
         rate, rows, _, el = oracle_rows_rate(w, q_h, k_h, v_h, args.cpu_seconds, seed=1)
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{rows} random (b,h,i) rows of {w.name} in {el:.1f}s, "
                          "fp64, single thread"}
+        leg_cpu = leg_cpu_baselines(w, q_h, k_h, v_h, seconds=3.0)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -632,6 +725,12 @@ def main():
         "clocks": clk,
         "sweep": sweep or None,
     }
+    for leg, base in leg_cpu.items():
+        if leg == "prologue":
+            for kname, kb_ in base.items():
+                line["prologue"][kname]["cpu_baseline"] = kb_
+        else:
+            line[leg]["cpu_baseline"] = base
     print(json.dumps(line), flush=True)
     return 0
 
