@@ -215,10 +215,9 @@ HostPipe* host_pipe(int dev) {
   return &h;
 }
 
-// Bytes of fp32 workspace the backward needs: the dQ accumulator
-// [B,Hq,T,d] and D [B,Hq,T].
-size_t bwd_workspace_bytes(int B, int Hq, int T, int d) {
-  return static_cast<size_t>(B) * Hq * T * (static_cast<size_t>(d) + 1) * 4;
+// Bytes of fp32 workspace the backward needs: D = rowsum(dO * O) [B,Hq,T].
+size_t bwd_workspace_bytes(int B, int Hq, int T, int /*d*/) {
+  return static_cast<size_t>(B) * Hq * T * 4;
 }
 
 int sm_count(int dev) {
@@ -238,33 +237,34 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                const void* dout, void* dq, void* dk, void* dv, float* ws, int B, int Hq, int Hkv,
                int T, int causal, float scale, cudaStream_t stream) {
   using C = BwdCfg<D>;
+  using Q = tessera::DqCfg<D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
   static std::atomic<int> attr_set[64];
   if (attr_set[dev].load(std::memory_order_acquire) == 0) {
     if (cudaFuncSetAttribute(tessera::attn_bwd_dkdv_sm100_kernel<D>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
+                             C::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(tessera::attn_bwd_dq_sm100_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Q::SMEM_BYTES) != cudaSuccess)
       return TESSERA_ERR_CUDA;
     attr_set[dev].store(1, std::memory_order_release);
   }
   const int sms = sm_count(dev);
   if (sms <= 0) return TESSERA_ERR_CUDA;
   const long long rows = static_cast<long long>(B) * Hq * T;
-  float* dq_acc = ws;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
   if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
       !make_map(&tm_v, v, B * Hkv, T, D) || !make_map(&tm_do, dout, B * Hq, T, D))
     return TESSERA_ERR_CUDA;
-  float* dvec = ws + rows * D;
-  // 1. D = rowsum(dO * O), dQ accumulator = 0
+  float* dvec = ws;
+  // 1. D = rowsum(dO * O)
   const long long prep_blocks = (rows + 7) / 8;  // 8 warps (rows) per block
   const unsigned pb = static_cast<unsigned>(prep_blocks < 4L * sms * 16 ? prep_blocks : 4L * sms * 16);
   tessera::attn_bwd_prep_kernel<D><<<pb, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dvec, dq_acc,
-      rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dvec, rows);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-  // 2. dK, dV and the dQ partials
   BwdParams p;
   p.B = B;
   p.Hq = Hq;
@@ -275,25 +275,27 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.nqb = (T + C::BM - 1) / C::BM;
-  const long long units = static_cast<long long>(B) * Hkv * p.nqb;
-  if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
-  p.num_units = static_cast<int>(units);
   p.lse = lse;
   p.dvec = dvec;
-  p.dq_acc = dq_acc;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  // 2. dK, dV: units (batch, key/value head, key block)
+  const long long kv_units = static_cast<long long>(B) * Hkv * p.nqb;
+  const long long q_units = static_cast<long long>(B) * Hq * p.nqb;
+  if (q_units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
+  p.num_units = static_cast<int>(kv_units);
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
-  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+  const unsigned grid = static_cast<unsigned>(kv_units < sms ? kv_units : sms);
   tessera::attn_bwd_dkdv_sm100_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
       tm_q, tm_k, tm_v, tm_do, p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-  // 3. dQ = bf16(scale * accumulator)
-  const long long n8 = rows * D / 8;
-  const long long cb = (n8 + 255) / 256;
-  const unsigned cg = static_cast<unsigned>(cb < 4L * sms * 8 ? cb : 4L * sms * 8);
-  tessera::attn_bwd_dq_convert_kernel<<<cg, 256, 0, stream>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+  // 3. dQ: units (batch, query head, query block)
+  p.num_units = static_cast<int>(q_units);
+  p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
+  const unsigned qgrid = static_cast<unsigned>(q_units < sms ? q_units : sms);
+  tessera::attn_bwd_dq_sm100_kernel<D><<<qgrid, Q::THREADS, Q::SMEM_BYTES, stream>>>(
+      tm_q, tm_k, tm_v, tm_do, p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = 3;
   return TESSERA_OK;
@@ -336,7 +338,7 @@ int check_bwd_args(const void* q, const void* k, const void* v, const void* o, c
 // Workspace of tessera_attn_bwd_noalloc: a device array of the library's own
 // module (one per device, set up when the module loads), so that entry point
 // needs no allocation.  Calls that overlap in time on one device share it.
-constexpr size_t kNoAllocScratchBytes = 272ull << 20;
+constexpr size_t kNoAllocScratchBytes = 16ull << 20;
 __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
 
 // Address of g_bwd_scratch on the current device (looked up once per device).

@@ -3,46 +3,30 @@
 //
 // Method: the exact gradient of the forward (chain rule through the row
 // softmax), computed tile by tile from the saved LSE as FlashAttention does:
-//   P^T  = exp(scale*K Q^T - LSE)          (keys x queries, recomputed)
-//   dP^T = V dO^T
-//   dS^T = P^T * (dP^T - D),  D_i = <dO_i, O_i>
+//   P    = exp(scale*Q K^T - LSE)          (recomputed, never stored)
+//   dP   = dO V^T
+//   dS   = P * (dP - D),  D_i = <dO_i, O_i>
 //   dV  += P^T dO,   dK += scale * dS^T Q,   dQ += scale * dS K
 // The pages list the attention backward as not yet built; the forward it
 // differentiates is the FlashAttention forward they name (hysenlabs.com
 // Tessera review, "The kernel set and its torch fallback").
 //
-// Three launches:
-//   1. attn_bwd_prep_kernel: D = rowsum(dO * O) in fp32; zeroes the fp32 dQ
-//      accumulator.
+// Three launches, no atomics and no fp32 accumulator in global memory:
+//   1. attn_bwd_prep_kernel: D = rowsum(dO * O) in fp32.
 //   2. attn_bwd_dkdv_sm100_kernel<D>: one CTA per SM walks units
 //      (batch, key/value head, 128-key block), heaviest first.  A unit keeps
 //      its K and V tiles in shared memory and its dK, dV accumulators in
 //      tensor memory while it visits every (query head of the group, 128-row
-//      query block) the keys are visible to; each visit adds its dQ partial
-//      (128 rows x D, fp32) into the accumulator with vector reductions,
-//      issued by a warpgroup of their own so that they overlap the next
-//      visits (the reductions are bound by L2 throughput, ~4,000 cycles per
-//      visit, about the time of the rest of a visit).
-//   3. attn_bwd_dq_convert_kernel: dQ = bf16(scale * accumulator).
-//
-// Kernel 2 warp roles (384 threads):
-//   warps 0-3   compute: P^T, dS^T (thread r owns key row r), then dK, dV
-//   warp  4     MMA issue (lane 0) and TMEM allocation
-//   warp  5     TMA producer (lane 0)
-//   warps 6-7   idle
-//   warps 8-11  dQ read-out: thread r loads query row r of the dQ partial from
-//               TMEM, frees the columns, then adds it into the accumulator
-// Tensor memory (512 columns):
-//   S^T  [0, 128)      P^T (bf16 pairs) written over its first 64 columns;
-//                      the dQ partial (D columns) written over it afterwards
-//   dP^T [128, 256)    dS^T (bf16 pairs) written over its first 64 columns
-//   dV   [256, 256 + D),  dK  [256 + D, 256 + 2 D)
-// Per visit the MMA warp issues S^T = K Q^T and dP^T = V dO^T, waits for P^T
-// and dS^T, then issues dV += P^T dO, dK += dS^T Q and dQp = dS K (A = dS from
-// shared memory, written there by the compute warps in the 128-byte swizzled
-// layout the MMA reads).  tcgen05 MMAs from one thread run in order, so dQp
-// overwrites P^T only after dV has read it; the next visit's S^T waits until
-// the read-out warps have loaded dQp into registers.
+//      query block) the keys are visible to, with keys as the MMA rows:
+//      S^T = K Q^T, dP^T = V dO^T, then dV += P^T dO, dK += dS^T Q.
+//   3. attn_bwd_dq_sm100_kernel<D>: one CTA per SM walks units (batch, query
+//      head, 128-row query block), heaviest first, like the forward: per key
+//      block S = Q K^T and dP = dO V^T (both recomputed), dS, then
+//      dQ += dS K into tensor memory; dQ is written once, in bf16.
+// Kernel 3 recomputes two products that kernel 2 also forms (seven products
+// per query/key block pair instead of five); in exchange no dQ partial ever
+// goes through L2 reductions, which bound the single-kernel form (a 64 KB
+// fp32 partial per visit).
 #pragma once
 
 #include "attn_fwd_sm100.cuh"
@@ -50,15 +34,58 @@
 namespace tessera {
 
 enum BwdWaitCode : uint32_t {
-  kErrBwdKv = 11,      // K/V tiles of a unit
-  kErrBwdStage = 12,   // Q/dO stage full or empty
-  kErrBwdS = 13,       // S^T and dP^T complete
-  kErrBwdP = 14,       // P^T and dS^T written
-  kErrBwdDq = 15,      // dQ partial complete or read out
-  kErrBwdDkv = 16,     // dK, dV complete
+  kErrBwdKv = 11,      // K/V tiles (kernel 2: of a unit; kernel 3: ring stages)
+  kErrBwdStage = 12,   // Q/dO tiles full or empty
+  kErrBwdS = 13,       // S (S^T) complete
+  kErrBwdP = 14,       // P^T written (kernel 2); dP read (kernel 3)
+  kErrBwdDq = 15,      // dS written; dP complete
+  kErrBwdDkv = 16,     // dK, dV (kernel 2) or dQ (kernel 3) complete
   kErrBwdDrain = 17,
 };
 
+// ------------------------------------------------------------------ kernel 1
+// D[row] = sum_c dO[row,c] * O[row,c] (fp32), one warp per row.  rows = B*Hq*T.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                            const __nv_bfloat16* __restrict__ dout,
+                                                            float* __restrict__ dvec,
+                                                            long long rows) {
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long long r = wid; r < rows; r += warps) {
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(o + r * D);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(dout + r * D);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = lane; c < D / 2; c += 32) {
+      const float2 a = __bfloat1622float2(o2[c]);
+      const float2 b = __bfloat1622float2(g2[c]);
+      acc = fmaf(a.x, b.x, acc);
+      acc = fmaf(a.y, b.y, acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) dvec[r] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ kernel 2
+// Warp roles (256 threads):
+//   warps 0-3   compute: P^T, dS^T (thread r owns key row r), then dK, dV
+//   warp  4     MMA issue (lane 0) and TMEM allocation
+//   warp  5     TMA producer (lane 0)
+//   warps 6-7   idle
+// Tensor memory (512 columns):
+//   S^T  [0, 128)      P^T (bf16 pairs) written over its first 64 columns
+//   dP^T [128, 256)    dS^T (bf16 pairs) written over its first 64 columns
+//   dV   [256, 256 + D),  dK  [256 + D, 256 + 2 D)
+// Per visit v the MMA warp issues, in this order:
+//   (once P^T(v) is written)  dV += P^T(v) dO(v), then S^T(v+1);
+//   (once dS^T(v) is written) dK += dS^T(v) Q(v), then dP^T(v+1).
+// tcgen05 MMAs from one thread run in order, so S^T(v+1) overwrites P^T(v)
+// only after dV has read it, and dP^T(v+1) overwrites dS^T(v) only after dK
+// has; the compute warps form P^T(v+1) while dK(v) and dP^T(v+1) run.
 template <int D>
 struct BwdCfg {
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
@@ -71,12 +98,10 @@ struct BwdCfg {
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = TILE_BYTES;
   static constexpr int QDO_OFF = 2 * TILE_BYTES;   // stage s: Q at +2s tiles, dO at +2s+1
-  static constexpr int DS_OFF = QDO_OFF + NST * 2 * TILE_BYTES;
-  static constexpr int DS_BYTES = 128 * 128 * 2;   // dS [keys][queries], two 64-query sub-tiles
-  static constexpr int LD_OFF = DS_OFF + DS_BYTES; // LSE*log2(e) [128], D [128]
+  static constexpr int LD_OFF = QDO_OFF + NST * 2 * TILE_BYTES;  // LSE*log2(e) [128], D [128]
   static constexpr int BAR_OFF = LD_OFF + 2 * 128 * 4;
-  // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, p_full, dq_full,
-  // dq_free, dkv_full, drain
+  // kv_full, kv_empty, st_full[NST], st_empty[NST], s_full, dp_full, p_full,
+  // ds_full, dkv_full, drain
   static constexpr int NBAR = 2 + 2 * NST + 6;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack to align the base to 1 KB
@@ -85,10 +110,9 @@ struct BwdCfg {
   static constexpr int DPT_COL = 128;
   static constexpr int DV_COL = 256;
   static constexpr int DK_COL = 256 + D;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 256;
   static constexpr int MMA_WARP = 4;
   static constexpr int TMA_WARP = 5;
-  static constexpr int READ_WARP0 = 8;  // warps 8-11: lane quadrant = warp % 4
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DK_COL + D <= 512, "tensor memory budget");
 };
@@ -99,10 +123,10 @@ struct BwdParams {
   float scale_log2;          // scale * log2(e)
   float scale;
   int nqb;                   // ceil(T / 128): query blocks and key blocks
-  int num_units;             // B * Hkv * nqb
+  int num_units;             // kernel 2: B * Hkv * nqb; kernel 3: B * Hq * nqb
   const float* lse;          // [B, Hq, T]
   const float* dvec;         // D = rowsum(dO * O) [B, Hq, T]
-  float* dq_acc;             // [B, Hq, T, D] fp32
+  __nv_bfloat16* dq;         // [B, Hq, T, D]
   __nv_bfloat16* dk;         // [B, Hkv, T, D]
   __nv_bfloat16* dv;
   unsigned long long launch_id;
@@ -127,6 +151,7 @@ __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdParams& p, int u) {
   return w;
 }
 
+// The k-th unit of this CTA (snake order over the heaviest-first list), or -1.
 __device__ __forceinline__ int bwd_unit_of(const BwdParams& p, int k) {
   const int c = (k & 1) ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
                         : static_cast<int>(blockIdx.x);
@@ -141,68 +166,6 @@ __device__ __forceinline__ void bwd_visit(const BwdParams& p, const BwdUnit& w, 
   head = w.g * p.G + v % p.G;
 }
 
-// ------------------------------------------------------------------ kernel 1
-// D[row] = sum_c dO[row,c] * O[row,c] (fp32), one warp per row; and the fp32
-// dQ accumulator set to zero.  rows = B*Hq*T.
-template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
-                                                            const __nv_bfloat16* __restrict__ dout,
-                                                            float* __restrict__ dvec,
-                                                            float* __restrict__ dq_acc,
-                                                            long long rows) {
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  for (long long r = wid; r < rows; r += warps) {
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(o + r * D);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(dout + r * D);
-    float acc = 0.f;
-#pragma unroll
-    for (int c = lane; c < D / 2; c += 32) {
-      const float2 a = __bfloat1622float2(o2[c]);
-      const float2 b = __bfloat1622float2(g2[c]);
-      acc = fmaf(a.x, b.x, acc);
-      acc = fmaf(a.y, b.y, acc);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) dvec[r] = acc;
-    float4* z = reinterpret_cast<float4*>(dq_acc + r * D);
-#pragma unroll
-    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
-// ------------------------------------------------------------------ kernel 3
-// dQ = bf16(scale * acc), 8 elements per thread step.
-__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ acc,
-                                                                  __nv_bfloat16* __restrict__ dq,
-                                                                  long long n8, float scale) {
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += stride) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-    uint4 r;
-    r.x = ptx::pack_bf16x2(a.x * scale, a.y * scale);
-    r.y = ptx::pack_bf16x2(a.z * scale, a.w * scale);
-    r.z = ptx::pack_bf16x2(b.x * scale, b.y * scale);
-    r.w = ptx::pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = r;
-  }
-}
-
-// Byte offset of dS[key r][query c .. c + 7] (16-byte chunk) in the dS tile:
-// two sub-tiles of 64 queries, each [128 keys][64 queries] with the 128-byte
-// swizzle (8-row atoms of 1 KB; chunk j of row r stored at chunk j ^ (r % 8)).
-__device__ __forceinline__ uint32_t ds_chunk_offset(int r, int c) {
-  const int sub = c >> 6;
-  const int chunk = (c & 63) >> 3;
-  return static_cast<uint32_t>(sub * (128 * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
-                               ((chunk ^ (r & 7)) << 4));
-}
-
-// ------------------------------------------------------------------ kernel 2
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -217,7 +180,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint8_t* sK = smem + C::K_OFF;
   uint8_t* sV = smem + C::V_OFF;
   uint8_t* sQdO = smem + C::QDO_OFF;
-  uint8_t* sDS = smem + C::DS_OFF;
   float* sLse = reinterpret_cast<float*>(smem + C::LD_OFF);
   float* sD = sLse + 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -226,9 +188,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint64_t* st_full = bars + 2;
   uint64_t* st_empty = st_full + C::NST;
   uint64_t* s_full = st_empty + C::NST;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* dq_full = s_full + 2;
-  uint64_t* dq_free = s_full + 3;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* ds_full = s_full + 3;
   uint64_t* dkv_full = s_full + 4;
   uint64_t* drain = s_full + 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SLOT_OFF);
@@ -244,9 +206,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       ptx::mbar_init(&st_empty[s], 1);
     }
     ptx::mbar_init(s_full, 1);
-    ptx::mbar_init(p_full, 4);   // one arrival per compute warp
-    ptx::mbar_init(dq_full, 1);
-    ptx::mbar_init(dq_free, 4);   // one arrival per read-out warp
+    ptx::mbar_init(dp_full, 1);
+    ptx::mbar_init(p_full, 4);    // one arrival per compute warp
+    ptx::mbar_init(ds_full, 4);
     ptx::mbar_init(dkv_full, 1);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
@@ -324,84 +286,84 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const bool leader = lane == 0;
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
     constexpr uint32_t kIdescG = ptx::idesc_bf16_f32(128, D, false, true);     // dV, dK (A TMEM)
-    constexpr uint32_t kIdescQ = ptx::idesc_bf16_f32(128, D, true, true);      // dQp = dS K
     constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);  // SBO 1 KB, 128-B swizzle
     const uint32_t k_addr = ptx::smem_u32(sK);
     const uint32_t v_addr = ptx::smem_u32(sV);
     const uint32_t qdo_addr = ptx::smem_u32(sQdO);
-    const uint32_t ds_addr = ptx::smem_u32(sDS);
-    int vis = 0;    // visits issued so far (stage ring position; s_full/p_full/dq phases)
+    // X^T = Y Z^T into TMEM column col: Y (K or V) and Z (Q or dO) both
+    // K-major (d innermost); K step kk is 32 B, or the next 16 KB sub-tile.
+    auto issue_t = [&](uint32_t col, uint32_t y_addr, uint32_t z_addr) {
+      const uint32_t ya = ptx::sdesc_sw128_lo(y_addr, 16);
+      const uint32_t zb = ptx::sdesc_sw128_lo(z_addr, 16);
+      ptx::mma_ss_lohi<0>(tmem + col, ya, kDescHi, zb, kDescHi, kIdescS);
+#pragma unroll
+      for (int kk = 1; kk < D / 16; ++kk) {
+        const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
+        ptx::mma_ss_lohi<1>(tmem + col, ya + st, kDescHi, zb + st, kDescHi, kIdescS);
+      }
+    };
+    // G += A^T Z into TMEM column col: A from TMEM column a_col (bf16 pairs,
+    // K = queries, 8 columns per 16), Z (dO or Q) with queries as K and d as
+    // N (MN-major); K step kk is 16 query rows = 2 KB further into the tile.
+    auto issue_g = [&](uint32_t col, uint32_t a_col, uint32_t z_addr, uint32_t first) {
+      const uint32_t zb = ptx::sdesc_sw128_lo(z_addr, C::SUB_BYTES);
+      ptx::mma_ts_lohi_rt(tmem + col, tmem + a_col, zb, kDescHi, kIdescG, first);
+#pragma unroll
+      for (int kk = 1; kk < 8; ++kk)
+        ptx::mma_ts_lohi<1>(tmem + col, tmem + a_col + kk * 8, zb + kk * (2048 >> 4), kDescHi,
+                            kIdescG);
+    };
+    int vis = 0;    // visits issued so far (stage ring position; barrier phases)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = bwd_unit_of(p, k);
       if (u < 0) break;
       const BwdUnit w = decode_bwd_unit(p, u);
       if (!warp_wait(kv_full, k & 1, kErrBwdKv, p.launch_id)) break;
+      // the unit's first S^T and dP^T
+      if (!warp_wait(&st_full[vis % C::NST], (vis / C::NST) & 1, kErrBwdStage, p.launch_id))
+        break;
+      ptx::tc_fence_after();
+      if (leader) {
+        const uint32_t q_addr = qdo_addr + (vis % C::NST) * 2 * C::TILE_BYTES;
+        issue_t(C::ST_COL, k_addr, q_addr);
+        ptx::tc_commit(s_full);
+        issue_t(C::DPT_COL, v_addr, q_addr + C::TILE_BYTES);
+        ptx::tc_commit(dp_full);
+      }
+      __syncwarp();
       for (int v = 0; v < w.nvisit; ++v, ++vis) {
         const int s = vis % C::NST;
-        ok = warp_wait(&st_full[s], (vis / C::NST) & 1, kErrBwdStage, p.launch_id);
-        // the previous visit's dQ partial has been read out of S^T's columns
-        if (ok && vis > 0) ok = warp_wait(dq_free, (vis - 1) & 1, kErrBwdDq, p.launch_id);
+        const int s1 = (vis + 1) % C::NST;
+        const bool more = v + 1 < w.nvisit;
+        const uint32_t q_addr = qdo_addr + s * 2 * C::TILE_BYTES;
+        const uint32_t q1_addr = qdo_addr + s1 * 2 * C::TILE_BYTES;
+        const uint32_t first = (v == 0) ? 0u : 1u;
+        ok = warp_wait(p_full, vis & 1, kErrBwdP, p.launch_id);
+        if (ok && more)
+          ok = warp_wait(&st_full[s1], ((vis + 1) / C::NST) & 1, kErrBwdStage, p.launch_id);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t q_addr = qdo_addr + s * 2 * C::TILE_BYTES;
-        const uint32_t do_addr = q_addr + C::TILE_BYTES;
         if (leader) {
-          // S^T = K Q^T and dP^T = V dO^T: both operands K-major (d innermost)
-          const uint32_t ka = ptx::sdesc_sw128_lo(k_addr, 16);
-          const uint32_t va = ptx::sdesc_sw128_lo(v_addr, 16);
-          const uint32_t qb_ = ptx::sdesc_sw128_lo(q_addr, 16);
-          const uint32_t gb = ptx::sdesc_sw128_lo(do_addr, 16);
-          ptx::mma_ss_lohi<0>(tmem + C::ST_COL, ka, kDescHi, qb_, kDescHi, kIdescS);
-#pragma unroll
-          for (int kk = 1; kk < D / 16; ++kk) {
-            const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
-            ptx::mma_ss_lohi<1>(tmem + C::ST_COL, ka + st, kDescHi, qb_ + st, kDescHi, kIdescS);
+          issue_g(C::DV_COL, C::ST_COL, q_addr + C::TILE_BYTES, first);  // dV += P^T dO
+          if (more) {
+            issue_t(C::ST_COL, k_addr, q1_addr);                         // S^T(v+1)
+            ptx::tc_commit(s_full);
           }
-          ptx::mma_ss_lohi<0>(tmem + C::DPT_COL, va, kDescHi, gb, kDescHi, kIdescS);
-#pragma unroll
-          for (int kk = 1; kk < D / 16; ++kk) {
-            const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
-            ptx::mma_ss_lohi<1>(tmem + C::DPT_COL, va + st, kDescHi, gb + st, kDescHi, kIdescS);
-          }
-          ptx::tc_commit(s_full);
         }
         __syncwarp();
-        if (!warp_wait(p_full, vis & 1, kErrBwdP, p.launch_id)) {
+        if (!warp_wait(ds_full, vis & 1, kErrBwdDq, p.launch_id)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         if (leader) {
-          const uint32_t first = (v == 0) ? 0u : 1u;
-          // dV += P^T dO and dK += dS^T Q: A from TMEM (K = queries, 8 columns
-          // per 16), B = dO / Q with queries as K and d as N (MN-major); K
-          // step kk is 16 query rows = 2 KB further into the tile.
-          const uint32_t gb = ptx::sdesc_sw128_lo(do_addr, C::SUB_BYTES);
-          const uint32_t qb_ = ptx::sdesc_sw128_lo(q_addr, C::SUB_BYTES);
-          ptx::mma_ts_lohi_rt(tmem + C::DV_COL, tmem + C::ST_COL, gb, kDescHi, kIdescG, first);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            ptx::mma_ts_lohi<1>(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, gb + kk * (2048 >> 4),
-                                kDescHi, kIdescG);
-          ptx::mma_ts_lohi_rt(tmem + C::DK_COL, tmem + C::DPT_COL, qb_, kDescHi, kIdescG, first);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            ptx::mma_ts_lohi<1>(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8,
-                                qb_ + kk * (2048 >> 4), kDescHi, kIdescG);
-          // dQp = dS K: A = dS (M = queries, K = keys) MN-major in shared
-          // memory, two 64-query sub-tiles 16 KB apart; B = K (K = keys,
-          // N = d) MN-major.  K step kk is 16 keys = 2 KB.
-          const uint32_t da = ptx::sdesc_sw128_lo(ds_addr, C::SUB_BYTES);
-          const uint32_t kb_ = ptx::sdesc_sw128_lo(k_addr, C::SUB_BYTES);
-          ptx::mma_ss_lohi<0>(tmem + C::ST_COL, da, kDescHi, kb_, kDescHi, kIdescQ);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            ptx::mma_ss_lohi<1>(tmem + C::ST_COL, da + kk * (2048 >> 4), kDescHi,
-                                kb_ + kk * (2048 >> 4), kDescHi, kIdescQ);
-          ptx::tc_commit(dq_full);
+          issue_g(C::DK_COL, C::DPT_COL, q_addr, first);                 // dK += dS^T Q
           ptx::tc_commit(&st_empty[s]);
-          if (v == w.nvisit - 1) {
+          if (more) {
+            issue_t(C::DPT_COL, v_addr, q1_addr + C::TILE_BYTES);        // dP^T(v+1)
+            ptx::tc_commit(dp_full);
+          } else {
             ptx::tc_commit(dkv_full);
             ptx::tc_commit(kv_empty);
           }
@@ -419,7 +381,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t st_addr = tmem + lane_base + C::ST_COL;
     const uint32_t dpt_addr = tmem + lane_base + C::DPT_COL;
-    const uint32_t ds_base = ptx::smem_u32(sDS);
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     int vis = 0;
@@ -451,51 +412,73 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           sD[row] = (qr < p.T) ? p.dvec[qrow0 + row] : 0.f;
         }
         ptx::bar_sync_named(1, 128);
-        // A warp whose wait gives up still reaches the read-out's barriers
-        // below (every warp takes the same barrier sequence in each visit).
-        ok = warp_wait(s_full, vis & 1, kErrBwdS, p.launch_id);
         const bool diag = p.causal && qb == w.kb;
-        if (ok) {
-          ptx::tc_fence_after();
+        // P^T: all 128 query columns of this key row, kept in fp32 for dS^T
+        ok = warp_wait(s_full, vis & 1, kErrBwdS, p.launch_id);
+        if (!ok) continue;
+        ptx::tc_fence_after();
+        uint32_t pr[4][32];
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {  // 32 query columns at a time
-            uint32_t sr[32], gr[32];
-            ptx::tmem_ld32(st_addr + 32 * c4, sr);
-            ptx::tmem_ld32(dpt_addr + 32 * c4, gr);
-            ptx::tmem_ld_wait();
-            ptx::reg_fence(sr);
-            ptx::reg_fence(gr);
-            uint32_t pp[16], dd[16];
+        for (int c4 = 0; c4 < 4; ++c4) ptx::tmem_ld32(st_addr + 32 * c4, pr[c4]);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) ptx::reg_fence(pr[c4]);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t pp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float pv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = 32 * c4 + 2 * i + e;
+              float pe = ptx::ex2(fmaf(__uint_as_float(pr[c4][2 * i + e]), sl2, -sLse[col]));
+              if (!key_ok || (diag && col < row)) pe = 0.f;  // key past T, or key > query
+              pv[e] = pe;
+              pr[c4][2 * i + e] = __float_as_uint(pe);
+            }
+            pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
+          }
+          ptx::tmem_st16(st_addr + 16 * c4, pp);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(p_full);
+        // dS^T = P^T (dP^T - D), two halves of 64 query columns
+        ok = warp_wait(dp_full, vis & 1, kErrBwdDq, p.launch_id);
+        if (!ok) continue;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t gr[2][32];
+          ptx::tmem_ld32(dpt_addr + 64 * h, gr[0]);
+          ptx::tmem_ld32(dpt_addr + 64 * h + 32, gr[1]);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(gr[0]);
+          ptx::reg_fence(gr[1]);
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c4 = 2 * h + c2;
+            uint32_t dd[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float pv[2], dv[2];
+              float dv[2];
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 const int col = 32 * c4 + 2 * i + e;
-                const float x = fmaf(__uint_as_float(sr[2 * i + e]), sl2, -sLse[col]);
-                float pe = ptx::ex2(x);
-                if (!key_ok || (diag && col < row)) pe = 0.f;  // key past T, or key > query
-                pv[e] = pe;
-                dv[e] = pe * (__uint_as_float(gr[2 * i + e]) - sD[col]);
+                dv[e] = __uint_as_float(pr[c4][2 * i + e]) *
+                        (__uint_as_float(gr[c2][2 * i + e]) - sD[col]);
               }
-              pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
               dd[i] = ptx::pack_bf16x2(dv[0], dv[1]);
             }
-            ptx::tmem_st16(st_addr + 16 * c4, pp);
             ptx::tmem_st16(dpt_addr + 16 * c4, dd);
-            // dS row `row`, queries 32*c4 .. 32*c4+31, into the swizzled tile
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              ptx::st_shared_v4(ds_base + ds_chunk_offset(row, 32 * c4 + 8 * j), dd[4 * j],
-                                dd[4 * j + 1], dd[4 * j + 2], dd[4 * j + 3]);
           }
-          ptx::tmem_st_wait();
-          ptx::fence_proxy_async_smem();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(p_full);
         }
-
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ds_full);
       }
       if (stop) break;
       // A warp whose wait gave up skips its work but walks on to the next
@@ -536,48 +519,410 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // fence) is what lets the MMA warp overwrite them.
       ptx::tc_fence_before();
     }
-  } else if (warp >= C::READ_WARP0) {
-    // ======================= dQ read-out ==================================
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;  // query row within the visit's block
-    const uint32_t src = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::ST_COL;
-    int vis = 0;
+  }
+
+  // ---- teardown -------------------------------------------------------------
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ kernel 3
+// Warp roles (384 threads):
+//   warps 0-7   compute: warp w owns query rows 32 (w % 4) .. + 31 (TMEM lane
+//               quadrant w % 4) and key columns 64 (w / 4) .. + 63 of each
+//               S / dP tile (and d columns D/2 (w / 4) .. of dQ)
+//   warp  8     MMA issue (lane 0) and TMEM allocation
+//   warp  9     TMA producer (lane 0)
+//   warps 10-11 idle
+// Tensor memory (512 columns):
+//   S    two buffers [0, 128) and [128, 256), alternating by key block; dS
+//        (bf16 pairs) written over each half's own columns: keys 0-63 at
+//        buffer + [0, 32), keys 64-127 at buffer + [64, 96)
+//   dP   [256, 384)
+//   dQ   [384, 384 + D)
+// Per key block j the MMA warp issues, in this order:
+//   (once the compute warps have read dP(j)) dP(j+1);
+//   (once dS(j) is written) dQ += dS(j) K_j, then S(j+2) into S(j)'s buffer.
+// S(j+1) is already in the other buffer, so the compute warps go from block
+// j to block j+1 without waiting for an MMA.
+template <int D>
+struct DqCfg {
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+  static constexpr int BM = 128;                  // query rows per unit
+  static constexpr int BN = 128;                  // keys per block
+  static constexpr int SUB = D / 64;
+  static constexpr int SUB_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NSTAGE = (D == 128) ? 5 : 10;  // K/V ring (K_j, V_j alternate)
+  static constexpr int Q_OFF = 0;
+  static constexpr int DO_OFF = TILE_BYTES;
+  static constexpr int KV_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
+  // q_full, q_empty, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], dp_full,
+  // dp_free, ds_full, dq_full, drain
+  static constexpr int NBAR = 2 + 2 * NSTAGE + 7;
+  static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int S_COL = 0;
+  static constexpr int DP_COL = 256;
+  static constexpr int DQ_COL = 384;
+  static constexpr int THREADS = 384;
+  static constexpr int MMA_WARP = 8;
+  static constexpr int TMA_WARP = 9;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(DQ_COL + D <= 512, "tensor memory budget");
+};
+
+// Unit u of kernel 3: step = u / (B * Hq) from the heaviest query block down
+// (causal); batch and query head from the rest.
+struct DqUnit {
+  int b, h, qb, n;  // n: key blocks visited
+};
+
+__device__ __forceinline__ DqUnit decode_dq_unit(const BwdParams& p, int u) {
+  DqUnit w;
+  const int bh = u % (p.B * p.Hq);
+  const int step = u / (p.B * p.Hq);
+  w.b = bh / p.Hq;
+  w.h = bh % p.Hq;
+  w.qb = p.nqb - 1 - step;
+  w.n = p.causal ? w.qb + 1 : p.nqb;
+  return w;
+}
+
+// P and dS of one row (this thread) over 64 key columns of a block; s holds
+// the raw scores on entry and P on return (fp32), ds the packed bf16 dS.
+// Masked keys (kv0 + c > lim) get P = 0 when kMasked.
+template <bool kMasked>
+__device__ __forceinline__ void dq_p_tile(uint32_t (&s)[2][32], float sl2, float lse_l2,
+                                          int kv0, int lim) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    float pe = ptx::ex2(fmaf(__uint_as_float(s[c >> 5][c & 31]), sl2, -lse_l2));
+    if (kMasked && kv0 + c > lim) pe = 0.f;
+    s[c >> 5][c & 31] = __float_as_uint(pe);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
+    attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v,
+                             const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using C = DqCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+
+  uint8_t* sQ = smem + C::Q_OFF;
+  uint8_t* sDO = smem + C::DO_OFF;
+  uint8_t* sKV = smem + C::KV_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = kv_full + C::NSTAGE;
+  uint64_t* s_full = kv_empty + C::NSTAGE;  // [2]
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* dp_free = s_full + 3;
+  uint64_t* ds_full = s_full + 4;
+  uint64_t* dq_full = s_full + 5;
+  uint64_t* drain = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SLOT_OFF);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    ptx::mbar_init(q_empty, 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    ptx::mbar_init(&s_full[0], 1);
+    ptx::mbar_init(&s_full[1], 1);
+    ptx::mbar_init(dp_full, 1);
+    ptx::mbar_init(dp_free, 8);   // one arrival per compute warp
+    ptx::mbar_init(ds_full, 8);
+    ptx::mbar_init(dq_full, 1);
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::TMA_WARP && lane == 0) {
+    ptx::prefetch_tensormap(&tm_q);
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+    ptx::prefetch_tensormap(&tm_do);
+  }
+  if (warp == C::MMA_WARP) {
+    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::TMA_WARP) {
+    // ======================= TMA producer =================================
+    // Per unit: K_0, V_0, then Q and dO (once the previous unit's last S and
+    // dP no longer read them), then K_1, V_1, K_2, V_2, ... into the ring.
+    const bool leader = lane == 0;
+    const uint64_t keep = ptx::policy_evict_last();
+    const uint64_t once = ptx::policy_evict_first();
+    int idx = 0;  // K/V tiles loaded so far (ring position)
+    int kq = 0;   // Q/dO loads issued so far (Q buffer phases)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = bwd_unit_of(p, k);
       if (u < 0) break;
-      const BwdUnit w = decode_bwd_unit(p, u);
-      for (int v = 0; v < w.nvisit; ++v, ++vis) {
-        if (!warp_wait(dq_full, vis & 1, kErrBwdDq, p.launch_id)) {
+      const DqUnit w = decode_dq_unit(p, u);
+      const int kv_plane = w.b * p.Hkv + w.h / p.G;
+      const int q_plane = w.b * p.Hq + w.h;
+      const int q_at = min(2, 2 * w.n);
+      for (int i = 0; i <= 2 * w.n; ++i) {
+        if (i == q_at) {
+          if (!warp_wait(q_empty, (kq & 1) ^ 1u, kErrBwdStage, p.launch_id)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            ptx::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+            for (int c = 0; c < C::SUB; ++c) {
+              ptx::tma_load_3d_hint(sQ + c * C::SUB_BYTES, &tm_q, q_full, c * 64, w.qb * C::BM,
+                                    q_plane, once);
+              ptx::tma_load_3d_hint(sDO + c * C::SUB_BYTES, &tm_do, q_full, c * 64, w.qb * C::BM,
+                                    q_plane, once);
+            }
+          }
+          __syncwarp();
+          ++kq;
+        }
+        if (i == 2 * w.n) break;
+        const int s = idx % C::NSTAGE;
+        if (!warp_wait(&kv_empty[s], ((idx / C::NSTAGE) & 1) ^ 1u, kErrBwdKv, p.launch_id)) {
+          ok = false;
+          break;
+        }
+        if (leader) {
+          ptx::mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+          const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+          for (int c = 0; c < C::SUB; ++c)
+            ptx::tma_load_3d_hint(sKV + s * C::TILE_BYTES + c * C::SUB_BYTES, map, &kv_full[s],
+                                  c * 64, (i >> 1) * C::BN, kv_plane, keep);
+        }
+        __syncwarp();
+        ++idx;
+      }
+    }
+    if (!ok) {
+      // Gave up: let the copies already in flight land before the CTA exits.
+      if (kq > 0) warp_wait(q_full, (kq - 1) & 1, kErrBwdStage, p.launch_id);
+      for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
+        warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrBwdKv, p.launch_id);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ======================= MMA issue ====================================
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);  // S, dP
+    constexpr uint32_t kIdescQ = ptx::idesc_bf16_f32(128, D, false, true);     // dQ (A TMEM)
+    constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);
+    const uint32_t q_addr = ptx::smem_u32(sQ);
+    const uint32_t do_addr = ptx::smem_u32(sDO);
+    const uint32_t kv_addr = ptx::smem_u32(sKV);
+    // X = Y Z^T into TMEM column col; Y (Q or dO) and Z (K or V) K-major.
+    auto issue_x = [&](uint32_t col, uint32_t y_addr, uint32_t z_addr) {
+      const uint32_t ya = ptx::sdesc_sw128_lo(y_addr, 16);
+      const uint32_t zb = ptx::sdesc_sw128_lo(z_addr, 16);
+      ptx::mma_ss_lohi<0>(tmem + col, ya, kDescHi, zb, kDescHi, kIdescS);
+#pragma unroll
+      for (int kk = 1; kk < D / 16; ++kk) {
+        const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
+        ptx::mma_ss_lohi<1>(tmem + col, ya + st, kDescHi, zb + st, kDescHi, kIdescS);
+      }
+    };
+    auto stage = [&](int i) { return kv_addr + (i % C::NSTAGE) * C::TILE_BYTES; };
+    auto kv_ready = [&](int i) {
+      return warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrBwdKv, p.launch_id);
+    };
+    int base = 0;  // ring position of the unit's K_0
+    int sc = 0;    // key blocks so far (S buffer = sc & 1; s_full phase = (sc >> 1) & 1)
+    int kq = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = bwd_unit_of(p, k);
+      if (u < 0) break;
+      const DqUnit w = decode_dq_unit(p, u);
+      if (!warp_wait(q_full, kq & 1, kErrBwdStage, p.launch_id)) break;
+      ++kq;
+      // prologue: S(0), dP(0), S(1)
+      ok = kv_ready(base) && kv_ready(base + 1) && (w.n < 2 || kv_ready(base + 2));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (leader) {
+        issue_x(C::S_COL + 128 * (sc & 1), q_addr, stage(base));
+        ptx::tc_commit(&s_full[sc & 1]);
+        issue_x(C::DP_COL, do_addr, stage(base + 1));
+        ptx::tc_commit(dp_full);
+        if (w.n >= 2) {
+          issue_x(C::S_COL + 128 * ((sc + 1) & 1), q_addr, stage(base + 2));
+          ptx::tc_commit(&s_full[(sc + 1) & 1]);
+        }
+        if (w.n == 1) ptx::tc_commit(q_empty);
+      }
+      __syncwarp();
+      for (int j = 0; j < w.n; ++j, ++sc) {
+        const int kidx = base + 2 * j, vidx = base + 2 * j + 1;
+        // dP(j+1) once every compute warp has read dP(j)
+        ok = warp_wait(dp_free, sc & 1, kErrBwdP, p.launch_id);
+        if (ok && j + 1 < w.n) ok = kv_ready(vidx + 2);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (leader) {
+          if (j + 1 < w.n) {
+            issue_x(C::DP_COL, do_addr, stage(vidx + 2));
+            ptx::tc_commit(dp_full);
+          }
+          ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);  // V_j: dP(j) was its last reader
+          // the unit's last S and dP are issued: Q and dO may be replaced
+          if (j == w.n - 2) ptx::tc_commit(q_empty);
+        }
+        __syncwarp();
+        // dQ += dS(j) K_j: A = dS from TMEM (keys 0-63 at buffer + 0, keys
+        // 64-127 at buffer + 64, 8 columns per 16 keys); B = K_j with keys as
+        // K and d as N (MN-major), K step kk = 16 keys = 2 KB.
+        ok = warp_wait(ds_full, sc & 1, kErrBwdDq, p.launch_id);
+        if (ok && j + 2 < w.n) ok = kv_ready(kidx + 4);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (leader) {
+          const uint32_t buf = C::S_COL + 128 * (sc & 1);
+          const uint32_t kb = ptx::sdesc_sw128_lo(stage(kidx), C::SUB_BYTES);
+          ptx::mma_ts_lohi_rt(tmem + C::DQ_COL, tmem + buf, kb, kDescHi, kIdescQ,
+                              j > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 1; kk < 8; ++kk)
+            ptx::mma_ts_lohi<1>(tmem + C::DQ_COL, tmem + buf + (kk >> 2) * 64 + (kk & 3) * 8,
+                                kb + kk * (2048 >> 4), kDescHi, kIdescQ);
+          ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);  // K_j: dQ(j) was its last reader
+          if (j == w.n - 1) ptx::tc_commit(dq_full);
+          if (j + 2 < w.n) {
+            issue_x(buf, q_addr, stage(kidx + 4));      // S(j+2) over S(j)'s buffer
+            ptx::tc_commit(&s_full[sc & 1]);
+          }
+        }
+        __syncwarp();
+      }
+      base += 2 * w.n;
+    }
+    if (leader) ptx::tc_commit(drain);
+    __syncwarp();
+    warp_wait(drain, 0, kErrBwdDrain, p.launch_id);
+  } else if (warp < 8) {
+    // ======================= compute warps ================================
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int r = quad * 32 + lane;  // query row within the block
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const float sl2 = p.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    int sc = 0;
+    int units = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = bwd_unit_of(p, k);
+      if (u < 0) break;
+      const DqUnit w = decode_dq_unit(p, u);
+      const int q_row = w.qb * C::BM + r;
+      const bool row_ok = q_row < p.T;
+      const long long grow = (static_cast<long long>(w.b) * p.Hq + w.h) * p.T + q_row;
+      const float lse_l2 = row_ok ? p.lse[grow] * kLog2e : INFINITY;
+      const float dval = row_ok ? p.dvec[grow] : 0.f;
+      const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
+      for (int j = 0; j < w.n; ++j, ++sc) {
+        const uint32_t buf = C::S_COL + 128 * (sc & 1);
+        if (!warp_wait(&s_full[sc & 1], (sc >> 1) & 1, kErrBwdS, p.launch_id)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        uint32_t r[D / 32][32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(src + 32 * c, r[c]);
+        uint32_t sv[2][32];
+        ptx::tmem_ld32(tmem + lane_base + buf + 64 * half, sv[0]);
+        ptx::tmem_ld32(tmem + lane_base + buf + 64 * half + 32, sv[1]);
         ptx::tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) ptx::reg_fence(r[c]);
-        // dQp is in registers: its TMEM columns are free for the next S^T
+        ptx::reg_fence(sv[0]);
+        ptx::reg_fence(sv[1]);
+        const int kv0 = j * C::BN + 64 * half;
+        const int row0 = w.qb * C::BM + quad * 32;  // this warp's first query row
+        const bool edge = p.causal ? (kv0 + 63 > row0) : (kv0 + 64 > p.T);
+        if (edge)
+          dq_p_tile<true>(sv, sl2, lse_l2, kv0, lim);
+        else
+          dq_p_tile<false>(sv, sl2, lse_l2, kv0, lim);
+        if (!warp_wait(dp_full, sc & 1, kErrBwdDq, p.launch_id)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        uint32_t gv[2][32];
+        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + 64 * half, gv[0]);
+        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + 64 * half + 32, gv[1]);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(gv[0]);
+        ptx::reg_fence(gv[1]);
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(dq_free);
-        int head, qb;
-        bwd_visit(p, w, v, head, qb);
-        if (qb * C::BM + row < p.T) {
-          float* dst =
-              p.dq_acc + ((static_cast<long long>(w.b) * p.Hq + head) * p.T + qb * C::BM + row) * D;
+        if (lane == 0) ptx::mbar_arrive(dp_free);
+        uint32_t ds[32];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c)
+        for (int i = 0; i < 32; ++i) {
+          const int c0 = 2 * i, c1 = 2 * i + 1;
+          ds[i] = ptx::pack_bf16x2(
+              __uint_as_float(sv[c0 >> 5][c0 & 31]) * (__uint_as_float(gv[c0 >> 5][c0 & 31]) - dval),
+              __uint_as_float(sv[c1 >> 5][c1 & 31]) * (__uint_as_float(gv[c1 >> 5][c1 & 31]) - dval));
+        }
+        ptx::tmem_st32(tmem + lane_base + buf + 64 * half, ds);
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ds_full);
+      }
+      if (!ok) break;
+
+      // ---- epilogue: dQ = scale * acc -> bf16 -------------------------------
+      if (!warp_wait(dq_full, units & 1, kErrBwdDkv, p.launch_id)) break;
+      ++units;
+      ptx::tc_fence_after();
+      constexpr int HC = D / 2;  // d columns per warp
+      uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * D + HC * half);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              ptx::red_add_v4_f32(dst + 32 * c + 4 * i, __uint_as_float(r[c][4 * i]),
-                                  __uint_as_float(r[c][4 * i + 1]),
-                                  __uint_as_float(r[c][4 * i + 2]),
-                                  __uint_as_float(r[c][4 * i + 3]));
+      for (int c = 0; c < HC / 32; ++c) {
+        uint32_t a[32];
+        ptx::tmem_ld32(tmem + lane_base + C::DQ_COL + HC * half + 32 * c, a);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(a);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = ptx::pack_bf16x2(__uint_as_float(a[2 * i]) * p.scale,
+                                   __uint_as_float(a[2 * i + 1]) * p.scale);
+        if (row_ok) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                         pk[4 * v4 + 3]);
         }
       }
+      // dQ has been read; the next unit's first dS arrival (after this fence)
+      // is what lets the MMA warp overwrite it.
+      ptx::tc_fence_before();
     }
   }
 

@@ -124,16 +124,18 @@ int tessera_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o
  * dq               bf16 [B, Hq, T, d] device, written
  * dk, dv           bf16 [B, Hkv, T, d] device, written
  * workspace        device memory of at least
- *                  tessera_attn_bwd_workspace_bytes(B, Hq, T, d) bytes, 16-byte
- *                  aligned, owned by the caller; overwritten (no contents need
- *                  to be set before the call)
+ *                  tessera_attn_bwd_workspace_bytes(B, Hq, T, d) bytes
+ *                  (B*Hq*T fp32: D), 16-byte aligned, owned by the caller;
+ *                  overwritten (no contents need to be set before the call)
  * other arguments  as in tessera_attn_fwd
  *
  * Checks as in tessera_attn_fwd, plus: every pointer non-NULL (lse too) and
  * 16-byte aligned, a large enough workspace, and no overlap between
  * dq/dk/dv/workspace and any input or each other.  Queues three kernels on
- * `stream` (tessera_attn_last_launch_count() = 3); bounded waits as in the
- * forward.
+ * `stream` (tessera_attn_last_launch_count() = 3): D, then dK/dV (key blocks
+ * as units), then dQ (query blocks as units, S and dP recomputed); no
+ * atomics, so the result does not depend on scheduling.  Bounded waits as in
+ * the forward.
  */
 size_t tessera_attn_bwd_workspace_bytes(int B, int Hq, int T, int d);
 int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
@@ -145,7 +147,7 @@ int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
  * tessera_attn_bwd without a caller-supplied workspace.  (The pages have no
  * counterpart: this is an interface of this library.)  The workspace is a
  * device array in the library itself, of
- * tessera_attn_bwd_noalloc_max_workspace_bytes() bytes (272 MiB) on every
+ * tessera_attn_bwd_noalloc_max_workspace_bytes() bytes (16 MiB) on every
  * device the library runs on; the call allocates nothing and calls no
  * allocating routine.  Nothing in the array needs to start at zero: each call
  * sets all it reads.  Arguments, checks and results are those of
