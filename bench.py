@@ -543,7 +543,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--only", choices=["decode", "prologue", "varlen"],
+    ap.add_argument("--only", choices=["backward", "decode", "prologue", "varlen"],
                     help="time one extra leg alone and print its object (for profiling it)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -616,7 +616,6 @@ def main():
     bwd_times, bwd_launches, bwd_ws = time_backward(w, q, k, v, g, bwd_steps, 3, flush, stream,
                                                     tess, torch)
     bwd_max_ms = max_over_ranks(sum(bwd_times), dev)
-    bwd_value = 2.5 * w.flops * bwd_steps * world / (bwd_max_ms * 1e-3) / 1e12
     err = tess.tessera_attn_device_error()
     if err != 0:
         raise SystemExit(f"device-side wait gave up in the backward (code {err})")
@@ -710,14 +709,8 @@ def main():
                 "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per key/value-head chunk "
                         "(H2D copy, kernel, D2H copy; copies overlap kernels) -> pinned host O/LSE"},
         "gpu_launches": launches,
-        "backward": {"metric": "causal GQA attn bwd TFLOP/s (bf16)", "value": round(bwd_value, 2),
-                     "unit": UNIT, "steps": bwd_steps,
-                     "ms_per_step": round(bwd_max_ms / bwd_steps, 5),
-                     "flops_per_step": 2.5 * w.flops,
-                     "flop_count": "5*B*Hq*T^2*d: five products over the causal triangle, "
-                                   "counted as the forward's 2*B*Hq*T^2*d counts two",
-                     "gpu_launches": bwd_launches, "workspace_bytes": bwd_ws,
-                     "l2": "flushed before every timed step"},
+        "backward": backward_line(w, bwd_times, bwd_max_ms, bwd_steps, bwd_launches, bwd_ws,
+                                  world, peaks, peak_src),
         "decode": decode_line(wd, dec_times, dec_max_ms, dec_steps, dec_launches, dec_ws, world,
                               peaks, peak_src),
         "varlen": varlen_line(inputs.VARLEN, vl_times, vl_launches, peaks, peak_src),
@@ -744,7 +737,16 @@ def one_leg(args, tess, torch, dev, world, rank, local):
     clocks.start()
     time.sleep(0.3)
     t0 = time.time()
-    if args.only == "decode":
+    w = inputs.WORKLOADS[args.workload]
+    if args.only == "backward":
+        q, k, v = (t.to(dev) for t in inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
+                                                     rank_seed(w.seed, rank), w.sigma_qk))
+        g = inputs.make_grad(w.B, w.Hq, w.T, w.d,
+                             rank_seed(w.seed, rank) + inputs.GRAD_SEED_OFFSET).to(dev)
+        times, launches, ws = time_backward(w, q, k, v, g, args.steps, args.warmup, flush,
+                                            stream, tess, torch)
+        max_ms = max_over_ranks(sum(times), dev)
+    elif args.only == "decode":
         wd = inputs.DECODE
         times, launches, ws = time_decode(wd, args.steps, args.warmup, flush, stream, tess, torch,
                                           dev)
@@ -767,7 +769,10 @@ def one_leg(args, tess, torch, dev, world, rank, local):
     if rank != 0:
         return 0
     peaks, peak_src = load_peaks()
-    if args.only == "decode":
+    if args.only == "backward":
+        line = backward_line(w, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
+        line["config"] = {"workload": args.workload}
+    elif args.only == "decode":
         line = decode_line(wd, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
     elif args.only == "varlen":
         line = varlen_line(inputs.VARLEN, times, launches, peaks, peak_src)
@@ -778,6 +783,28 @@ def one_leg(args, tess, torch, dev, world, rank, local):
                  "clocks": clocks.summary()})
     print(json.dumps(line), flush=True)
     return 0
+
+
+def backward_line(w, times, max_ms, steps, launches, ws_bytes, world, peaks, peak_src):
+    """The backward's object of the JSON line: tensor-bound, TFLOP/s of the
+    five products over the causal triangle against the measured bf16 peak.
+    The kernels issue seven (the dQ kernel recomputes S and dP)."""
+    flops = 2.5 * w.flops
+    value = flops * steps * world / (max_ms * 1e-3) / 1e12
+    achieved = flops / (statistics.mean(times) * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"metric": "causal GQA attn bwd TFLOP/s (bf16)", "value": round(value, 2),
+            "unit": UNIT, "steps": steps, "ms_per_step": round(max_ms / steps, 5),
+            "flops_per_step": flops,
+            "flop_count": "5*B*Hq*T^2*d: five products over the causal triangle, "
+                          "counted as the forward's 2*B*Hq*T^2*d counts two",
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "issued_flops_per_step": 3.5 * w.flops,
+                         "issued_frac": round(1.4 * achieved / peak, 4)},
+            "gpu_launches": launches, "workspace_bytes": ws_bytes,
+            "l2": "flushed before every timed step"}
 
 
 def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak_src):

@@ -295,7 +295,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
   const unsigned qgrid = static_cast<unsigned>(q_units < sms ? q_units : sms);
   tessera::attn_bwd_dq_sm100_kernel<D><<<qgrid, Q::THREADS, Q::SMEM_BYTES, stream>>>(
-      tm_q, tm_k, tm_v, tm_do, p);
+      tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout),
+      p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = 3;
   return TESSERA_OK;

@@ -534,21 +534,33 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 // Warp roles (384 threads):
 //   warps 0-7   compute: warp w owns query rows 32 (w % 4) .. + 31 (TMEM lane
 //               quadrant w % 4) and key columns 64 (w / 4) .. + 63 of each
-//               S / dP tile (and d columns D/2 (w / 4) .. of dQ)
-//   warp  8     MMA issue (lane 0) and TMEM allocation
-//   warp  9     TMA producer (lane 0)
-//   warps 10-11 idle
-// Tensor memory (512 columns):
-//   S    two buffers [0, 128) and [128, 256), alternating by key block; dS
-//        (bf16 pairs) written over each half's own columns: keys 0-63 at
-//        buffer + [0, 32), keys 64-127 at buffer + [64, 96)
-//   dP   [256, 384)
-//   dQ   [384, 384 + D)
-// Per key block j the MMA warp issues, in this order:
-//   (once the compute warps have read dP(j)) dP(j+1);
-//   (once dS(j) is written) dQ += dS(j) K_j, then S(j+2) into S(j)'s buffer.
-// S(j+1) is already in the other buffer, so the compute warps go from block
-// j to block j+1 without waiting for an MMA.
+//               S / dP tile (and d columns D/2 (w / 4) .. of Q, dO and dQ)
+//   warp  8     MMA issue of S and dP (lane 0) and TMEM allocation
+//   warp  9     TMA producer (lane 0): K and V tiles only
+//   warp 10     MMA issue of dQ (lane 0)
+//   warp 11     idle
+// Tensor memory (512 columns for D = 128):
+//   S    [0, 128)
+//   dP   [128, 256)
+//   dQ   [256, 256 + D)
+//   Q    [256 + D, 256 + 3D/2)   the unit's query rows, bf16 pairs (A operand)
+//   dO   [256 + 3D/2, 256 + 2D)
+// Shared memory: the K/V ring and one dS tile [128 rows][128 keys] bf16 in
+// the 128-byte-swizzled K-major layout (two 64-key sub-tiles), the A operand
+// of dQ += dS K.
+// Q and dO are the A operands of S = Q K^T and dP = dO V^T straight from
+// tensor memory, so those products read only K or V from shared memory.  No
+// product's input aliases another's output, so each is issued as soon as its
+// inputs are free: per key block j
+//   warp 8 issues S(j+1)  once the compute warps have loaded S(j),
+//          and dP(j+1)    once they have loaded dP(j);
+//   warp 10 issues dQ += dS(j) K_j  once dS(j) is in shared memory.
+// The two issuers need no ordering between them: S and dP write only their
+// own columns and read Q, dO, K, V; dQ reads dS and K and writes only dQ.
+// K_j, read by S(j) and dQ(j), is released by warp 10 after dQ(j): S(j) is
+// complete by then (the compute warps loaded its result before writing dS).
+// A single issuer spent most of each block waiting on barriers in a fixed
+// order; two let dQ(j) go out while warp 8 waits for the next S / dP slot.
 template <int D>
 struct DqCfg {
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
@@ -557,25 +569,27 @@ struct DqCfg {
   static constexpr int SUB = D / 64;
   static constexpr int SUB_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int NSTAGE = (D == 128) ? 5 : 10;  // K/V ring (K_j, V_j alternate)
-  static constexpr int Q_OFF = 0;
-  static constexpr int DO_OFF = TILE_BYTES;
-  static constexpr int KV_OFF = 2 * TILE_BYTES;
-  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
-  // q_full, q_empty, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], dp_full,
-  // dp_free, ds_full, dq_full, drain
-  static constexpr int NBAR = 2 + 2 * NSTAGE + 7;
+  static constexpr int NSTAGE = (D == 128) ? 6 : 12;  // K/V ring (K_j, V_j alternate)
+  static constexpr int KV_OFF = 0;
+  static constexpr int DS_OFF = KV_OFF + NSTAGE * TILE_BYTES;
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int BAR_OFF = DS_OFF + DS_BYTES;
+  // kv_full[NSTAGE], kv_empty[NSTAGE], q_ready, s_full, s_free, dp_full,
+  // dp_free, ds_full, ds_free, dq_full, drain (warp 8), drain (warp 10)
+  static constexpr int NBAR = 2 * NSTAGE + 10;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int S_COL = 0;
-  static constexpr int DP_COL = 256;
-  static constexpr int DQ_COL = 384;
+  static constexpr int DP_COL = 128;
+  static constexpr int DQ_COL = 256;
+  static constexpr int Q_COL = 256 + D;
+  static constexpr int DO_COL = 256 + D + D / 2;
   static constexpr int THREADS = 384;
   static constexpr int MMA_WARP = 8;
   static constexpr int TMA_WARP = 9;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(DQ_COL + D <= 512, "tensor memory budget");
+  static_assert(DO_COL + D / 2 <= 512, "tensor memory budget");
 };
 
 // Unit u of kernel 3: step = u / (B * Hq) from the heaviest query block down
@@ -595,9 +609,19 @@ __device__ __forceinline__ DqUnit decode_dq_unit(const BwdParams& p, int u) {
   return w;
 }
 
-// P and dS of one row (this thread) over 64 key columns of a block; s holds
-// the raw scores on entry and P on return (fp32), ds the packed bf16 dS.
-// Masked keys (kv0 + c > lim) get P = 0 when kMasked.
+// Byte offset of row r, columns c .. c + 7 (one 16-byte chunk) in a
+// [128 rows][128 columns] bf16 tile stored as two 64-column sub-tiles with the
+// 128-byte swizzle (8-row atoms of 1 KB; chunk j of row r at chunk j ^ (r % 8)).
+__device__ __forceinline__ uint32_t ds_chunk_offset(int r, int c) {
+  const int sub = c >> 6;
+  const int chunk = (c & 63) >> 3;
+  return static_cast<uint32_t>(sub * (128 * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                               ((chunk ^ (r & 7)) << 4));
+}
+
+// P of one row (this thread) over 64 key columns of a block: s holds the raw
+// scores on entry and P (fp32) on return.  Masked keys (kv0 + c > lim) get
+// P = 0 when kMasked.
 template <bool kMasked>
 __device__ __forceinline__ void dq_p_tile(uint32_t (&s)[2][32], float sl2, float lse_l2,
                                           int kv0, int lim) {
@@ -609,57 +633,71 @@ __device__ __forceinline__ void dq_p_tile(uint32_t (&s)[2][32], float sl2, float
   }
 }
 
+// D/2 bf16 of one row (16-byte aligned) as D/4 packed pairs, or zeros.
+template <int D>
+__device__ __forceinline__ void load_row_half(const __nv_bfloat16* src, bool ok,
+                                              uint32_t (&r)[D / 4]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) {
+    const uint4 v = ok ? __ldg(s4 + i) : make_uint4(0u, 0u, 0u, 0u);
+    r[4 * i] = v.x;
+    r[4 * i + 1] = v.y;
+    r[4 * i + 2] = v.z;
+    r[4 * i + 3] = v.w;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
-    attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
-                             const __grid_constant__ CUtensorMap tm_k,
+    attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v,
-                             const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+                             const __nv_bfloat16* __restrict__ q,
+                             const __nv_bfloat16* __restrict__ dout, const BwdParams p) {
   using C = DqCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
 
-  uint8_t* sQ = smem + C::Q_OFF;
-  uint8_t* sDO = smem + C::DO_OFF;
   uint8_t* sKV = smem + C::KV_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + C::NSTAGE;
-  uint64_t* s_full = kv_empty + C::NSTAGE;  // [2]
-  uint64_t* dp_full = s_full + 2;
-  uint64_t* dp_free = s_full + 3;
-  uint64_t* ds_full = s_full + 4;
-  uint64_t* dq_full = s_full + 5;
-  uint64_t* drain = s_full + 6;
+  uint64_t* q_ready = kv_empty + C::NSTAGE;
+  uint64_t* s_full = q_ready + 1;
+  uint64_t* s_free = q_ready + 2;
+  uint64_t* dp_full = q_ready + 3;
+  uint64_t* dp_free = q_ready + 4;
+  uint64_t* ds_full = q_ready + 5;
+  uint64_t* ds_free = q_ready + 6;
+  uint64_t* dq_full = q_ready + 7;
+  uint64_t* drain = q_ready + 8;
+  uint64_t* drain2 = q_ready + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SLOT_OFF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(q_full, 1);
-    ptx::mbar_init(q_empty, 1);
     for (int s = 0; s < C::NSTAGE; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
-    ptx::mbar_init(&s_full[0], 1);
-    ptx::mbar_init(&s_full[1], 1);
+    ptx::mbar_init(q_ready, 8);   // one arrival per compute warp
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(s_free, 8);
     ptx::mbar_init(dp_full, 1);
-    ptx::mbar_init(dp_free, 8);   // one arrival per compute warp
+    ptx::mbar_init(dp_free, 8);
     ptx::mbar_init(ds_full, 8);
+    ptx::mbar_init(ds_free, 1);
     ptx::mbar_init(dq_full, 1);
     ptx::mbar_init(drain, 1);
+    ptx::mbar_init(drain2, 1);
     ptx::fence_mbar_init();
   }
   if (warp == C::TMA_WARP && lane == 0) {
-    ptx::prefetch_tensormap(&tm_q);
     ptx::prefetch_tensormap(&tm_k);
     ptx::prefetch_tensormap(&tm_v);
-    ptx::prefetch_tensormap(&tm_do);
   }
   if (warp == C::MMA_WARP) {
     ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -672,40 +710,17 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
 
   if (warp == C::TMA_WARP) {
     // ======================= TMA producer =================================
-    // Per unit: K_0, V_0, then Q and dO (once the previous unit's last S and
-    // dP no longer read them), then K_1, V_1, K_2, V_2, ... into the ring.
+    // Per unit: K_0, V_0, K_1, V_1, ... into the ring.
     const bool leader = lane == 0;
     const uint64_t keep = ptx::policy_evict_last();
-    const uint64_t once = ptx::policy_evict_first();
     int idx = 0;  // K/V tiles loaded so far (ring position)
-    int kq = 0;   // Q/dO loads issued so far (Q buffer phases)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = bwd_unit_of(p, k);
       if (u < 0) break;
       const DqUnit w = decode_dq_unit(p, u);
       const int kv_plane = w.b * p.Hkv + w.h / p.G;
-      const int q_plane = w.b * p.Hq + w.h;
-      const int q_at = min(2, 2 * w.n);
-      for (int i = 0; i <= 2 * w.n; ++i) {
-        if (i == q_at) {
-          if (!warp_wait(q_empty, (kq & 1) ^ 1u, kErrBwdStage, p.launch_id)) {
-            ok = false;
-            break;
-          }
-          if (leader) {
-            ptx::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
-            for (int c = 0; c < C::SUB; ++c) {
-              ptx::tma_load_3d_hint(sQ + c * C::SUB_BYTES, &tm_q, q_full, c * 64, w.qb * C::BM,
-                                    q_plane, once);
-              ptx::tma_load_3d_hint(sDO + c * C::SUB_BYTES, &tm_do, q_full, c * 64, w.qb * C::BM,
-                                    q_plane, once);
-            }
-          }
-          __syncwarp();
-          ++kq;
-        }
-        if (i == 2 * w.n) break;
+      for (int i = 0; i < 2 * w.n; ++i, ++idx) {
         const int s = idx % C::NSTAGE;
         if (!warp_wait(&kv_empty[s], ((idx / C::NSTAGE) & 1) ^ 1u, kErrBwdKv, p.launch_id)) {
           ok = false;
@@ -719,33 +734,31 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
                                   c * 64, (i >> 1) * C::BN, kv_plane, keep);
         }
         __syncwarp();
-        ++idx;
       }
     }
     if (!ok) {
       // Gave up: let the copies already in flight land before the CTA exits.
-      if (kq > 0) warp_wait(q_full, (kq - 1) & 1, kErrBwdStage, p.launch_id);
       for (int i = max(0, idx - C::NSTAGE); i < idx; ++i)
         warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrBwdKv, p.launch_id);
     }
   } else if (warp == C::MMA_WARP) {
-    // ======================= MMA issue ====================================
+    // ======================= MMA issue: S and dP ==========================
     const bool leader = lane == 0;
     constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);  // S, dP
-    constexpr uint32_t kIdescQ = ptx::idesc_bf16_f32(128, D, false, true);     // dQ (A TMEM)
+    constexpr uint32_t kIdescQ = ptx::idesc_bf16_f32(128, D, false, true);     // dQ
     constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);
-    const uint32_t q_addr = ptx::smem_u32(sQ);
-    const uint32_t do_addr = ptx::smem_u32(sDO);
     const uint32_t kv_addr = ptx::smem_u32(sKV);
-    // X = Y Z^T into TMEM column col; Y (Q or dO) and Z (K or V) K-major.
-    auto issue_x = [&](uint32_t col, uint32_t y_addr, uint32_t z_addr) {
-      const uint32_t ya = ptx::sdesc_sw128_lo(y_addr, 16);
+    const uint32_t ds_addr = ptx::smem_u32(smem + C::DS_OFF);
+    // X = A Z^T into TMEM column col: A from TMEM column a_col (bf16 pairs, K =
+    // d, 8 columns per 16), Z (K or V) K-major in shared memory; K step kk is
+    // 32 B, or the next 16 KB sub-tile.
+    auto issue_x = [&](uint32_t col, uint32_t a_col, uint32_t z_addr) {
       const uint32_t zb = ptx::sdesc_sw128_lo(z_addr, 16);
-      ptx::mma_ss_lohi<0>(tmem + col, ya, kDescHi, zb, kDescHi, kIdescS);
+      ptx::mma_ts_lohi<0>(tmem + col, tmem + a_col, zb, kDescHi, kIdescS);
 #pragma unroll
       for (int kk = 1; kk < D / 16; ++kk) {
         const uint32_t st = (kk >> 2) * (C::SUB_BYTES >> 4) + (kk & 3) * 2;
-        ptx::mma_ss_lohi<1>(tmem + col, ya + st, kDescHi, zb + st, kDescHi, kIdescS);
+        ptx::mma_ts_lohi<1>(tmem + col, tmem + a_col + kk * 8, zb + st, kDescHi, kIdescS);
       }
     };
     auto stage = [&](int i) { return kv_addr + (i % C::NSTAGE) * C::TILE_BYTES; };
@@ -753,70 +766,49 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
       return warp_wait(&kv_full[i % C::NSTAGE], (i / C::NSTAGE) & 1, kErrBwdKv, p.launch_id);
     };
     int base = 0;  // ring position of the unit's K_0
-    int sc = 0;    // key blocks so far (S buffer = sc & 1; s_full phase = (sc >> 1) & 1)
-    int kq = 0;
+    int sc = 0;    // key blocks so far (barrier phases)
+    int units = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int u = bwd_unit_of(p, k);
       if (u < 0) break;
       const DqUnit w = decode_dq_unit(p, u);
-      if (!warp_wait(q_full, kq & 1, kErrBwdStage, p.launch_id)) break;
-      ++kq;
-      // prologue: S(0), dP(0), S(1)
-      ok = kv_ready(base) && kv_ready(base + 1) && (w.n < 2 || kv_ready(base + 2));
+      // Q and dO of the unit are in tensor memory; S(0), dP(0)
+      ok = warp_wait(q_ready, units & 1, kErrBwdStage, p.launch_id) && kv_ready(base) &&
+           kv_ready(base + 1);
+      ++units;
       if (!ok) break;
       ptx::tc_fence_after();
       if (leader) {
-        issue_x(C::S_COL + 128 * (sc & 1), q_addr, stage(base));
-        ptx::tc_commit(&s_full[sc & 1]);
-        issue_x(C::DP_COL, do_addr, stage(base + 1));
+        issue_x(C::S_COL, C::Q_COL, stage(base));
+        ptx::tc_commit(s_full);
+        issue_x(C::DP_COL, C::DO_COL, stage(base + 1));
         ptx::tc_commit(dp_full);
-        if (w.n >= 2) {
-          issue_x(C::S_COL + 128 * ((sc + 1) & 1), q_addr, stage(base + 2));
-          ptx::tc_commit(&s_full[(sc + 1) & 1]);
-        }
-        if (w.n == 1) ptx::tc_commit(q_empty);
+        ptx::tc_commit(&kv_empty[(base + 1) % C::NSTAGE]);  // V_0: dP(0) was its reader
       }
       __syncwarp();
       for (int j = 0; j < w.n; ++j, ++sc) {
-        const int kidx = base + 2 * j, vidx = base + 2 * j + 1;
-        // dP(j+1) once every compute warp has read dP(j)
-        ok = warp_wait(dp_free, sc & 1, kErrBwdP, p.launch_id);
-        if (ok && j + 1 < w.n) ok = kv_ready(vidx + 2);
+        const int kidx = base + 2 * j;
+        const bool more = j + 1 < w.n;
+        // S(j+1) once every compute warp has loaded S(j)
+        ok = warp_wait(s_free, sc & 1, kErrBwdP, p.launch_id);
+        if (ok && more) ok = kv_ready(kidx + 2);
         if (!ok) break;
         ptx::tc_fence_after();
-        if (leader) {
-          if (j + 1 < w.n) {
-            issue_x(C::DP_COL, do_addr, stage(vidx + 2));
-            ptx::tc_commit(dp_full);
-          }
-          ptx::tc_commit(&kv_empty[vidx % C::NSTAGE]);  // V_j: dP(j) was its last reader
-          // the unit's last S and dP are issued: Q and dO may be replaced
-          if (j == w.n - 2) ptx::tc_commit(q_empty);
+        if (leader && more) {
+          issue_x(C::S_COL, C::Q_COL, stage(kidx + 2));
+          ptx::tc_commit(s_full);
         }
         __syncwarp();
-        // dQ += dS(j) K_j: A = dS from TMEM (keys 0-63 at buffer + 0, keys
-        // 64-127 at buffer + 64, 8 columns per 16 keys); B = K_j with keys as
-        // K and d as N (MN-major), K step kk = 16 keys = 2 KB.
-        ok = warp_wait(ds_full, sc & 1, kErrBwdDq, p.launch_id);
-        if (ok && j + 2 < w.n) ok = kv_ready(kidx + 4);
+        // dP(j+1) once every compute warp has loaded dP(j)
+        ok = warp_wait(dp_free, sc & 1, kErrBwdP, p.launch_id);
+        if (ok && more) ok = kv_ready(kidx + 3);
         if (!ok) break;
         ptx::tc_fence_after();
-        if (leader) {
-          const uint32_t buf = C::S_COL + 128 * (sc & 1);
-          const uint32_t kb = ptx::sdesc_sw128_lo(stage(kidx), C::SUB_BYTES);
-          ptx::mma_ts_lohi_rt(tmem + C::DQ_COL, tmem + buf, kb, kDescHi, kIdescQ,
-                              j > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            ptx::mma_ts_lohi<1>(tmem + C::DQ_COL, tmem + buf + (kk >> 2) * 64 + (kk & 3) * 8,
-                                kb + kk * (2048 >> 4), kDescHi, kIdescQ);
-          ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);  // K_j: dQ(j) was its last reader
-          if (j == w.n - 1) ptx::tc_commit(dq_full);
-          if (j + 2 < w.n) {
-            issue_x(buf, q_addr, stage(kidx + 4));      // S(j+2) over S(j)'s buffer
-            ptx::tc_commit(&s_full[sc & 1]);
-          }
+        if (leader && more) {
+          issue_x(C::DP_COL, C::DO_COL, stage(kidx + 3));
+          ptx::tc_commit(dp_full);
+          ptx::tc_commit(&kv_empty[(kidx + 3) % C::NSTAGE]);  // V_{j+1}: dP(j+1) its reader
         }
         __syncwarp();
       }
@@ -825,6 +817,43 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     if (leader) ptx::tc_commit(drain);
     __syncwarp();
     warp_wait(drain, 0, kErrBwdDrain, p.launch_id);
+  } else if (warp == 10) {
+    // ======================= dQ MMA issue =================================
+    const bool leader = lane == 0;
+    constexpr uint32_t kIdescQ = ptx::idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t kDescHi = ptx::sdesc_sw128_hi(1024);
+    const uint32_t kv_addr = ptx::smem_u32(sKV);
+    const uint32_t ds_addr = ptx::smem_u32(smem + C::DS_OFF);
+    int base = 0, sc = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = bwd_unit_of(p, k);
+      if (u < 0) break;
+      const DqUnit w = decode_dq_unit(p, u);
+      for (int j = 0; j < w.n; ++j, ++sc) {
+        const int kidx = base + 2 * j;
+        ok = warp_wait(ds_full, sc & 1, kErrBwdDq, p.launch_id);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (leader) {
+          const uint32_t da = ptx::sdesc_sw128_lo(ds_addr, 16);
+          const uint32_t kb = ptx::sdesc_sw128_lo(kv_addr + (kidx % C::NSTAGE) * C::TILE_BYTES, C::SUB_BYTES);
+          ptx::mma_ss_lohi_rt(tmem + C::DQ_COL, da, kDescHi, kb, kDescHi, kIdescQ, j > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 1; kk < 8; ++kk)
+            ptx::mma_ss_lohi<1>(tmem + C::DQ_COL, da + (kk >> 2) * (16384 >> 4) + (kk & 3) * 2,
+                                kDescHi, kb + kk * (2048 >> 4), kDescHi, kIdescQ);
+          ptx::tc_commit(ds_free);
+          ptx::tc_commit(&kv_empty[kidx % C::NSTAGE]);
+          if (j == w.n - 1) ptx::tc_commit(dq_full);
+        }
+        __syncwarp();
+      }
+      base += 2 * w.n;
+    }
+    if (leader) ptx::tc_commit(drain2);
+    __syncwarp();
+    warp_wait(drain2, 0, kErrBwdDrain, p.launch_id);
   } else if (warp < 8) {
     // ======================= compute warps ================================
     const int quad = warp & 3;
@@ -833,6 +862,8 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int HC = D / 2;  // d columns of Q, dO, dQ per warp
+    const uint32_t ds_base = ptx::smem_u32(smem + C::DS_OFF);
     int sc = 0;
     int units = 0;
     bool ok = true;
@@ -846,19 +877,39 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
       const float lse_l2 = row_ok ? p.lse[grow] * kLog2e : INFINITY;
       const float dval = row_ok ? p.dvec[grow] : 0.f;
       const int lim = p.causal ? min(q_row, p.T - 1) : p.T - 1;  // last visible key
+      // This row's halves of Q and dO into tensor memory (zeros past T).  The
+      // previous unit's S and dP have completed: their results were loaded.
+      {
+        uint32_t qa[D / 4], ga[D / 4];
+        load_row_half<D>(q + grow * D + HC * half, row_ok, qa);
+        load_row_half<D>(dout + grow * D + HC * half, row_ok, ga);
+        if constexpr (D == 128) {
+          ptx::tmem_st32(tmem + lane_base + C::Q_COL + 32 * half, qa);
+          ptx::tmem_st32(tmem + lane_base + C::DO_COL + 32 * half, ga);
+        } else {
+          ptx::tmem_st16(tmem + lane_base + C::Q_COL + 16 * half, qa);
+          ptx::tmem_st16(tmem + lane_base + C::DO_COL + 16 * half, ga);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(q_ready);
+      }
       for (int j = 0; j < w.n; ++j, ++sc) {
-        const uint32_t buf = C::S_COL + 128 * (sc & 1);
-        if (!warp_wait(&s_full[sc & 1], (sc >> 1) & 1, kErrBwdS, p.launch_id)) {
+        if (!warp_wait(s_full, sc & 1, kErrBwdS, p.launch_id)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         uint32_t sv[2][32];
-        ptx::tmem_ld32(tmem + lane_base + buf + 64 * half, sv[0]);
-        ptx::tmem_ld32(tmem + lane_base + buf + 64 * half + 32, sv[1]);
+        ptx::tmem_ld32(tmem + lane_base + C::S_COL + 64 * half, sv[0]);
+        ptx::tmem_ld32(tmem + lane_base + C::S_COL + 64 * half + 32, sv[1]);
         ptx::tmem_ld_wait();
         ptx::reg_fence(sv[0]);
         ptx::reg_fence(sv[1]);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(s_free);
         const int kv0 = j * C::BN + 64 * half;
         const int row0 = w.qb * C::BM + quad * 32;  // this warp's first query row
         const bool edge = p.causal ? (kv0 + 63 > row0) : (kv0 + 64 > p.T);
@@ -872,8 +923,9 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         }
         ptx::tc_fence_after();
         uint32_t gv[2][32];
-        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + 64 * half, gv[0]);
-        ptx::tmem_ld32(tmem + lane_base + C::DP_COL + 64 * half + 32, gv[1]);
+        const uint32_t dp_addr = tmem + lane_base + C::DP_COL + 64 * half;
+        ptx::tmem_ld32(dp_addr, gv[0]);
+        ptx::tmem_ld32(dp_addr + 32, gv[1]);
         ptx::tmem_ld_wait();
         ptx::reg_fence(gv[0]);
         ptx::reg_fence(gv[1]);
@@ -888,9 +940,17 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
               __uint_as_float(sv[c0 >> 5][c0 & 31]) * (__uint_as_float(gv[c0 >> 5][c0 & 31]) - dval),
               __uint_as_float(sv[c1 >> 5][c1 & 31]) * (__uint_as_float(gv[c1 >> 5][c1 & 31]) - dval));
         }
-        ptx::tmem_st32(tmem + lane_base + buf + 64 * half, ds);
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
+        // dS row r, keys 64 half .. + 63, into the swizzled tile once dQ(j-1)
+        // has read the previous one
+        if (!warp_wait(ds_free, (sc & 1) ^ 1u, kErrBwdDq, p.launch_id)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          ptx::st_shared_v4(ds_base + ds_chunk_offset(r, 64 * half + 8 * c), ds[4 * c],
+                            ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
+        ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(ds_full);
       }
@@ -900,7 +960,6 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
       if (!warp_wait(dq_full, units & 1, kErrBwdDkv, p.launch_id)) break;
       ++units;
       ptx::tc_fence_after();
-      constexpr int HC = D / 2;  // d columns per warp
       uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * D + HC * half);
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) {
