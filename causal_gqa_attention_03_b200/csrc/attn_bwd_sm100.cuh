@@ -71,14 +71,18 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 }
 
 // ------------------------------------------------------------------ kernel 2
-// Warp roles (256 threads):
-//   warps 0-3   compute: P^T, dS^T (thread r owns key row r), then dK, dV
-//   warp  4     MMA issue (lane 0) and TMEM allocation
-//   warp  5     TMA producer (lane 0)
-//   warps 6-7   idle
+// Warp roles (384 threads):
+//   warps 0-7   compute: warp w owns key rows 32 (w % 4) .. + 31 (TMEM lane
+//               quadrant w % 4) and query columns 64 (w / 4) .. + 63 of each
+//               visit: P^T, dS^T, then its D/2 columns of dK, dV.  Two warps
+//               per lane quadrant overlap one's MUFU work with the other's.
+//   warp  8     MMA issue (lane 0) and TMEM allocation
+//   warp  9     TMA producer (lane 0)
+//   warps 10-11 idle
 // Tensor memory (512 columns):
-//   S^T  [0, 128)      P^T (bf16 pairs) written over its first 64 columns
-//   dP^T [128, 256)    dS^T (bf16 pairs) written over its first 64 columns
+//   S^T  [0, 128)      P^T (bf16 pairs) written over each half's own
+//                      columns: queries 0-63 at +[0, 32), 64-127 at +[64, 96)
+//   dP^T [128, 256)    dS^T (bf16 pairs) in the same split layout
 //   dV   [256, 256 + D),  dK  [256 + D, 256 + 2 D)
 // Per visit v the MMA warp issues, in this order:
 //   (once P^T(v) is written)  dV += P^T(v) dO(v), then S^T(v+1);
@@ -110,9 +114,9 @@ struct BwdCfg {
   static constexpr int DPT_COL = 128;
   static constexpr int DV_COL = 256;
   static constexpr int DK_COL = 256 + D;
-  static constexpr int THREADS = 256;
-  static constexpr int MMA_WARP = 4;
-  static constexpr int TMA_WARP = 5;
+  static constexpr int THREADS = 384;
+  static constexpr int MMA_WARP = 8;
+  static constexpr int TMA_WARP = 9;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DK_COL + D <= 512, "tensor memory budget");
 };
@@ -207,8 +211,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(dp_full, 1);
-    ptx::mbar_init(p_full, 4);    // one arrival per compute warp
-    ptx::mbar_init(ds_full, 4);
+    ptx::mbar_init(p_full, 8);    // one arrival per compute warp
+    ptx::mbar_init(ds_full, 8);
     ptx::mbar_init(dkv_full, 1);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
@@ -303,15 +307,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       }
     };
     // G += A^T Z into TMEM column col: A from TMEM column a_col (bf16 pairs,
-    // K = queries, 8 columns per 16), Z (dO or Q) with queries as K and d as
-    // N (MN-major); K step kk is 16 query rows = 2 KB further into the tile.
+    // K = queries, 8 columns per 16; queries 64-127 at +64), Z (dO or Q) with
+    // queries as K and d as N (MN-major); K step kk is 16 query rows = 2 KB
+    // further into the tile.
     auto issue_g = [&](uint32_t col, uint32_t a_col, uint32_t z_addr, uint32_t first) {
       const uint32_t zb = ptx::sdesc_sw128_lo(z_addr, C::SUB_BYTES);
       ptx::mma_ts_lohi_rt(tmem + col, tmem + a_col, zb, kDescHi, kIdescG, first);
 #pragma unroll
       for (int kk = 1; kk < 8; ++kk)
-        ptx::mma_ts_lohi<1>(tmem + col, tmem + a_col + kk * 8, zb + kk * (2048 >> 4), kDescHi,
-                            kIdescG);
+        ptx::mma_ts_lohi<1>(tmem + col, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
+                            zb + kk * (2048 >> 4), kDescHi, kIdescG);
     };
     int vis = 0;    // visits issued so far (stage ring position; barrier phases)
     bool ok = true;
@@ -375,29 +380,32 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (leader) ptx::tc_commit(drain);
     __syncwarp();
     warp_wait(drain, 0, kErrBwdDrain, p.launch_id);
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ======================= compute warps ================================
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t st_addr = tmem + lane_base + C::ST_COL;
-    const uint32_t dpt_addr = tmem + lane_base + C::DPT_COL;
+    // warp w: key rows 32 (w % 4) .. + 31, query columns 64 (w / 4) .. + 63
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t st_addr = tmem + lane_base + C::ST_COL + 64 * half;
+    const uint32_t dpt_addr = tmem + lane_base + C::DPT_COL + 64 * half;
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     int vis = 0;
     int units = 0;
     bool ok = true;
-    bool stop = false;  // every compute warp has learnt that one gave up
+    bool stop = false;
     for (int k = 0; !stop; ++k) {
       const int u = bwd_unit_of(p, k);
       if (u < 0) break;
       const BwdUnit w = decode_bwd_unit(p, u);
-      const int key = w.kb * C::BN + row;  // this thread's key row (P^T, dS^T, dK, dV)
+      const int key = w.kb * C::BN + row;
       const bool key_ok = key < p.T;
       for (int v = 0; v < w.nvisit; ++v, ++vis) {
-        // The four compute warps meet at two named barriers per visit; a warp
-        // whose wait gave up keeps taking part until the first one, where all
-        // four learn of it and stop together.
-        if (!ptx::bar_red_and(1, 128, ok)) {
+        // The eight compute warps meet at two named barriers per visit; a
+        // warp whose wait gave up keeps taking part until the first one,
+        // where all eight learn of it and stop together.
+        if (!ptx::bar_red_and(1, 256, ok)) {
           stop = true;
           break;
         }
@@ -408,73 +416,64 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // (+inf / 0 past T, so those columns of P^T and dS^T are zero).
         {
           const int qr = qb * C::BM + row;
-          sLse[row] = (qr < p.T) ? p.lse[qrow0 + row] * kLog2e : INFINITY;
-          sD[row] = (qr < p.T) ? p.dvec[qrow0 + row] : 0.f;
+          if (half == 0)
+            sLse[row] = (qr < p.T) ? p.lse[qrow0 + row] * kLog2e : INFINITY;
+          else
+            sD[row] = (qr < p.T) ? p.dvec[qrow0 + row] : 0.f;
         }
-        ptx::bar_sync_named(1, 128);
+        ptx::bar_sync_named(1, 256);
         const bool diag = p.causal && qb == w.kb;
-        // P^T: all 128 query columns of this key row, kept in fp32 for dS^T
         ok = warp_wait(s_full, vis & 1, kErrBwdS, p.launch_id);
         if (!ok) continue;
         ptx::tc_fence_after();
-        uint32_t pr[4][32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) ptx::tmem_ld32(st_addr + 32 * c4, pr[c4]);
+        uint32_t pr[2][32];
+        ptx::tmem_ld32(st_addr, pr[0]);
+        ptx::tmem_ld32(st_addr + 32, pr[1]);
         ptx::tmem_ld_wait();
+        ptx::reg_fence(pr[0]);
+        ptx::reg_fence(pr[1]);
+        uint32_t pp[32];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) ptx::reg_fence(pr[c4]);
+        for (int i = 0; i < 32; ++i) {
+          float pv[2];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t pp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float pv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = 32 * c4 + 2 * i + e;
-              float pe = ptx::ex2(fmaf(__uint_as_float(pr[c4][2 * i + e]), sl2, -sLse[col]));
-              if (!key_ok || (diag && col < row)) pe = 0.f;  // key past T, or key > query
-              pv[e] = pe;
-              pr[c4][2 * i + e] = __float_as_uint(pe);
-            }
-            pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
+            const int col = 64 * half + c;
+            float pe = ptx::ex2(fmaf(__uint_as_float(pr[c >> 5][c & 31]), sl2, -sLse[col]));
+            if (!key_ok || (diag && col < row)) pe = 0.f;
+            pv[e] = pe;
+            pr[c >> 5][c & 31] = __float_as_uint(pe);
           }
-          ptx::tmem_st16(st_addr + 16 * c4, pp);
+          pp[i] = ptx::pack_bf16x2(pv[0], pv[1]);
         }
+        ptx::tmem_st32(st_addr, pp);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(p_full);
-        // dS^T = P^T (dP^T - D), two halves of 64 query columns
         ok = warp_wait(dp_full, vis & 1, kErrBwdDq, p.launch_id);
         if (!ok) continue;
         ptx::tc_fence_after();
+        uint32_t gr[2][32];
+        ptx::tmem_ld32(dpt_addr, gr[0]);
+        ptx::tmem_ld32(dpt_addr + 32, gr[1]);
+        ptx::tmem_ld_wait();
+        ptx::reg_fence(gr[0]);
+        ptx::reg_fence(gr[1]);
+        uint32_t dd[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t gr[2][32];
-          ptx::tmem_ld32(dpt_addr + 64 * h, gr[0]);
-          ptx::tmem_ld32(dpt_addr + 64 * h + 32, gr[1]);
-          ptx::tmem_ld_wait();
-          ptx::reg_fence(gr[0]);
-          ptx::reg_fence(gr[1]);
+        for (int i = 0; i < 32; ++i) {
+          float dv[2];
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const int c4 = 2 * h + c2;
-            uint32_t dd[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float dv[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int col = 32 * c4 + 2 * i + e;
-                dv[e] = __uint_as_float(pr[c4][2 * i + e]) *
-                        (__uint_as_float(gr[c2][2 * i + e]) - sD[col]);
-              }
-              dd[i] = ptx::pack_bf16x2(dv[0], dv[1]);
-            }
-            ptx::tmem_st16(dpt_addr + 16 * c4, dd);
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
+            dv[e] = __uint_as_float(pr[c >> 5][c & 31]) *
+                    (__uint_as_float(gr[c >> 5][c & 31]) - sD[64 * half + c]);
           }
+          dd[i] = ptx::pack_bf16x2(dv[0], dv[1]);
         }
+        ptx::tmem_st32(dpt_addr, dd);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
@@ -485,19 +484,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // unit's first barrier, where the others learn of it.
       if (!ok) continue;
 
-      // ---- unit epilogue: dV, scale * dK -> bf16 ------------------------------
+      // ---- unit epilogue: dV, scale * dK -> bf16 (this warp's D/2 columns) ----
       ok = warp_wait(dkv_full, units & 1, kErrBwdDkv, p.launch_id);
       ++units;
       if (!ok) continue;
       ptx::tc_fence_after();
+      constexpr int HC = D / 2;
       const long long krow = (static_cast<long long>(w.b) * p.Hkv + w.g) * p.T + key;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t src = tmem + lane_base + (which == 0 ? C::DV_COL : C::DK_COL);
+        const uint32_t src = tmem + lane_base + (which == 0 ? C::DV_COL : C::DK_COL) + HC * half;
         const float mul = which == 0 ? 1.f : p.scale;
-        uint4* out = reinterpret_cast<uint4*>((which == 0 ? p.dv : p.dk) + krow * D);
+        uint4* out = reinterpret_cast<uint4*>((which == 0 ? p.dv : p.dk) + krow * D + HC * half);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < HC / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(src + 32 * c, r);
           ptx::tmem_ld_wait();
@@ -515,8 +515,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
         }
       }
-      // dK, dV have been read; the next unit's first P^T arrival (after this
-      // fence) is what lets the MMA warp overwrite them.
       ptx::tc_fence_before();
     }
   }
