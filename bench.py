@@ -683,6 +683,9 @@ def main():
                 "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
                 "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
                 "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes}
+    if "bf16_tflops_sustained" in peaks:
+        # long runs settle at the power cap: the sustained GEMM figure beside it
+        roofline["frac_of_sustained"] = round(achieved / float(peaks["bf16_tflops_sustained"]), 4)
 
     cpu = None
     leg_cpu = {}
