@@ -314,10 +314,28 @@ def time_kernel(w, q, k, v, steps, warmup, flush, stream, tess, torch):
     return times, launches, o, lse
 
 
+def time_back_to_back(w, q, k, v, n, stream, tess, torch):
+    """Mean time of n forward launches queued back to back (no L2 flush
+    between them: the warm-L2 figure, and for tiny workloads the launch
+    rate), one CUDA-event pair around all of them."""
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=q.device)
+    for _ in range(3):
+        tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
 def time_backward(w, q, k, v, g, steps, warmup, flush, stream, tess, torch):
-    """The backward (3 launches: D prep, dK/dV + dQ partials, dQ conversion) on
-    the forward's O and LSE, each step after an L2 flush, CUDA events around
-    the three launches."""
+    """The backward (3 launches: D prep, dK/dV, dQ) on the forward's O and
+    LSE, each step after an L2 flush, CUDA events around the three
+    launches."""
     o, lse = tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, stream=stream)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     nbytes = tess.tessera_attn_bwd_workspace_bytes(w.B, w.Hq, w.T, w.d)
@@ -649,6 +667,13 @@ def main():
                 ms = statistics.median(ts)
                 sweep[name] = {"tflops": round(ws.flops / (ms * 1e-3) / 1e12, 1),
                                "ms": round(ms, 4)}
+            # warm L2 (no flush between launches); 1000 launches for the
+            # launch-bound smallest workloads
+            nb = 1000 if ws.flops < 1e9 else max(5, min(200, int(0.3 / max(ws.flops / 1.2e15, 1e-6))))
+            warm = time_back_to_back(ws, qs, ks, vs, nb, stream, tess, torch)
+            sweep[name]["warm_ms"] = round(warm, 4)
+            sweep[name]["warm_tflops"] = round(ws.flops / (warm * 1e-3) / 1e12, 1)
+            sweep[name]["warm_launches"] = nb
             gs = inputs.workload_grad(ws).to(dev)
             n = max(5, min(100, int(0.3 / max(2.5 * ws.flops / 5e14, 1e-6))))
             tb, _, _ = time_backward(ws, qs, ks, vs, gs, n, 3, flush, stream, tess, torch)
