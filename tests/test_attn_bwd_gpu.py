@@ -158,8 +158,9 @@ def test_bwd_guard_regions_untouched():
         assert torch.all(b[:pad] == 7.0) and torch.all(b[-pad:] == 7.0)
 
 
-def test_bwd_repeated_calls_bitwise():
-    B, Hq, Hkv, T, d = 1, 8, 2, 513, 128
+@pytest.mark.parametrize("B,Hq,Hkv,T,d", [(1, 8, 2, 513, 128), (2, 4, 4, 300, 64),
+                                           (1, 32, 1, 1000, 128)])
+def test_bwd_repeated_calls_bitwise(B, Hq, Hkv, T, d):
     dev = torch.device("cuda:0")
     q, k, v = (t.to(dev) for t in inputs.make_qkv(B, Hq, Hkv, T, d, seed=51))
     g = inputs.make_grad(B, Hq, T, d, seed=52).to(dev)
@@ -167,7 +168,7 @@ def test_bwd_repeated_calls_bitwise():
     a = [t.clone() for t in tess.attn_bwd(q, k, v, o, lse, g)]
     b = tess.attn_bwd(q, k, v, o, lse, g)
     torch.cuda.synchronize()
-    # dK, dV are summed in a fixed order; dQ sums partials with atomics, so
-    # its low bits may differ between calls
-    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
-    assert torch.allclose(a[0].float(), b[0].float(), rtol=1e-2, atol=1e-3)
+    # every gradient is summed in a fixed order (no atomics): the same bits on
+    # every call, whatever the CTAs' timing
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
