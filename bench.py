@@ -734,8 +734,9 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per key/value-head chunk "
-                        "(H2D copy, kernel, D2H copy; copies overlap kernels) -> pinned host O/LSE"},
+                "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per chunk of query heads "
+                        "(16 by default: H2D copy, kernel, D2H copy; copies overlap kernels) "
+                        "-> pinned host O/LSE"},
         "gpu_launches": launches,
         "backward": backward_line(w, bwd_times, bwd_max_ms, bwd_steps, bwd_launches, bwd_ws,
                                   world, peaks, peak_src),

@@ -609,14 +609,30 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
   if ((lse_h == nullptr) != (lse_d == nullptr) || chunks < 0) return TESSERA_ERR_INVALID_ARG;
   if (empty) return TESSERA_OK;
   if (!q_h || !k_h || !v_h || !o_h) return TESSERA_ERR_INVALID_ARG;
-  // Chunks are contiguous ranges of the B*Hkv (batch, key/value head) slices;
-  // each is one launch over a [1, n*G, T, d] view of the buffers.
+  // Chunks are contiguous ranges of the B*Hkv (batch, key/value head) slices,
+  // each one launch over a [1, n*G, T, d] view of the buffers; or, when more
+  // chunks than slices are asked for, each slice is cut into `split` runs of
+  // G/split query heads (split divides G), one launch each over a
+  // [1, G/split, T, d] view with that slice's K/V, uploaded with its first
+  // run.  Smaller pieces shorten the pipeline's fill (the first upload) and
+  // drain (the last kernel and download).
   const int slices = static_cast<int>(static_cast<long long>(B) * Hkv);
-  const int n_chunks = chunks == 0 ? (slices < 8 ? slices : 8) : (chunks < slices ? chunks : slices);
   const int G = Hq / Hkv;
+  const int target = chunks == 0 ? 16 : chunks;
+  int split = 1;
+  if (target > slices) {
+    const int want = (target + slices - 1) / slices;
+    split = G;
+    for (int s_ = want; s_ < G; ++s_)
+      if (G % s_ == 0) {
+        split = s_;
+        break;
+      }
+  }
+  const int n_chunks = split > 1 ? slices * split : (target < slices ? target : slices);
   const size_t kv_slice = static_cast<size_t>(T) * d * 2;   // bytes of one K (or V) head
-  const size_t q_slice = kv_slice * G;                      // bytes of one group of Q (or O) heads
-  const size_t lse_slice = static_cast<size_t>(T) * G * 4;  // bytes of one group of LSE rows
+  const size_t q_head = kv_slice;                           // bytes of one Q (or O) head
+  const size_t lse_head = static_cast<size_t>(T) * 4;       // bytes of one head's LSE rows
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_pipe_mu);
@@ -633,31 +649,48 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
   const auto m8 = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
   int launches = 0;
   for (int c = 0; c < n_chunks; ++c) {
-    const int s0 = static_cast<int>(static_cast<long long>(slices) * c / n_chunks);
-    const int s1 = static_cast<int>(static_cast<long long>(slices) * (c + 1) / n_chunks);
+    // this chunk: slices [s0, s1) (whole groups) or query heads [h0, h1) of slice s0
+    int s0, s1, h0, h1;
+    if (split > 1) {
+      s0 = c / split;
+      s1 = s0 + 1;
+      h0 = (c % split) * (G / split);
+      h1 = h0 + G / split;
+    } else {
+      s0 = static_cast<int>(static_cast<long long>(slices) * c / n_chunks);
+      s1 = static_cast<int>(static_cast<long long>(slices) * (c + 1) / n_chunks);
+      h0 = 0;
+      h1 = G;
+    }
     const int n = s1 - s0;
     if (n == 0) continue;
-    const size_t qo = q_slice * s0, ko = kv_slice * s0, lo = lse_slice * s0;
-    if (cudaMemcpyAsync(m8(q_d, qo), c8(q_h, qo), q_slice * n, cudaMemcpyHostToDevice, hp->in) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(m8(k_d, ko), c8(k_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(m8(v_d, ko), c8(v_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+    const bool whole = (h0 == 0 && h1 == G);
+    const int nq = whole ? n * G : h1 - h0;  // query heads of the launch
+    const size_t qo = q_head * (static_cast<size_t>(s0) * G + h0);
+    const size_t lo = lse_head * (static_cast<size_t>(s0) * G + h0);
+    const size_t ko = kv_slice * s0;
+    if (h0 == 0 &&
+        (cudaMemcpyAsync(m8(k_d, ko), c8(k_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+             cudaSuccess ||
+         cudaMemcpyAsync(m8(v_d, ko), c8(v_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
+             cudaSuccess))
+      return TESSERA_ERR_CUDA;
+    if (cudaMemcpyAsync(m8(q_d, qo), c8(q_h, qo), q_head * nq, cudaMemcpyHostToDevice, hp->in) !=
             cudaSuccess ||
         cudaEventRecord(hp->in_done, hp->in) != cudaSuccess ||
         cudaStreamWaitEvent(s, hp->in_done, 0) != cudaSuccess)
       return TESSERA_ERR_CUDA;
     const int lst = launch_d(d, m8(q_d, qo), m8(k_d, ko), m8(v_d, ko), m8(o_d, qo),
-                             lse_d ? reinterpret_cast<float*>(m8(lse_d, lo)) : nullptr, 1, n * G, n,
+                             lse_d ? reinterpret_cast<float*>(m8(lse_d, lo)) : nullptr, 1, nq, n,
                              T, causal, scale, s);
     if (lst != TESSERA_OK) return lst;
     ++launches;
     if (cudaEventRecord(hp->k_done, s) != cudaSuccess ||
         cudaStreamWaitEvent(hp->out, hp->k_done, 0) != cudaSuccess ||
-        cudaMemcpyAsync(m8(o_h, qo), c8(o_d, qo), q_slice * n, cudaMemcpyDeviceToHost, hp->out) !=
+        cudaMemcpyAsync(m8(o_h, qo), c8(o_d, qo), q_head * nq, cudaMemcpyDeviceToHost, hp->out) !=
             cudaSuccess)
       return TESSERA_ERR_CUDA;
-    if (lse_h && cudaMemcpyAsync(m8(lse_h, lo), c8(lse_d, lo), lse_slice * n,
+    if (lse_h && cudaMemcpyAsync(m8(lse_h, lo), c8(lse_d, lo), lse_head * nq,
                                  cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
       return TESSERA_ERR_CUDA;
   }

@@ -167,7 +167,10 @@ int tessera_attn_bwd_noalloc(const void *q, const void *k, const void *v, const 
  * The same operation on host buffers, pipelined over the host link.  (The
  * pages describe the kernel only; this transfer pipeline is this library's.)
  * The B*Hkv (batch, key/value head) slices are cut into `chunks` contiguous
- * ranges; for each range Q/K/V are copied host -> device, the kernel of
+ * ranges, or, when `chunks` exceeds B*Hkv, each slice is cut into `split`
+ * runs of G/split query heads (split = the smallest divisor of G that is at
+ * least ceil(chunks / (B*Hkv)), else G; the slice's K/V go with its first
+ * run).  For each piece Q (and K/V) are copied host -> device, the kernel of
  * tessera_attn_fwd runs on it, and O/LSE are copied device -> host.  Copies
  * run on two streams the library creates per device on first use (kept for
  * the life of the process), so one range's copies overlap the others' kernels
@@ -179,7 +182,9 @@ int tessera_attn_bwd_noalloc(const void *q, const void *k, const void *v, const 
  * o_h, lse_h     host outputs; lse_h may be NULL (then lse_d must be NULL).
  * q_d .. lse_d   device buffers of the full sizes, owned by the caller, with
  *                the rules of tessera_attn_fwd; they also hold the results.
- * chunks         0: the library's choice (min(B*Hkv, 8)); else clamped to B*Hkv.
+ * chunks         0: the library's choice (16, as above); 1..B*Hkv: that many
+ *                ranges of whole slices; more: slices cut by query heads.
+ *                Every choice gives the same bits as one tessera_attn_fwd.
  * stream         the host outputs are complete once the work queued on
  *                `stream` before the call returns has finished plus this
  *                call's work: synchronise `stream` before reading them.
