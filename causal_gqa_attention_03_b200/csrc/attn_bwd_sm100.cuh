@@ -35,12 +35,13 @@ namespace tessera {
 
 enum BwdWaitCode : uint32_t {
   kErrBwdKv = 11,      // K/V tiles (kernel 2: of a unit; kernel 3: ring stages)
-  kErrBwdStage = 12,   // Q/dO tiles full or empty
-  kErrBwdS = 13,       // S (S^T) complete
-  kErrBwdP = 14,       // P^T written (kernel 2); dP read (kernel 3)
-  kErrBwdDq = 15,      // dS written; dP complete
+  kErrBwdStage = 12,   // Q/dO stages full or empty (kernel 2); Q/dO in TMEM (kernel 3)
+  kErrBwdS = 13,       // S^T (kernel 2) or S (kernel 3) complete
+  kErrBwdP = 14,       // P^T written (kernel 2); S or dP loaded by the compute warps (kernel 3)
+  kErrBwdDq = 15,      // dS^T written, dP^T complete (kernel 2); dS written or its tile
+                       // free, dP complete (kernel 3)
   kErrBwdDkv = 16,     // dK, dV (kernel 2) or dQ (kernel 3) complete
-  kErrBwdDrain = 17,
+  kErrBwdDrain = 17,   // the MMAs issued, before tensor memory is freed
 };
 
 // ------------------------------------------------------------------ kernel 1
