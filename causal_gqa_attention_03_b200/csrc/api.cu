@@ -254,6 +254,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const int sms = sm_count(dev);
   if (sms <= 0) return TESSERA_ERR_CUDA;
   const long long rows = static_cast<long long>(B) * Hq * T;
+  const int nqb = (T + C::BM - 1) / C::BM;
+  const long long kv_units = static_cast<long long>(B) * Hkv * nqb;  // kernel 2
+  const long long q_units = static_cast<long long>(B) * Hq * nqb;    // kernel 3
+  if (q_units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;  // before any launch
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
   if (!make_map(&tm_q, q, B * Hq, T, D) || !make_map(&tm_k, k, B * Hkv, T, D) ||
       !make_map(&tm_v, v, B * Hkv, T, D) || !make_map(&tm_do, dout, B * Hq, T, D))
@@ -274,16 +278,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.nqb = (T + C::BM - 1) / C::BM;
+  p.nqb = nqb;
   p.lse = lse;
   p.dvec = dvec;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   // 2. dK, dV: units (batch, key/value head, key block)
-  const long long kv_units = static_cast<long long>(B) * Hkv * p.nqb;
-  const long long q_units = static_cast<long long>(B) * Hq * p.nqb;
-  if (q_units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
   p.num_units = static_cast<int>(kv_units);
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
   const unsigned grid = static_cast<unsigned>(kv_units < sms ? kv_units : sms);
