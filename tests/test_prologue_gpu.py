@@ -72,6 +72,25 @@ def test_rmsnorm_in_place_and_large_rows_sampled():
     check_norm(y[sel].cpu(), ref, "sampled rows")
 
 
+@pytest.mark.parametrize("dim", [4096, 8192])
+def test_rmsnorm_wide_rows_guard_regions_and_odd_counts(dim):
+    # wide rows go through shared memory by bulk copy: fewer rows than the
+    # grid's warps, an odd count, and untouched memory on both sides of y
+    pad = 64
+    for rows in (1, 5, 4097):
+        x = _bf16((rows, dim), 300 + rows, 1.5)
+        w = _bf16((dim,), 301)
+        buf = torch.full((rows * dim + 2 * pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+        out = buf[pad:pad + rows * dim].view(rows, dim)
+        tess.rmsnorm(x.to(DEV), w.to(DEV), 1e-6, out=out)
+        torch.cuda.synchronize()
+        assert tess.tessera_attn_device_error() == 0
+        assert torch.all(buf[:pad] == 7.0) and torch.all(buf[-pad:] == 7.0)
+        sel = np.unique(np.r_[0, rows - 1, np.arange(0, rows, max(1, rows // 7))])
+        ref = oracle.rmsnorm_f64(x[sel].double().numpy(), w.double().numpy(), 1e-6)
+        check_norm(out[sel].cpu(), ref, (rows, dim))
+
+
 def test_rmsnorm_zero_row_and_guard_regions():
     dim = 512
     x = torch.zeros((3, dim), dtype=torch.bfloat16)
