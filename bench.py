@@ -471,7 +471,7 @@ def prologue_line(w, res, peaks, peak_src):
         line[name] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 5),
                       "bytes_per_step": nbytes, "gpu_launches": launches,
                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
-                                   "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                   "unit": "GB/s", "frac": round(gbs / hbm, 4), "traffic": None,
                                    "peak_source": f"{peak_src} hbm_gbs"}}
     return line
 
@@ -527,15 +527,15 @@ def varlen_line(wv, times, launches, peaks, peak_src):
             "flop_count": "sum over sequences of the metric's 2*Hq*T_b^2*d",
             "config": wv.describe(), "gpu_launches": launches,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak,
-                         "unit": UNIT, "frac": round(tf / peak, 4),
+                         "unit": UNIT, "frac": round(tf / peak, 4), "traffic": None,
                          "peak_source": f"{peak_src} bf16_tflops (burst)"},
             "l2": "flushed before every timed step"}
 
 
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
-    tessera_attn_fwd_host (copies pipelined with the kernels over key/value-head
-    chunks).  Each step returns with the outputs on the host."""
+    tessera_attn_fwd_host (copies pipelined with the kernels over chunks of
+    query heads).  Each step returns with the outputs on the host."""
     staging = {"q": torch.empty(q_h.shape, dtype=torch.bfloat16, device=dev),
                "k": torch.empty(k_h.shape, dtype=torch.bfloat16, device=dev),
                "v": torch.empty(k_h.shape, dtype=torch.bfloat16, device=dev),
