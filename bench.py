@@ -17,6 +17,8 @@ on the host cores instead, on a bounded sample of rows of the same workload.
 from __future__ import annotations
 
 import argparse
+import contextlib
+import dataclasses
 import datetime
 import itertools
 import json
@@ -178,6 +180,61 @@ def oracle_rows_rate(w, q, k, v, seconds: float, seed: int, max_rows: int | None
     return flops / el / 1e12, rows_done, flops, el
 
 
+def oracle_allcore_rate(w, q, k, v, seconds: float, seed: int, threads: int | None = None,
+                        run_rows: int = 128):
+    """Time the fp64 oracle on every host core for about `seconds` of wall time.
+
+    The workload's rows are cut into runs of `run_rows` consecutive rows of one
+    (b, h) (oracle.fwd_runs); runs are taken in a seeded random order and
+    handed to `threads` host threads (default: every core this process may
+    use), each run one call of the oracle's row entry.  Submission stops once
+    `seconds` have passed; the runs in flight then finish.  Returns (TFLOP/s,
+    runs done, total runs, flops done, elapsed, threads); flops are the
+    metric's 4*d per visible key per row (oracle.run_flops).
+    """
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor, FIRST_COMPLETED, wait
+    import oracle
+    qb, kb, vb = inputs.bf16_bits(q), inputs.bf16_bits(k), inputs.bf16_bits(v)
+    threads = threads or oracle.host_threads()
+    runs = oracle.fwd_runs(w.B, w.Hq, w.T, w.causal, run_rows)
+    order = np.random.default_rng(seed).permutation(len(runs))
+
+    def one(run):
+        b, h, i0, i1 = run
+        rows = np.empty((i1 - i0, 3), dtype=np.int64)
+        rows[:, 0], rows[:, 1], rows[:, 2] = b, h, np.arange(i0, i1)
+        oracle.attn_rows_bf16(qb, kb, vb, rows, causal=w.causal, scale=w.scale)
+        return oracle.run_flops(run, w.d, w.T, w.causal)
+
+    flops, done, nxt = 0.0, 0, 0
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        pending = set()
+        while nxt < len(order) and len(pending) < threads:
+            pending.add(pool.submit(one, runs[order[nxt]]))
+            nxt += 1
+        while pending:
+            fin, pending = wait(pending, return_when=FIRST_COMPLETED)
+            for f in fin:
+                flops += f.result()
+                done += 1
+            if time.perf_counter() - t0 < seconds:
+                while nxt < len(order) and len(pending) < threads:
+                    pending.add(pool.submit(one, runs[order[nxt]]))
+                    nxt += 1
+    el = time.perf_counter() - t0
+    return flops / el / 1e12, done, len(runs), flops, el, threads
+
+
+def config_of(w, world: int) -> dict:
+    """The `config` object of the JSON line, the same in both arms."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "causal": w.causal, "sigma_qk": w.sigma_qk, "seed": w.seed,
+            "l2": "flushed before every timed step (256 MB write, outside the events)",
+            "parallelism": f"dp{world} (independent batch per GPU)"}
+
+
 # Host copies of small parts of the extra legs' inputs, kept for the oracle's
 # timing (filled by the time_* functions).
 SAMPLES = {}
@@ -217,16 +274,17 @@ def leg_cpu_baselines(w, q_h, k_h, v_h, seconds: float):
     out["backward"] = {"value": fl[0] / el / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
                        "sample": f"{8 * n} random dQ rows of {w.name} in {el:.1f}s "
                                  "(6*d*(i+1) flops per row), fp64, single thread"}
-    if "decode" in SAMPLES:
-        qd, sk, sv, st_, sn = SAMPLES["decode"]
+    for key, wd in (("decode", inputs.DECODE), ("decode_d64", inputs.DECODE_D64)):
+        if key not in SAMPLES:
+            continue
+        qd, sk, sv, st_, sn = SAMPLES[key]
         qn, skn, svn = qd.double().numpy(), sk.double().numpy(), sv.double().numpy()
-        wd = inputs.DECODE
         nbytes = float(int(sn.sum()) * wd.Hkv * wd.d * 4 + 2 * len(sn) * wd.Hq * wd.d * 2)
         n, el = timed(lambda: oracle.paged_decode_f64(qn, skn, svn, st_, sn, scale=wd.scale))
-        out["decode"] = {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": 1,
-                         "kind": "oracle",
-                         "sample": f"{len(sn)} sequences ({int(sn.sum())} tokens) of {wd.name}, "
-                                   f"{n} steps in {el:.1f}s, fp64, single thread"}
+        out[key] = {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": 1,
+                    "kind": "oracle",
+                    "sample": f"{len(sn)} sequences ({int(sn.sum())} tokens) of {wd.name}, "
+                              f"{n} steps in {el:.1f}s, fp64, single thread"}
     if "varlen" in SAMPLES:
         qv, kv, vv = (inputs.bf16_bits(t) for t in SAMPLES["varlen"])
         T = qv.shape[2]
@@ -265,28 +323,31 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     q, k, v = inputs.workload_inputs(w)
-    step_seconds = 0.5
+    step_seconds = 2.0
     for i in range(args.warmup):
-        oracle_rows_rate(w, q, k, v, step_seconds, seed=100 + i)
+        oracle_allcore_rate(w, q, k, v, step_seconds / 4, seed=100 + i)
     flops = 0.0
     el = 0.0
-    rows = 0
+    runs = 0
+    threads = 1
     for i in range(args.steps):
-        _, r, f, e = oracle_rows_rate(w, q, k, v, step_seconds, seed=1000 + i)
+        _, r, total_runs, f, e, threads = oracle_allcore_rate(w, q, k, v, step_seconds,
+                                                              seed=1000 + i)
         flops += f
         el += e
-        rows += r
+        runs += r
     value = flops / el / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, **{k_: getattr(w, k_) for k_ in
-                                          ("B", "T", "Hq", "Hkv", "d", "causal")}},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} random (b,h,i) rows of {w.name}, "
-                                   f"{args.steps} steps of ~{step_seconds}s, single thread"},
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "nproc": os.cpu_count(),
+                         "sample": f"{runs} random 128-row runs of {w.name} (of {total_runs}), "
+                                   f"{args.steps} steps of ~{step_seconds}s on {threads} host "
+                                   "threads, fp64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -294,6 +355,16 @@ def run_reference(args, w):
 
 
 # --------------------------------------------------------------------- GPU arm
+def nvtx(name: str):
+    """An nvtx range around one timed launch (a profiler's timeline shows
+    which leg and step it belongs to); a no-op where torch lacks nvtx."""
+    import torch
+    try:
+        return torch.cuda.nvtx.range(name)
+    except (AttributeError, RuntimeError):
+        return contextlib.nullcontext()
+
+
 def time_kernel(w, q, k, v, steps, warmup, flush, stream, tess, torch):
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=q.device)
@@ -307,7 +378,9 @@ def time_kernel(w, q, k, v, steps, warmup, flush, stream, tess, torch):
     for i in range(steps):
         flush.zero_()
         starts[i].record(stream)
-        tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        with nvtx(f"attn_fwd {w.name} step {i}"):
+            tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                          stream=stream)
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
@@ -356,14 +429,15 @@ def time_backward(w, q, k, v, g, steps, warmup, flush, stream, tess, torch):
     for i in range(steps):
         flush.zero_()
         starts[i].record(stream)
-        call()
+        with nvtx(f"{call.__qualname__.split('.')[0]} step {i}"):
+            call()
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes
 
 
-def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
+def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev, sample_key="decode"):
     """One decode step over the paged cache of ``wd`` (2 launches: the split-KV
     partial kernel and the merge), CUDA events around both launches.  The
     step reads far more than L2 holds (2.43 GB for the serving batch), so
@@ -390,7 +464,8 @@ def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
     torch.cuda.synchronize()
     for i in range(steps):
         starts[i].record(stream)
-        call()
+        with nvtx(f"{call.__qualname__.split('.')[0]} step {i}"):
+            call()
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
@@ -407,7 +482,7 @@ def time_decode(wd, steps, warmup, flush, stream, tess, torch, dev):
     tab_h, lens_h = table.cpu().numpy(), lens.cpu().numpy()
     pick = [int(lens_h.argmax()), int(len(lens_h) // 2)]
     sk, sv, st_, sn = inputs.gather_sequences(tab_h, lens_h, pick, wd.bs, kc, vc)
-    SAMPLES["decode"] = (q[pick].cpu(), sk, sv, st_, sn)
+    SAMPLES[sample_key] = (q[pick].cpu(), sk, sv, st_, sn)
     del q, kc, vc, table, lens, o, lse, ws
     return ([s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches, nbytes,
             [s_.elapsed_time(e) for s_, e in zip(fs, fe)])
@@ -505,7 +580,8 @@ def time_varlen(wv, steps, warmup, flush, stream, tess, torch, dev):
     for i in range(steps):
         flush.zero_()
         starts[i].record(stream)
-        call()
+        with nvtx(f"{call.__qualname__.split('.')[0]} step {i}"):
+            call()
         launches += tess.tessera_attn_last_launch_count()
         ends[i].record(stream)
     torch.cuda.synchronize()
@@ -515,6 +591,25 @@ def time_varlen(wv, steps, warmup, flush, stream, tess, torch, dev):
                               for t in (q, k, v))
     del q, k, v, o, lse
     return [s_.elapsed_time(e) for s_, e in zip(starts, ends)], launches
+
+
+def noncausal_line(wn, times, max_ms, steps, launches, world, peaks, peak_src):
+    """The full-attention (causal = 0) forward on the headline workload's
+    inputs: TFLOP/s of 4*B*Hq*T^2*d against the measured bf16 peak."""
+    value = wn.flops * steps * world / (max_ms * 1e-3) / 1e12
+    achieved = wn.flops / (statistics.mean(times) * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"metric": "GQA attn fwd TFLOP/s (bf16), full attention (no causal mask)",
+            "value": round(value, 2), "unit": UNIT, "steps": steps,
+            "ms_per_step": round(max_ms / steps, 5), "flops_per_step": wn.flops,
+            "flop_count": "4*B*Hq*T^2*d: QK^T and PV over every key",
+            "config": {"workload": wn.name, "B": wn.B, "T": wn.T, "Hq": wn.Hq, "Hkv": wn.Hkv,
+                       "d": wn.d, "causal": False},
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         **north_star_roofline(achieved, wn)},
+            "gpu_launches": launches, "l2": "flushed before every timed step"}
 
 
 def varlen_line(wv, times, launches, peaks, peak_src):
@@ -554,8 +649,9 @@ def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(steps):
-        step()
+    for i in range(steps):
+        with nvtx(f"attn_fwd_host {w.name} step {i}"):
+            step()
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
@@ -663,6 +759,22 @@ def main():
     if err != 0:
         raise SystemExit(f"device-side error in the decode step (code {err})")
 
+    # the same serving batch at head dimension 64 (CUDA-core decode kernel)
+    wd64 = inputs.DECODE_D64
+    d64_times, d64_launches, d64_ws, d64_flushed = time_decode(
+        wd64, dec_steps, 3, flush, stream, tess, torch, dev, sample_key="decode_d64")
+    d64_max_ms = max_over_ranks(sum(d64_times), dev)
+    err = tess.tessera_attn_device_error()
+    if err != 0:
+        raise SystemExit(f"device-side error in the d=64 decode step (code {err})")
+
+    # the headline workload without the causal mask (full attention)
+    wn = dataclasses.replace(w, causal=False, name=w.name + "_noncausal")
+    nc_steps = max(5, min(args.steps, 50))
+    nc_times, nc_launches, _, _ = time_kernel(wn, q, k, v, nc_steps, 3, flush, stream, tess,
+                                              torch)
+    nc_max_ms = max_over_ranks(sum(nc_times), dev)
+
     # the packed variable-length forward on its mixed-length batch
     vl_times, vl_launches = time_varlen(inputs.VARLEN, max(5, min(args.steps, 50)), 3, flush,
                                         stream, tess, torch, dev)
@@ -721,8 +833,8 @@ def main():
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                 "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
-                "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
-                "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes}
+                "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes,
+                **north_star_roofline(achieved, w)}
     if "bf16_tflops_sustained" in peaks:
         # long runs settle at the power cap: the sustained GEMM figure beside it
         roofline["frac_of_sustained"] = round(achieved / float(peaks["bf16_tflops_sustained"]), 4)
@@ -730,10 +842,16 @@ def main():
     cpu = None
     leg_cpu = {}
     if not args.no_cpu_baseline and world == 1:
-        rate, rows, _, el = oracle_rows_rate(w, q_h, k_h, v_h, args.cpu_seconds, seed=1)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{rows} random (b,h,i) rows of {w.name} in {el:.1f}s, "
-                         "fp64, single thread"}
+        rate, runs, total_runs, fl, el, threads = oracle_allcore_rate(
+            w, q_h, k_h, v_h, args.cpu_seconds, seed=1)
+        rate1, rows1, _, el1 = oracle_rows_rate(w, q_h, k_h, v_h, 3.0, seed=1)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "nproc": os.cpu_count(),
+               "sample": f"{runs} random 128-row runs of {w.name} ({100.0 * fl / w.flops:.1f}% "
+                         f"of its flops, {runs} of {total_runs} runs) in {el:.1f}s on "
+                         f"{threads} host threads, fp64",
+               "single_thread": {"value": rate1, "unit": UNIT, "cores": 1,
+                                 "sample": f"{rows1} random (b,h,i) rows in {el1:.1f}s"}}
         leg_cpu = leg_cpu_baselines(w, q_h, k_h, v_h, seconds=3.0)
 
     line = {
@@ -741,10 +859,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "causal": w.causal, "sigma_qk": w.sigma_qk, "seed": w.seed,
-                   "l2": "flushed before every timed step (256 MB write, outside the events)",
-                   "parallelism": f"dp{world} (independent batch per GPU)"},
+        "config": config_of(w, world),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -757,6 +872,10 @@ def main():
                                   world, peaks, peak_src),
         "decode": decode_line(wd, dec_times, dec_max_ms, dec_steps, dec_launches, dec_ws, world,
                               peaks, peak_src, dec_flushed),
+        "decode_d64": decode_line(wd64, d64_times, d64_max_ms, dec_steps, d64_launches, d64_ws,
+                                  world, peaks, peak_src, d64_flushed),
+        "noncausal": noncausal_line(wn, nc_times, nc_max_ms, nc_steps, nc_launches, world,
+                                    peaks, peak_src),
         "varlen": varlen_line(inputs.VARLEN, vl_times, vl_launches, peaks, peak_src),
         "prologue": prologue_line(w, pro, peaks, peak_src),
         "clocks": clk,
@@ -878,6 +997,17 @@ def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak
             "ms_per_step_write_flush": (round(statistics.median(flushed), 5) if flushed else None),
             "write_flush_note": "a 256 MB write before each step, outside the events: its dirty "
                                 "lines are written back during the step"}
+
+
+def north_star_roofline(achieved: float, w) -> dict:
+    """The target's own roofline for a forward launch: the lesser of the
+    nominal dense bf16 rate (2.25 PFLOP/s) and the I/O bytes (Q, K, V, O, LSE)
+    over a nominal 8 TB/s, with the target of 60 % of it for the largest
+    causal workload."""
+    roof = min(NOMINAL_BF16_TFLOPS, w.flops / w.io_bytes * NOMINAL_HBM_GBS * 1e9 / 1e12)
+    frac = achieved / roof
+    return {"north_star_peak": round(roof, 1), "frac_north_star": round(frac, 4),
+            "north_star_target_frac": 0.60, "north_star_target_met": bool(frac >= 0.60)}
 
 
 # The files the forward kernel is built from: its traffic record stays valid

@@ -203,14 +203,31 @@ struct HostPipe {
 std::mutex g_pipe_mu;
 HostPipe g_pipes[64];
 
+// Destroys whatever a partial set-up created and clears the handles, so a
+// later call starts from nothing instead of leaking the earlier objects.
+void host_pipe_reset(HostPipe& h) {
+  for (cudaEvent_t* e : {&h.start, &h.in_done, &h.k_done, &h.out_done}) {
+    if (*e != nullptr) cudaEventDestroy(*e);
+    *e = nullptr;
+  }
+  for (cudaStream_t* s : {&h.in, &h.out}) {
+    if (*s != nullptr) cudaStreamDestroy(*s);
+    *s = nullptr;
+  }
+  h.ready = false;
+}
+
 HostPipe* host_pipe(int dev) {
   HostPipe& h = g_pipes[dev];
   if (h.ready) return &h;
-  if (cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess)
-    return nullptr;
+  bool ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess;
   for (cudaEvent_t* e : {&h.start, &h.in_done, &h.k_done, &h.out_done})
-    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    host_pipe_reset(h);
+    return nullptr;
+  }
   h.ready = true;
   return &h;
 }

@@ -40,8 +40,9 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Causal attention forward FLOPs as the metric counts them: 2*B*Hq*T^2*d."""
-        return 2.0 * self.B * self.Hq * self.T * self.T * self.d
+        """Attention forward FLOPs as the metric counts them: 2*B*Hq*T^2*d when
+        causal (QK^T and PV over the causal half), 4*B*Hq*T^2*d otherwise."""
+        return (2.0 if self.causal else 4.0) * self.B * self.Hq * self.T * self.T * self.d
 
     @property
     def io_bytes(self) -> int:
@@ -221,6 +222,9 @@ class DecodeWorkload:
 # (Hq=32, Hkv=8, d=128) serving 64 sequences with contexts up to 16384 tokens.
 DECODE = DecodeWorkload("decode_b64_hq32_hkv8_d128_bs16_len1to16384", B=64, Hq=32, Hkv=8,
                         d=128, bs=16, max_len=16384, seed=11)
+# The same serving batch at head dimension 64 (the CUDA-core decode kernel).
+DECODE_D64 = DecodeWorkload("decode_b64_hq32_hkv8_d64_bs16_len1to16384", B=64, Hq=32, Hkv=8,
+                            d=64, bs=16, max_len=16384, seed=11)
 
 
 def make_paged_device(w: DecodeWorkload, device, spare_blocks: int = 3):

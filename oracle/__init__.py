@@ -28,6 +28,7 @@ import ctypes
 import os
 import subprocess
 import threading
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -166,6 +167,131 @@ def attn_rows_bf16(q_bits, k_bits, v_bits, rows, causal: bool = True,
     if rc != 0:
         raise ValueError(f"oracle_attn_rows_bf16 failed with code {rc}")
     return o, lse
+
+
+def host_threads() -> int:
+    """Host cores this process may run on (its CPU affinity), at least 1."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def fwd_runs(B: int, Hq: int, T: int, causal: bool, run_rows: int = 256):
+    """The work units of attn_fwd_bf16_threaded: runs (b, h, i0, i1) of up to
+    ``run_rows`` consecutive query rows of one head, longest causal extent
+    first (a stable sort, so equal extents keep (b, h) order)."""
+    runs = [(b, h, i0, min(i0 + run_rows, T)) for b in range(B) for h in range(Hq)
+            for i0 in range(0, T, run_rows)]
+    if causal:
+        runs.sort(key=lambda r: -r[3])
+    return runs
+
+
+def run_flops(run, d: int, T: int, causal: bool) -> float:
+    """Multiply-add work of one run: 4*d flops per visible key per row (the
+    QK^T dot product and the PV accumulation), as the metric counts them."""
+    _, _, i0, i1 = run
+    if causal:
+        keys = (i1 * (i1 + 1) - i0 * (i0 + 1)) // 2
+    else:
+        keys = (i1 - i0) * T
+    return 4.0 * d * keys
+
+
+def attn_fwd_bf16_threaded(q_bits, k_bits, v_bits, causal: bool = True,
+                           scale: float | None = None, threads: int | None = None,
+                           run_rows: int = 256, runs=None, lib: ctypes.CDLL | None = None):
+    """Every output row of attention on bf16 inputs, on all host cores.
+
+    q_bits: uint16 [B,Hq,T,d]; k_bits, v_bits: uint16 [B,Hkv,T,d] (bf16 bit
+    patterns).  The rows are cut into runs of up to ``run_rows`` consecutive
+    rows of one (b, h) (``fwd_runs``); each run is one call of the C row entry
+    ``oracle_attn_rows_bf16``, writing straight into its slice of the outputs.
+    ctypes releases the GIL during the call, so ``threads`` host threads
+    (default: every core this process may use) work on runs at once.  A row's
+    arithmetic is ``attend_one_row``'s whichever thread runs it, so the result
+    is bit for bit that of one call over all rows.  ``runs`` restricts the work
+    to the given runs (rows outside them are left as NaN).
+    Returns (O [B,Hq,T,d], LSE [B,Hq,T]) in fp64.
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    B, Hq, T, d = q_bits.shape
+    Hkv = k_bits.shape[1]
+    if k_bits.shape != (B, Hkv, T, d) or v_bits.shape != k_bits.shape:
+        raise ValueError("k and v must be [B,Hkv,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.full((B, Hq, T, d), np.nan)
+    lse = np.full((B, Hq, T), np.nan)
+    lib = lib or load()
+    if runs is None:
+        runs = fwd_runs(B, Hq, T, causal, run_rows)
+    qp, kp, vp = (_ptr(a, ctypes.c_uint16) for a in (q_bits, k_bits, v_bits))
+
+    def one(run):
+        b, h, i0, i1 = run
+        rows = np.empty((i1 - i0, 3), dtype=np.int64)
+        rows[:, 0] = b
+        rows[:, 1] = h
+        rows[:, 2] = np.arange(i0, i1)
+        rc = lib.oracle_attn_rows_bf16(qp, kp, vp, B, Hq, Hkv, T, d, int(bool(causal)),
+                                       float(scale), _ptr(rows, ctypes.c_int64), i1 - i0,
+                                       _ptr(o[b, h, i0:i1], ctypes.c_double),
+                                       _ptr(lse[b, h, i0:i1], ctypes.c_double))
+        if rc != 0:
+            raise ValueError(f"oracle_attn_rows_bf16 failed with code {rc} on run {run}")
+
+    with ThreadPoolExecutor(max_workers=threads or host_threads()) as pool:
+        for f in [pool.submit(one, r) for r in runs]:
+            f.result()
+    return o, lse
+
+
+def attn_bwd_threaded(q, k, v, dout, causal: bool = True, scale: float | None = None,
+                      threads: int | None = None, lib: ctypes.CDLL | None = None):
+    """attn_bwd_f64 with its (b, key/value head) slices on all host cores.
+
+    Each slice -- its G query heads, their dO rows, one K/V head -- is one
+    call of ``oracle_attn_bwd_f64`` on contiguous views (B = 1, Hkv = 1).  A
+    slice's dK/dV sums run over the same heads and rows in the same order as
+    in one call over the whole problem, and a dQ row depends only on its own
+    slice, so the result is bit for bit that call's.
+    Returns (dQ, dK, dV) in fp64.
+    """
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape or dout.shape != q.shape:
+        raise ValueError("k, v must be [B,Hkv,T,d] and dout [B,Hq,T,d] matching q")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    G = Hq // Hkv
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(k.shape)
+    lib = lib or load()
+    dp = ctypes.c_double
+
+    def one(bg):
+        b, g = bg
+        hs = slice(g * G, (g + 1) * G)
+        rc = lib.oracle_attn_bwd_f64(_ptr(q[b, hs], dp), _ptr(k[b, g], dp), _ptr(v[b, g], dp),
+                                     _ptr(dout[b, hs], dp), _ptr(dq[b, hs], dp),
+                                     _ptr(dk[b, g], dp), _ptr(dv[b, g], dp), 1, G, 1, T, d,
+                                     int(bool(causal)), float(scale))
+        if rc != 0:
+            raise ValueError(f"oracle_attn_bwd_f64 failed with code {rc} on slice {bg}")
+
+    with ThreadPoolExecutor(max_workers=threads or host_threads()) as pool:
+        for f in [pool.submit(one, (b, g)) for b in range(B) for g in range(Hkv)]:
+            f.result()
+    return dq, dk, dv
 
 
 def attn_bwd_f64(q, k, v, dout, causal: bool = True, scale: float | None = None,

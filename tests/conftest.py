@@ -17,3 +17,17 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
     return oracle.load()
+
+
+@pytest.fixture(scope="session")
+def parity_log():
+    """Appends one JSON record per call to the file named by TESSERA_PARITY_LOG
+    (when set): the whole-tensor error figures of the every-element checks."""
+    import json
+    path = os.environ.get("TESSERA_PARITY_LOG")
+
+    def record(**fields):
+        if path:
+            with open(path, "a") as f:
+                f.write(json.dumps(fields) + "\n")
+    return record

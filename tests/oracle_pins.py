@@ -556,8 +556,52 @@ def pin_varlen_equal_lengths(lib):
     assert np.array_equal(lv, lse.transpose(1, 0, 2).reshape(Hq, B * T))
 
 
+def pin_threaded_forward(lib):
+    """The all-core driver gives, bit for bit, the full fp64 entry's result,
+    whatever the thread count and run length (a ragged run length, rows of
+    several heads and batches, causal and full)."""
+    from causal_gqa_attention_03_b200.inputs import make_qkv, bf16_bits
+    B, Hq, Hkv, T, d = 2, 6, 2, 203, 32
+    q, k, v = make_qkv(B, Hq, Hkv, T, d, seed=17, sigma_qk=2.5)
+    scale = 0.2
+    for causal in (True, False):
+        o, lse = oracle.attn_fwd_f64(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                     causal=causal, scale=scale, lib=lib)
+        for threads, run_rows in ((1, 256), (3, 37), (8, 64)):
+            to, tl = oracle.attn_fwd_bf16_threaded(bf16_bits(q), bf16_bits(k), bf16_bits(v),
+                                                   causal=causal, scale=scale, threads=threads,
+                                                   run_rows=run_rows, lib=lib)
+            assert np.array_equal(to, o) and np.array_equal(tl, lse)
+    # the runs cover every row exactly once, and their flop counts sum to the
+    # closed form 4 d sum_i (i + 1) = 2 d T (T + 1) per head
+    runs = oracle.fwd_runs(B, Hq, T, True, 37)
+    seen = np.zeros((B, Hq, T), dtype=int)
+    for b, h, i0, i1 in runs:
+        seen[b, h, i0:i1] += 1
+    assert np.all(seen == 1)
+    total = sum(oracle.run_flops(r, d, T, True) for r in runs)
+    assert total == B * Hq * 2.0 * d * T * (T + 1)
+    assert sum(oracle.run_flops(r, d, T, False) for r in runs) == B * Hq * 4.0 * d * T * T
+
+
+def pin_threaded_backward(lib):
+    """The per-slice threaded backward gives, bit for bit, one call's result."""
+    B, Hq, Hkv, T, d = 2, 6, 2, 37, 16
+    q = _rand((B, Hq, T, d), 1201, 1.5)
+    k = _rand((B, Hkv, T, d), 1202, 1.5)
+    v = _rand((B, Hkv, T, d), 1203)
+    g = _rand((B, Hq, T, d), 1204)
+    for causal in (True, False):
+        ref = oracle.attn_bwd_f64(q, k, v, g, causal=causal, scale=0.3, lib=lib)
+        for threads in (1, 4):
+            got = oracle.attn_bwd_threaded(q, k, v, g, causal=causal, scale=0.3,
+                                           threads=threads, lib=lib)
+            for r, x in zip(ref, got):
+                assert np.array_equal(r, x)
+
+
 ALL_PINS = [pin_varlen_library, pin_varlen_equal_lengths, pin_rmsnorm_library, pin_rmsnorm_invariants, pin_rope_complex,
             pin_rope_invariants, pin_closed_forms, pin_library_sdpa, pin_decimal_large_logits, pin_invariants,
             pin_rows_entry, pin_bwd_library_autograd, pin_bwd_finite_differences,
             pin_bwd_invariants, pin_bwd_dq_rows_entry, pin_decode_library,
-            pin_decode_invariants]
+            pin_decode_invariants, pin_threaded_forward, pin_threaded_backward]

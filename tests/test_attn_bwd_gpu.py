@@ -11,6 +11,8 @@ dQ, dK, dV, with R = max |reference| over the compared elements,
 max |err| <= 2.5e-2 * R and mean |err| <= 2.5e-3 * R.
 
 * small shapes and the two smallest synthetic workloads: every element;
+* the T = 4096 workload: every element of dQ, dK and dV against the oracle's
+  full backward, its (batch, K/V head) slices run on every host core;
 * the larger workloads: sampled dQ rows computed one by one by the oracle, and
   properties that hold at any size (sum_j dV[j] equals the group's summed dO;
   sum_j dK[j] = 0), checked in fp64 on the GPU.
@@ -58,6 +60,7 @@ def check_grad(got, ref, what):
     err = np.abs(got - ref)
     assert err.max() <= REL_MAX * R, f"{what}: max err {err.max():.3e} vs R {R:.3e}"
     assert err.mean() <= REL_MEAN * R, f"{what}: mean err {err.mean():.3e} vs R {R:.3e}"
+    return float(err.max() / R), float(err.mean() / R)
 
 
 def oracle_bwd(q, k, v, g, causal, scale):
@@ -97,6 +100,24 @@ def test_bwd_small_workloads_every_element(name):
 
 
 LARGE = [n for n in inputs.WORKLOADS if n not in (inputs.SMALL, inputs.TAIL)]
+FULL_BWD = "b4_t4096_hq16_hkv4_d128"
+
+
+def test_bwd_t4096_workload_every_element(parity_log):
+    import time
+    w = inputs.WORKLOADS[FULL_BWD]
+    q, k, v = inputs.workload_inputs(w)
+    g = inputs.workload_grad(w)
+    got = run_gpu_bwd(q, k, v, g, True, w.scale)
+    t0 = time.perf_counter()
+    ref = oracle.attn_bwd_threaded(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                   g.double().numpy(), causal=True, scale=w.scale)
+    el = time.perf_counter() - t0
+    for gname, a, r in zip(("dQ", "dK", "dV"), got, ref):
+        rmax, rmean = check_grad(a.numpy(), r, f"{gname} {FULL_BWD}")
+        parity_log(test="backward every element", workload=FULL_BWD, grad=gname,
+                   max_err_over_R=rmax, mean_err_over_R=rmean, elements=int(r.size),
+                   oracle_s=round(el, 1), oracle_threads=oracle.host_threads())
 
 
 @pytest.mark.parametrize("name", LARGE)

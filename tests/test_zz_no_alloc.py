@@ -43,10 +43,11 @@ def _both(q, k, v, g, causal, scale):
 
 
 def _same(ref, got, what):
-    # dK and dV are summed in a fixed order: bit for bit.  dQ adds partials
-    # with atomics, so only its rounding may differ.
-    assert torch.equal(ref[1], got[1]) and torch.equal(ref[2], got[2]), what
-    assert torch.allclose(ref[0].float(), got[0].float(), rtol=2e-2, atol=1e-3), what
+    # Both entry points run the same three launches on the same data, and no
+    # gradient is summed with atomics: dQ, dK and dV must agree bit for bit.
+    # A stale row of the scratch array would show up here.
+    for r, g_, name in zip(ref, got, ("dQ", "dK", "dV")):
+        assert torch.equal(r, g_), f"{what}: {name} differs"
 
 
 @pytest.mark.gpu
