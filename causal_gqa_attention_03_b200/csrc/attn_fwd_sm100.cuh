@@ -240,11 +240,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // s: the row's 128 raw scores.  Masked keys (kv0 + c > lim) become -inf when
 // kMasked.  Updates the running (possibly stale) max m in scaled log2 units,
 // sets alpha = 2^(m_old - m_new) (1 when m is kept) and rescale, writes P as
-// bf16 pairs into pk and returns the row sum of the fp32 p.
+// bf16 pairs into pk, and returns the row sum of the fp32 p (for the LSE)
+// and, in applied, the row sum of the bf16-rounded p that the P.V product
+// applies (O is normalised by it, so O stays an exact convex combination of
+// V rows whatever the rounding of the dominant weights).
 template <bool kMasked>
 __device__ __forceinline__ float softmax_row_tile(float (&s)[128], uint32_t (&pk)[2][32], float& m,
                                                   float& alpha, bool& rescale, float sl2, int kv0,
-                                                  int lim) {
+                                                  int lim, float& applied) {
   if (kMasked) {
 #pragma unroll
     for (int c = 0; c < 128; ++c)
@@ -268,9 +271,9 @@ __device__ __forceinline__ float softmax_row_tile(float (&s)[128], uint32_t (&pk
   const float neg_m = (m == -INFINITY) ? 0.f : -m;
   const float2 sl2_2 = make_float2(sl2, sl2);
   const float2 nm_2 = make_float2(neg_m, neg_m);
-  float2 acc[4];
+  float2 acc[4], accb[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+  for (int k = 0; k < 4; ++k) acc[k] = accb[k] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 64; ++c) {
     const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sl2_2, nm_2);
@@ -282,9 +285,13 @@ __device__ __forceinline__ float softmax_row_tile(float (&s)[128], uint32_t (&pk
       pv.y = ptx::ex2(x.y);
     }
     acc[c & 3] = __fadd2_rn(acc[c & 3], pv);
-    pk[c >> 5][c & 31] = ptx::pack_bf16x2(pv.x, pv.y);
+    const uint32_t packed = ptx::pack_bf16x2(pv.x, pv.y);
+    pk[c >> 5][c & 31] = packed;
+    accb[c & 3] = ptx::add_bf16x2_f32(accb[c & 3], packed);
   }
   const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  const float2 ab = __fadd2_rn(__fadd2_rn(accb[0], accb[1]), __fadd2_rn(accb[2], accb[3]));
+  applied = ab.x + ab.y;
   return a.x + a.y;
 }
 
@@ -532,6 +539,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const int q_row = w.qblk[t] * C::BM + row;
       float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale)
       float l = 0.f;        // running sum of 2^(x - m)
+      float lb = 0.f;       // running sum of the bf16-rounded 2^(x - m) that P.V applies
       for (int j = 0; j < n_t; ++j) {
         if (!warp_wait(&s_full[t], scnt & 1, kErrWaitSFull, p.launch_id)) {
           ok = false;
@@ -554,10 +562,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         float alpha;
         bool rescale;
         uint32_t pk[2][32];
+        float applied;
         const float rowsum =
-            edge ? softmax_row_tile<true>(sv, pk, m, alpha, rescale, sl2, kv0, lim)
-                 : softmax_row_tile<false>(sv, pk, m, alpha, rescale, sl2, kv0, lim);
+            edge ? softmax_row_tile<true>(sv, pk, m, alpha, rescale, sl2, kv0, lim, applied)
+                 : softmax_row_tile<false>(sv, pk, m, alpha, rescale, sl2, kv0, lim, applied);
         l = l * alpha + rowsum;
+        lb = lb * alpha + applied;
         ptx::tmem_st32(s_addr + 0, pk[0]);
         ptx::tmem_st32(s_addr + 32, pk[1]);
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
@@ -584,7 +594,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       if (!warp_wait(&o_full[t], ocnt & 1, kErrWaitOFull, p.launch_id)) break;
       ++ocnt;
       ptx::tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (lb > 0.f) ? 1.f / lb : 0.f;
       const bool store = q_row < w.T;
       // O and LSE element offsets of this row: [B,Hq,T,d] / [B,Hq,T], or packed
       // [total,Hq,d] / [Hq,total]
