@@ -16,7 +16,6 @@
 
 #include "tessera_attn.h"
 #include "attn_fwd_sm100.cuh"
-#include "attn_fwd_pair_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
 #include "paged_decode.cuh"
 #include "paged_decode_tc.cuh"
@@ -49,15 +48,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // [planes, T, d] bf16 viewed as a 3-D tensor (d innermost); boxes of
 // 64 columns x 128 rows x 1 plane with the 128-byte swizzle.  Rows at or past
 // T read as zero.
-bool make_map(CUtensorMap* map, const void* base, int planes, int T, int d,
-              unsigned box_rows = 128) {
+bool make_map(CUtensorMap* map, const void* base, int planes, int T, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
                         static_cast<cuuint64_t>(planes)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t elem[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                   strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -159,79 +157,6 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   return TESSERA_OK;
 }
 
-// One launch of the CTA-pair forward (head dimension 128, fixed length):
-// clusters of two CTAs, as many as fit on the device at once, each walking
-// its share of the units.
-int launch_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                int Hkv, int T, int causal, float scale, cudaStream_t stream) {
-  using C = tessera::PairCfg;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return TESSERA_ERR_CUDA;
-  static std::atomic<int> max_clusters[64];
-  if (dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
-  int clusters = max_clusters[dev].load(std::memory_order_acquire);
-  if (clusters == 0) {
-    if (cudaFuncSetAttribute(tessera::attn_fwd_pair_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return TESSERA_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(C::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&clusters, tessera::attn_fwd_pair_kernel, &cfg) !=
-            cudaSuccess ||
-        clusters <= 0)
-      return TESSERA_ERR_CUDA;
-    max_clusters[dev].store(clusters, std::memory_order_release);
-  }
-
-  CUtensorMap tm_q, tm_kh, tm_v, tm_o;
-  if (!make_map(&tm_q, q, B * Hq, T, C::D) || !make_map(&tm_kh, k, B * Hkv, T, C::D, 64) ||
-      !make_map(&tm_v, v, B * Hkv, T, C::D) || !make_map(&tm_o, o, B * Hq, T, C::D))
-    return TESSERA_ERR_CUDA;
-
-  FwdParams p;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.T = T;
-  p.G = Hq / Hkv;
-  p.causal = causal ? 1 : 0;
-  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.nqb = (T + C::BM - 1) / C::BM;
-  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
-  long long units;
-  if (p.pair_heads) {
-    p.units_per_step = B * Hkv * (p.G / 2);
-    units = static_cast<long long>(p.units_per_step) * p.nqb;
-  } else {
-    p.units_per_step = B * Hq;
-    units = static_cast<long long>(p.units_per_step) * ((p.nqb + 1) / 2);
-  }
-  if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
-  p.num_units = static_cast<int>(units);
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
-  p.cu_seqlens = nullptr;
-  p.total = 0;
-
-  const unsigned grid = 2u * static_cast<unsigned>(units < clusters ? units : clusters);
-  tessera::attn_fwd_pair_kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tm_q, tm_kh, tm_v,
-                                                                              tm_o, p);
-  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-  g_last_launches = 1;
-  return TESSERA_OK;
-}
-
 // Checks shared by the entry points (before any CUDA call).  Returns
 // TESSERA_OK with *empty set when there is nothing to compute.
 int check_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -265,7 +190,7 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
 int launch_d(int d, const void* q, const void* k, const void* v, void* o, float* lse, int B,
              int Hq, int Hkv, int T, int causal, float scale, cudaStream_t s) {
   if (d == 64) return launch<64>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
-  return launch_pair(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
+  return launch<128>(q, k, v, o, lse, B, Hq, Hkv, T, causal, scale, s);
 }
 
 // Streams and events of the host-buffer pipeline, created on first use per

@@ -190,9 +190,12 @@ __device__ __forceinline__ int unit_of(const FwdParams& p, int k) {
 
 // Wait for the phase of `parity` on `bar`, giving up after limit_ns or as
 // soon as another CTA of the same launch has given up.  Returns false on give-up.
+// A phase that has already completed is seen by the non-blocking test (the
+// blocking try_wait costs a few hundred cycles even then).
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, uint32_t code,
                                              unsigned long long launch_id,
                                              uint64_t limit_ns = kWaitLimitNs) {
+  if (ptx::mbar_test_wait(bar, parity)) return true;
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {

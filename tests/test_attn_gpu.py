@@ -91,10 +91,9 @@ SMALL = [
     (1, 8, 1, 385, 128, True), (1, 1, 1, 640, 64, True), (2, 6, 3, 200, 128, True),
     (1, 2, 1, 1, 64, False), (1, 4, 2, 100, 64, False), (1, 3, 1, 129, 128, False),
     (2, 2, 2, 256, 128, False), (1, 4, 4, 383, 64, False), (1, 8, 2, 520, 128, False),
-    # head dimension 128 runs on CTA pairs: an odd number of 128-row blocks
-    # with G odd (the pair's second tile lies past T), key tails of at most 64
-    # rows (the odd CTA's half of the last K tile lies past T), units of one,
-    # two and many key tiles
+    # more head-dimension-128 shapes: an odd number of 128-row blocks with G
+    # odd (a unit's second tile lies past T), key tails of at most 64 rows,
+    # units of one, two and many key tiles
     (1, 3, 1, 300, 128, True), (1, 1, 1, 640, 128, True), (1, 5, 5, 333, 128, False),
     (2, 4, 1, 1000, 128, True), (1, 2, 1, 64, 128, True), (3, 6, 2, 190, 128, True),
 ]
