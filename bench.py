@@ -671,7 +671,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--only", choices=["backward", "decode", "prologue", "varlen"],
+    ap.add_argument("--only", choices=["forward", "backward", "decode", "prologue", "varlen"],
                     help="time one extra leg alone and print its object (for profiling it)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -901,7 +901,13 @@ def one_leg(args, tess, torch, dev, world, rank, local):
     time.sleep(0.3)
     t0 = time.time()
     w = inputs.WORKLOADS[args.workload]
-    if args.only == "backward":
+    if args.only == "forward":
+        q, k, v = (t.to(dev) for t in inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
+                                                     rank_seed(w.seed, rank), w.sigma_qk))
+        times, launches, _, _ = time_kernel(w, q, k, v, args.steps, args.warmup, flush, stream,
+                                            tess, torch)
+        max_ms = max_over_ranks(sum(times), dev)
+    elif args.only == "backward":
         q, k, v = (t.to(dev) for t in inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
                                                      rank_seed(w.seed, rank), w.sigma_qk))
         g = inputs.make_grad(w.B, w.Hq, w.T, w.d,
@@ -933,7 +939,17 @@ def one_leg(args, tess, torch, dev, world, rank, local):
     if rank != 0:
         return 0
     peaks, peak_src = load_peaks()
-    if args.only == "backward":
+    if args.only == "forward":
+        achieved = w.flops / (statistics.mean(times) * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        line = {"metric": METRIC, "value": round(w.flops * args.steps * world / (max_ms * 1e-3) / 1e12, 2),
+                "unit": UNIT, "steps": args.steps, "ms_per_step": round(max_ms / args.steps, 5),
+                "config": config_of(w, world), "gpu_launches": launches,
+                "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                             "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)",
+                             **north_star_roofline(achieved, w)}}
+    elif args.only == "backward":
         line = backward_line(w, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
         line["config"] = {"workload": args.workload}
     elif args.only == "decode":

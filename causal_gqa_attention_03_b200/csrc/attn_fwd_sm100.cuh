@@ -290,7 +290,7 @@ __device__ __forceinline__ float softmax_row_tile(float (&s)[128], uint32_t (&pk
     acc[c & 3] = __fadd2_rn(acc[c & 3], pv);
     const uint32_t packed = ptx::pack_bf16x2(pv.x, pv.y);
     pk[c >> 5][c & 31] = packed;
-    accb[c & 3] = ptx::add_bf16x2_f32(accb[c & 3], packed);
+    accb[c & 3] = __fadd2_rn(accb[c & 3], ptx::bf16x2_to_float2(packed));
   }
   const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
   const float2 ab = __fadd2_rn(__fadd2_rn(accb[0], accb[1]), __fadd2_rn(accb[2], accb[3]));
@@ -610,25 +610,46 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         orow = (static_cast<int64_t>(w.b) * p.Hq + w.head[t]) * p.T + q_row;
         lrow = orow;
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+      // The row as D/8 pieces of 16 bytes, then stored by lane pairs: lanes
+      // 2m and 2m+1 swap one piece per step (shfl.xor 1), so every warp store
+      // writes 32 contiguous bytes of each of 16 rows -- whole 32-byte
+      // sectors, 16 per 512-byte request.
+      uint32_t packed[D / 2];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         ptx::tmem_ld32(o_addr + 32 * c, ov);
         ptx::tmem_ld_wait();
         ptx::reg_fence(ov);
-        uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          packed[i] = ptx::pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
-                                       __uint_as_float(ov[2 * i + 1]) * inv_l);
-        if (store) {
+          packed[16 * c + i] = ptx::pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
+                                               __uint_as_float(ov[2 * i + 1]) * inv_l);
+      }
+      const bool odd = lane & 1;
+      __nv_bfloat16* const dst = p.o + orow * D;
+      const unsigned long long dst_bits = reinterpret_cast<unsigned long long>(dst);
+      uint4* const row_even =
+          reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, dst_bits, lane & ~1));
+      uint4* const row_odd =
+          reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, dst_bits, lane | 1));
+      const bool st_even = __shfl_sync(0xffffffffu, store, lane & ~1);
+      const bool st_odd = __shfl_sync(0xffffffffu, store, lane | 1);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            ptx::st_global_cs_v4(dst + c * 4 + v4,
-                                 make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2],
-                                            packed[4 * v4 + 3]));
+      for (int k = 0; k < D / 16; ++k) {
+        // pieces 2k (even lane's) and 2k+1 (odd lane's) of both rows
+        uint32_t send[4], recv[4], v1[4], v2[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          send[w] = odd ? packed[8 * k + w] : packed[8 * k + 4 + w];
+          recv[w] = __shfl_xor_sync(0xffffffffu, send[w], 1);
+          v1[w] = odd ? recv[w] : packed[8 * k + w];      // the even lane's row
+          v2[w] = odd ? packed[8 * k + 4 + w] : recv[w];  // the odd lane's row
         }
+        if (st_even)
+          ptx::st_global_cs_v4(row_even + 2 * k + odd, make_uint4(v1[0], v1[1], v1[2], v1[3]));
+        if (st_odd)
+          ptx::st_global_cs_v4(row_odd + 2 * k + odd, make_uint4(v2[0], v2[1], v2[2], v2[3]));
       }
       if (store && p.lse != nullptr)
         p.lse[lrow] = (l > 0.f) ? (m + ptx::lg2(l)) * 0.69314718055994530942f : -INFINITY;
