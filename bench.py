@@ -546,7 +546,8 @@ def prologue_line(w, res, peaks, peak_src):
         line[name] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 5),
                       "bytes_per_step": nbytes, "gpu_launches": launches,
                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
-                                   "unit": "GB/s", "frac": round(gbs / hbm, 4), "traffic": None,
+                                   "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                                   "traffic": traffic_bytes(name, w.name),
                                    "peak_source": f"{peak_src} hbm_gbs"}}
     return line
 
@@ -622,7 +623,7 @@ def varlen_line(wv, times, launches, peaks, peak_src):
             "flop_count": "sum over sequences of the metric's 2*Hq*T_b^2*d",
             "config": wv.describe(), "gpu_launches": launches,
             "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak,
-                         "unit": UNIT, "frac": round(tf / peak, 4), "traffic": None,
+                         "unit": UNIT, "frac": round(tf / peak, 4), "traffic": traffic_bytes("varlen", wv.name),
                          "peak_source": f"{peak_src} bf16_tflops (burst)"},
             "l2": "flushed before every timed step"}
 
@@ -823,13 +824,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    traffic = None
-    prof_traffic = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof_traffic):
-        with open(prof_traffic) as f:
-            tr = json.load(f)
-        if tr.get("workload") == w.name and tr.get("kernel_source_sha") == kernel_source_sha():
-            traffic = tr.get("bytes_per_launch")
+    traffic = traffic_bytes("forward", w.name)
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                 "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
@@ -946,7 +941,7 @@ def one_leg(args, tess, torch, dev, world, rank, local):
                 "unit": UNIT, "steps": args.steps, "ms_per_step": round(max_ms / args.steps, 5),
                 "config": config_of(w, world), "gpu_launches": launches,
                 "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                             "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                             "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic_bytes("forward", w.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)",
                              **north_star_roofline(achieved, w)}}
     elif args.only == "backward":
@@ -980,7 +975,7 @@ def backward_line(w, times, max_ms, steps, launches, ws_bytes, world, peaks, pea
             "flop_count": "5*B*Hq*T^2*d: five products over the causal triangle, "
                           "counted as the forward's 2*B*Hq*T^2*d counts two",
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                         "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic_bytes("backward", w.name),
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "issued_flops_per_step": 3.5 * w.flops,
                          "issued_frac": round(1.4 * achieved / peak, 4)},
@@ -1001,7 +996,7 @@ def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak
             "unit": "GB/s", "steps": steps, "ms_per_step": round(max_ms / steps, 5),
             "config": wd.describe(),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic_bytes("decode", wd.name),
                          "peak_source": f"{peak_src} hbm_gbs",
                          "bytes_per_step": nbytes,
                          "byte_count": "K and V rows of every cached token, q, o, lse, "
@@ -1026,19 +1021,38 @@ def north_star_roofline(achieved: float, w) -> dict:
             "north_star_target_frac": 0.60, "north_star_target_met": bool(frac >= 0.60)}
 
 
-# The files the forward kernel is built from: its traffic record stays valid
-# while they are unchanged.
-FWD_SOURCES = ("attn_fwd_sm100.cuh", "exp2_fma.cuh", "sm100_ptx.cuh")
+# The kernel headers each leg is built from: a leg's DRAM-traffic record in
+# profiles/traffic.json stays valid while they are unchanged.
+_FWD_SOURCES = ["attn_fwd_sm100.cuh", "exp2_fma.cuh", "sm100_ptx.cuh"]
+LEG_SOURCES = {"forward": _FWD_SOURCES, "varlen": _FWD_SOURCES,
+               "backward": ["attn_bwd_sm100.cuh"] + _FWD_SOURCES,
+               "decode": ["paged_decode_tc.cuh", "paged_decode.cuh"] + _FWD_SOURCES,
+               "rmsnorm": ["prologue.cuh"], "rope_qkv": ["prologue.cuh"]}
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(leg: str = "forward") -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_gqa_attention_03_b200", "csrc")
-    for name in FWD_SOURCES:
+    for name in LEG_SOURCES[leg]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def traffic_bytes(leg: str, workload: str):
+    """DRAM bytes (read + write) per launch of the leg's kernels, from the
+    one-pass ncu capture recorded in profiles/traffic.json; None when there is
+    no record for this workload or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get("records", {}).get(leg)
+    if (not rec or not str(rec.get("workload", "")).startswith(workload)
+            or rec.get("kernel_source_sha") != kernel_source_sha(leg)):
+        return None
+    return rec.get("bytes_per_launch")
 
 
 if __name__ == "__main__":
