@@ -12,7 +12,7 @@ scaling: independent batches, no collective on the data path); the reported
 time is the max over ranks.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
-on the host cores instead, on a bounded sample of rows of the same workload.
+on every host core instead, on bounded random samples of the same workload.
 """
 from __future__ import annotations
 
@@ -403,6 +403,22 @@ def time_back_to_back(w, q, k, v, n, stream, tess, torch):
         tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
     b.record(stream)
     torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def time_empty_launches(n, stream, torch):
+    """Mean time of n empty kernels (torch's 0-cycle sleep) queued back to
+    back on `stream`: the launch floor of the device and driver."""
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            torch.cuda._sleep(0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            torch.cuda._sleep(0)
+        b.record(stream)
+        torch.cuda.synchronize()
     return a.elapsed_time(b) / n
 
 
@@ -802,6 +818,10 @@ def main():
             sweep[name]["warm_ms"] = round(warm, 4)
             sweep[name]["warm_tflops"] = round(ws.flops / (warm * 1e-3) / 1e12, 1)
             sweep[name]["warm_launches"] = nb
+            if ws.flops < 1e9:
+                # the launch floor on the same stream: an empty kernel (torch's
+                # 0-cycle sleep) back to back, for the tiny workload's context
+                sweep[name]["empty_launch_ms"] = round(time_empty_launches(1000, stream, torch), 4)
             gs = inputs.workload_grad(ws).to(dev)
             n = max(5, min(100, int(0.3 / max(2.5 * ws.flops / 5e14, 1e-6))))
             tb, _, _ = time_backward(ws, qs, ks, vs, gs, n, 3, flush, stream, tess, torch)

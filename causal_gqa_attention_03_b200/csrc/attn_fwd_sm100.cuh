@@ -137,8 +137,21 @@ struct Unit {
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit w;
-  const int step = u / p.units_per_step;
-  const int r = u % p.units_per_step;
+  int step, r;
+  if (p.cu_seqlens != nullptr) {
+    // Packed sequences: sequence-major (all of sequence 0's units, heaviest
+    // first, then sequence 1's, ...), so the CTAs work on about one
+    // sequence's keys and values at a time and those stay in L2.
+    const int per_seq_step = p.units_per_step / p.B;
+    const int per_seq = per_seq_step * (p.pair_heads ? p.nqb : (p.nqb + 1) >> 1);
+    const int b = u / per_seq;
+    const int rest = u % per_seq;
+    step = rest / per_seq_step;
+    r = b * per_seq_step + rest % per_seq_step;
+  } else {
+    step = u / p.units_per_step;
+    r = u % p.units_per_step;
+  }
   if (p.pair_heads) {
     const int half = p.G >> 1;
     const int hp = r % half;
