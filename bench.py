@@ -428,7 +428,7 @@ def time_backward(w, q, k, v, g, steps, warmup, flush, stream, tess, torch):
     launches."""
     o, lse = tess.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, stream=stream)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    nbytes = tess.tessera_attn_bwd_workspace_bytes(w.B, w.Hq, w.T, w.d)
+    nbytes = tess.tessera_attn_bwd_workspace_bytes_kv(w.B, w.Hq, w.Hkv, w.T, w.d)
     ws = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=q.device)
 
     def call():

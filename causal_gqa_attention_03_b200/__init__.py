@@ -9,6 +9,7 @@ Raw C-ABI names (integer pointers, sizes, stream handle):
     tessera_attn_fwd, tessera_attn_fwd_host, tessera_attn_device_error,
     tessera_status_str, tessera_attn_last_launch_count,
     tessera_attn_selftest_timeout, tessera_attn_bwd, tessera_attn_bwd_workspace_bytes,
+    tessera_attn_bwd_workspace_bytes_kv,
     tessera_attn_bwd_noalloc, tessera_attn_bwd_noalloc_max_workspace_bytes,
     tessera_attn_decode, tessera_attn_decode_workspace_bytes, tessera_rmsnorm,
     tessera_rope_qkv, tessera_attn_fwd_varlen
@@ -35,7 +36,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_
 
 # Symbols declared in include/tessera_attn.h.
 EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
-            "tessera_attn_bwd_workspace_bytes", "tessera_attn_bwd_noalloc",
+            "tessera_attn_bwd_workspace_bytes", "tessera_attn_bwd_workspace_bytes_kv",
+            "tessera_attn_bwd_noalloc",
             "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
             "tessera_status_str", "tessera_attn_last_launch_count",
             "tessera_attn_selftest_timeout", "tessera_attn_decode",
@@ -87,6 +89,8 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_bwd.restype = ci
             lib.tessera_attn_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
             lib.tessera_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.tessera_attn_bwd_workspace_bytes_kv.argtypes = [ci, ci, ci, ci, ci]
+            lib.tessera_attn_bwd_workspace_bytes_kv.restype = ctypes.c_size_t
             lib.tessera_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci,
                                                      ci, ci, ci, ci, ctypes.c_float, vp]
             lib.tessera_attn_bwd_noalloc.restype = ci
@@ -147,6 +151,10 @@ def tessera_attn_bwd(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: in
 
 def tessera_attn_bwd_workspace_bytes(B: int, Hq: int, T: int, d: int) -> int:
     return load_library().tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
+
+
+def tessera_attn_bwd_workspace_bytes_kv(B: int, Hq: int, Hkv: int, T: int, d: int) -> int:
+    return load_library().tessera_attn_bwd_workspace_bytes_kv(B, Hq, Hkv, T, d)
 
 
 def tessera_attn_bwd_noalloc(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: int,
@@ -318,8 +326,10 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = N
 
     q, o, dout: bf16 [B,Hq,T,d]; k, v: bf16 [B,Hkv,T,d]; lse: fp32 [B,Hq,T]
     from attn_fwd with the same arguments.  Outputs are bf16 and allocated
-    with torch unless given; the fp32 workspace likewise.  Queued on
-    ``stream`` (default: torch's current stream); does not synchronise.
+    with torch unless given; the fp32 workspace likewise (sized by
+    tessera_attn_bwd_workspace_bytes_kv, so shapes with few key/value units
+    get the balanced dK/dV form).  Queued on ``stream`` (default: torch's
+    current stream); does not synchronise.
     """
     import torch
 
@@ -342,7 +352,7 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = N
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    nbytes = tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
+    nbytes = tessera_attn_bwd_workspace_bytes_kv(B, Hq, Hkv, T, d)
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16) + 3) // 4, dtype=torch.float32, device=q.device)
     if stream is None:

@@ -237,6 +237,27 @@ size_t bwd_workspace_bytes(int B, int Hq, int T, int /*d*/) {
   return static_cast<size_t>(B) * Hq * T * 4;
 }
 
+// Parts per (batch, key/value head, key block) of the dK/dV kernel: doubled
+// while the units number under 512 (about four per SM) and the group's query
+// heads divide evenly, up to 8.  Depends on the shape only.
+int bwd_split(int B, int Hkv, int G, int T) {
+  const long long units = static_cast<long long>(B) * Hkv * ((T + 127) / 128);
+  int s = 1;
+  while (s < 8 && units * s < 512 && G % (2 * s) == 0) s *= 2;
+  return s;
+}
+
+// Byte offset of the split partials in the workspace (after D, 256-aligned)
+// and the whole workspace with them: [split][B*Hkv*T][2][d] fp32.
+size_t bwd_part_offset(int B, int Hq, int T, int d) {
+  return (bwd_workspace_bytes(B, Hq, T, d) + 255) & ~static_cast<size_t>(255);
+}
+size_t bwd_split_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int split) {
+  if (split <= 1) return bwd_workspace_bytes(B, Hq, T, d);
+  return bwd_part_offset(B, Hq, T, d) +
+         static_cast<size_t>(split) * B * Hkv * T * static_cast<size_t>(d) * 2 * 4;
+}
+
 int sm_count(int dev) {
   static std::atomic<int> counts[64];
   int sms = counts[dev].load(std::memory_order_acquire);
@@ -251,8 +272,8 @@ int sm_count(int dev) {
 
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-               const void* dout, void* dq, void* dk, void* dv, float* ws, int B, int Hq, int Hkv,
-               int T, int causal, float scale, cudaStream_t stream) {
+               const void* dout, void* dq, void* dk, void* dv, float* ws, size_t ws_bytes, int B,
+               int Hq, int Hkv, int T, int causal, float scale, cudaStream_t stream) {
   using C = BwdCfg<D>;
   using Q = tessera::DqCfg<D>;
   int dev = 0;
@@ -272,7 +293,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (sms <= 0) return TESSERA_ERR_CUDA;
   const long long rows = static_cast<long long>(B) * Hq * T;
   const int nqb = (T + C::BM - 1) / C::BM;
-  const long long kv_units = static_cast<long long>(B) * Hkv * nqb;  // kernel 2
+  // kernel 2's units, split by query heads when the workspace holds the partials
+  int split = bwd_split(B, Hkv, Hq / Hkv, T);
+  if (split > 1 && ws_bytes < bwd_split_workspace_bytes(B, Hq, Hkv, T, D, split)) split = 1;
+  const long long kv_units = static_cast<long long>(B) * Hkv * nqb * split;  // kernel 2
   const long long q_units = static_cast<long long>(B) * Hq * nqb;    // kernel 3
   if (q_units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;  // before any launch
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
@@ -301,13 +325,27 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  // 2. dK, dV: units (batch, key/value head, key block)
+  p.split = split;
+  p.dkv_part = split > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
+                                                    bwd_part_offset(B, Hq, T, D))
+                         : nullptr;
+  // 2. dK, dV: units (batch, key/value head, key block, query-head part)
   p.num_units = static_cast<int>(kv_units);
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
   const unsigned grid = static_cast<unsigned>(kv_units < sms ? kv_units : sms);
   tessera::attn_bwd_dkdv_sm100_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
       tm_q, tm_k, tm_v, tm_do, p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  if (split > 1) {
+    // 2b. dK, dV = the partials summed in part order
+    const long long kv_rows = static_cast<long long>(B) * Hkv * T;
+    const long long n4 = kv_rows * 2 * (D / 4);
+    const long long blocks = (n4 + 255) / 256;
+    const unsigned rb = static_cast<unsigned>(blocks < 8LL * sms ? blocks : 8LL * sms);
+    tessera::attn_bwd_dkv_reduce_kernel<D><<<rb, 256, 0, stream>>>(
+        p.dkv_part, p.dk, p.dv, kv_rows, split);
+    if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
+  }
   // 3. dQ: units (batch, query head, query block)
   p.num_units = static_cast<int>(q_units);
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
@@ -316,7 +354,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
       tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout),
       p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-  g_last_launches = 3;
+  g_last_launches = split > 1 ? 4 : 3;
   return TESSERA_OK;
 }
 
@@ -736,9 +774,15 @@ extern "C" int tessera_attn_bwd(const void* q, const void* k, const void* v, con
   if (st != TESSERA_OK || empty) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal,
-                                     scale, s);
-  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, T, causal, scale, s);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, workspace_bytes, B, Hq,
+                                     Hkv, T, causal, scale, s);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, workspace_bytes, B, Hq, Hkv, T,
+                         causal, scale, s);
+}
+
+extern "C" size_t tessera_attn_bwd_workspace_bytes_kv(int B, int Hq, int Hkv, int T, int d) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || T < 0 || (d != 64 && d != 128)) return 0;
+  return bwd_split_workspace_bytes(B, Hq, Hkv, T, d, bwd_split(B, Hkv, Hq / Hkv, T));
 }
 
 extern "C" size_t tessera_attn_bwd_noalloc_max_workspace_bytes(void) {
@@ -761,9 +805,10 @@ extern "C" int tessera_attn_bwd_noalloc(const void* q, const void* k, const void
   if (sst != TESSERA_OK) return sst;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* wsf = static_cast<float*>(ws);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, wsf, B, Hq, Hkv, T,
-                                     causal, scale, s);
-  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, wsf, B, Hq, Hkv, T, causal, scale, s);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, wsf, kNoAllocScratchBytes,
+                                     B, Hq, Hkv, T, causal, scale, s);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, wsf, kNoAllocScratchBytes, B, Hq, Hkv,
+                         T, causal, scale, s);
 }
 
 extern "C" size_t tessera_attn_decode_workspace_bytes(int B, int Hq, int max_seq_len, int d) {

@@ -11,7 +11,7 @@
 // differentiates is the FlashAttention forward they name (hysenlabs.com
 // Tessera review, "The kernel set and its torch fallback").
 //
-// Three launches, no atomics and no fp32 accumulator in global memory:
+// Three launches (four with split key/value units, below), no atomics:
 //   1. attn_bwd_prep_kernel: D = rowsum(dO * O) in fp32.
 //   2. attn_bwd_dkdv_sm100_kernel<D>: one CTA per SM walks units
 //      (batch, key/value head, 128-key block), heaviest first.  A unit keeps
@@ -27,6 +27,13 @@
 // per query/key block pair instead of five); in exchange no dQ partial ever
 // goes through L2 reductions, which bound the single-kernel form (a 64 KB
 // fp32 partial per visit).
+//
+// Few key/value units (B * Hkv * key blocks below about four per SM, e.g.
+// multi-query attention) leave SMs idle and put the heaviest unit on the
+// critical path.  When the caller's workspace allows, kernel 2's units are
+// then cut by query heads into `split` parts whose fp32 partial dK, dV are
+// summed by attn_bwd_dkv_reduce_kernel (a fourth launch) in a fixed order,
+// so results stay independent of scheduling.
 #pragma once
 
 #include "attn_fwd_sm100.cuh"
@@ -68,6 +75,37 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) dvec[r] = acc;
+  }
+}
+
+// dV, dK = the sum over `split` fp32 partials [split][rows][2][D] (dV first,
+// then dK, already scaled) -> bf16, in part order.  rows = B*Hkv*T.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dkv_reduce_kernel(
+    const float* __restrict__ part, __nv_bfloat16* __restrict__ dk,
+    __nv_bfloat16* __restrict__ dv, long long rows, int split) {
+  constexpr int V4 = D / 4;  // float4 groups per row and gradient
+  const long long n = rows * 2 * V4;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += stride) {
+    const long long row = i / (2 * V4);
+    const int which = static_cast<int>((i / V4) & 1);
+    const int c4 = static_cast<int>(i % V4);
+    const float4* src = reinterpret_cast<const float4*>(part) + i;
+    float4 acc = src[0];
+    for (int s = 1; s < split; ++s) {
+      const float4 x = src[static_cast<long long>(s) * rows * 2 * V4];
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    __nv_bfloat16* out = (which == 0 ? dv : dk) + row * D + 4 * c4;
+    uint2 packed;
+    packed.x = ptx::pack_bf16x2(acc.x, acc.y);
+    packed.y = ptx::pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(out) = packed;
   }
 }
 
@@ -135,24 +173,35 @@ struct BwdParams {
   __nv_bfloat16* dk;         // [B, Hkv, T, D]
   __nv_bfloat16* dv;
   unsigned long long launch_id;
+  // kernel 2: each (batch, key/value head, key block) is cut into `split`
+  // units by query heads (G / split each).  With split > 1 the units write
+  // fp32 partial dV, scale * dK to dkv_part [split][B*Hkv*T][2][D], which
+  // attn_bwd_dkv_reduce_kernel sums into dV, dK.
+  int split;
+  float* dkv_part;
 };
 
-// Unit u: key block kb = u / (B * Hkv) (ascending: the longest causal
-// extents first), batch and key/value head from the rest.
+// Unit u: key block kb = u / (B * Hkv * split) (ascending: the longest
+// causal extents first), batch, key/value head and query-head part from the
+// rest.
 struct BwdUnit {
   int b, g, kb;
+  int part;     // which G / split query heads of the group
   int qb0;      // first query block that sees the keys
-  int nvisit;   // G * (nqb - qb0)
+  int nvisit;   // (G / split) * (nqb - qb0)
 };
 
 __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdParams& p, int u) {
   BwdUnit w;
-  const int bg = u % (p.B * p.Hkv);
-  w.kb = u / (p.B * p.Hkv);
+  const int groups = p.B * p.Hkv * p.split;
+  const int rest = u % groups;
+  w.kb = u / groups;
+  w.part = rest % p.split;
+  const int bg = rest / p.split;
   w.b = bg / p.Hkv;
   w.g = bg % p.Hkv;
   w.qb0 = p.causal ? w.kb : 0;
-  w.nvisit = p.G * (p.nqb - w.qb0);
+  w.nvisit = (p.G / p.split) * (p.nqb - w.qb0);
   return w;
 }
 
@@ -164,11 +213,13 @@ __device__ __forceinline__ int bwd_unit_of(const BwdParams& p, int k) {
   return u < p.num_units ? static_cast<int>(u) : -1;
 }
 
-// Visit v of a unit: query block qb = qb0 + v / G, query head g*G + v % G.
+// Visit v of a unit: query block qb = qb0 + v / Gs, query head
+// g*G + part*Gs + v % Gs, with Gs = G / split heads per part.
 __device__ __forceinline__ void bwd_visit(const BwdParams& p, const BwdUnit& w, int v, int& head,
                                           int& qb) {
-  qb = w.qb0 + v / p.G;
-  head = w.g * p.G + v % p.G;
+  const int gs = p.G / p.split;
+  qb = w.qb0 + v / gs;
+  head = w.g * p.G + w.part * gs + v % gs;
 }
 
 template <int D>
@@ -485,7 +536,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // unit's first barrier, where the others learn of it.
       if (!ok) continue;
 
-      // ---- unit epilogue: dV, scale * dK -> bf16 (this warp's D/2 columns) ----
+      // ---- unit epilogue: dV, scale * dK -> bf16, or fp32 partials when the
+      // unit is one of `split` parts (this warp's D/2 columns) ----------------
       ok = warp_wait(dkv_full, units & 1, kErrBwdDkv, p.launch_id);
       ++units;
       if (!ok) continue;
@@ -497,6 +549,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const uint32_t src = tmem + lane_base + (which == 0 ? C::DV_COL : C::DK_COL) + HC * half;
         const float mul = which == 0 ? 1.f : p.scale;
         uint4* out = reinterpret_cast<uint4*>((which == 0 ? p.dv : p.dk) + krow * D + HC * half);
+        if (p.split > 1) {
+          float4* part = reinterpret_cast<float4*>(
+              p.dkv_part +
+              ((static_cast<long long>(w.part) * p.B * p.Hkv * p.T + krow) * 2 + which) * D +
+              HC * half);
+#pragma unroll
+          for (int c = 0; c < HC / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(src + 32 * c, r);
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(r);
+            if (key_ok) {
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4)
+                part[c * 8 + v4] = make_float4(
+                    __uint_as_float(r[4 * v4]) * mul, __uint_as_float(r[4 * v4 + 1]) * mul,
+                    __uint_as_float(r[4 * v4 + 2]) * mul, __uint_as_float(r[4 * v4 + 3]) * mul);
+            }
+          }
+          continue;
+        }
 #pragma unroll
         for (int c = 0; c < HC / 32; ++c) {
           uint32_t r[32];

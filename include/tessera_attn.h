@@ -126,7 +126,11 @@ int tessera_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o
  * workspace        device memory of at least
  *                  tessera_attn_bwd_workspace_bytes(B, Hq, T, d) bytes
  *                  (B*Hq*T fp32: D), 16-byte aligned, owned by the caller;
- *                  overwritten (no contents need to be set before the call)
+ *                  overwritten (no contents need to be set before the call);
+ *                  workspace_bytes gives its size.  With at least
+ *                  tessera_attn_bwd_workspace_bytes_kv(B, Hq, Hkv, T, d)
+ *                  bytes, shapes with few key/value units also get the
+ *                  balanced form below.
  * other arguments  as in tessera_attn_fwd
  *
  * Checks as in tessera_attn_fwd, plus: every pointer non-NULL (lse too) and
@@ -136,8 +140,27 @@ int tessera_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o
  * as units), then dQ (query blocks as units, S and dP recomputed); no
  * atomics, so the result does not depend on scheduling.  Bounded waits as in
  * the forward.
+ *
+ * Balanced form (the pages have no counterpart; this is a scheduling choice
+ * of this library).  When B * Hkv * ceil(T/128) is under 512 (about four
+ * units per SM: multi-query attention, few batches) and the workspace holds
+ * them, the dK/dV units are cut by query heads into split = 2, 4 or 8 parts
+ * (G / split heads each); each part writes fp32 partial dK, dV into the
+ * workspace and a fourth kernel sums them in part order into bf16
+ * (tessera_attn_last_launch_count() = 4).  The split depends on the shape
+ * and the workspace size only, so the result still does not depend on
+ * scheduling; it differs from the three-kernel form only in the rounding of
+ * the dK/dV sums.
  */
 size_t tessera_attn_bwd_workspace_bytes(int B, int Hq, int T, int d);
+
+/*
+ * Workspace bytes with which tessera_attn_bwd uses its balanced form for this
+ * shape: tessera_attn_bwd_workspace_bytes(B, Hq, T, d) when the shape has
+ * enough key/value units, else D (256-byte aligned) followed by
+ * split * B * Hkv * T * d * 2 fp32 partials.  0 for invalid sizes.
+ */
+size_t tessera_attn_bwd_workspace_bytes_kv(int B, int Hq, int Hkv, int T, int d);
 int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
                      const float *lse, const void *dout, void *dq, void *dk, void *dv,
                      void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
@@ -153,7 +176,8 @@ int tessera_attn_bwd(const void *q, const void *k, const void *v, const void *o,
  * sets all it reads.  Arguments, checks and results are those of
  * tessera_attn_bwd; a problem whose workspace
  * (tessera_attn_bwd_workspace_bytes) exceeds the array returns
- * TESSERA_ERR_TOO_LARGE before any CUDA call.  Calls whose work overlaps in
+ * TESSERA_ERR_TOO_LARGE before any CUDA call.  The balanced form is used
+ * when tessera_attn_bwd_workspace_bytes_kv fits in the array.  Calls whose work overlaps in
  * time on one device (other streams or threads) share the array and race:
  * queue them on one stream.
  */

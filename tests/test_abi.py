@@ -121,6 +121,18 @@ def test_bwd_workspace_bytes(lib):
     assert tess.tessera_attn_bwd_workspace_bytes(2, 8, 100, 64) == 2 * 8 * 100 * 4
     assert tess.tessera_attn_bwd_workspace_bytes(1, 1, 1, 128) == 4
     assert tess.tessera_attn_bwd_workspace_bytes(1, 1, 1, 96) == 0
+    # the balanced dK/dV form: D (256-byte aligned) + split * B*Hkv*T*d*2 fp32
+    # when B*Hkv*ceil(T/128) < 512; split doubles while G allows, up to 8
+    assert tess.tessera_attn_bwd_workspace_bytes_kv(1, 8, 1, 1000, 128) == \
+        32000 + 8 * 1 * 1 * 1000 * 128 * 2 * 4
+    assert tess.tessera_attn_bwd_workspace_bytes_kv(2, 6, 3, 300, 64) == \
+        ((2 * 6 * 300 * 4 + 255) // 256) * 256 + 2 * 2 * 3 * 300 * 64 * 2 * 4
+    for shape in [(1, 32, 8, 16384, 128), (2, 8, 8, 100, 64), (8, 32, 32, 2048, 128)]:
+        B, Hq, Hkv, T, d = shape  # enough units, or G = 1: the three-kernel form
+        assert tess.tessera_attn_bwd_workspace_bytes_kv(*shape) == \
+            tess.tessera_attn_bwd_workspace_bytes(B, Hq, T, d)
+    assert tess.tessera_attn_bwd_workspace_bytes_kv(1, 3, 2, 10, 64) == 0
+    assert tess.tessera_attn_bwd_workspace_bytes_kv(1, 2, 1, 10, 96) == 0
 
 
 @pytest.mark.parametrize("kw,status", [
