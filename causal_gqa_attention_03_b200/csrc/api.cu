@@ -326,6 +326,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.split = split;
+  // batch-major dK/dV units when one batch alone has two units per CTA
+  p.kv_batch_major =
+      (B > 1 && static_cast<long long>(Hkv) * split * nqb >= 2LL * sms) ? 1 : 0;
   p.dkv_part = split > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
                                                     bwd_part_offset(B, Hq, T, D))
                          : nullptr;

@@ -179,11 +179,14 @@ struct BwdParams {
   // attn_bwd_dkv_reduce_kernel sums into dV, dK.
   int split;
   float* dkv_part;
+  // kernel 2: 1 = batch-major unit order (set when one batch has at least
+  // two units per CTA: its Q and dO then stay in L2 without costing balance)
+  int kv_batch_major;
 };
 
-// Unit u: key block kb = u / (B * Hkv * split) (ascending: the longest
-// causal extents first), batch, key/value head and query-head part from the
-// rest.
+// Unit u: key block kb (ascending: the longest causal extents first), then
+// batch, key/value head and query-head part; or batch first
+// (kv_batch_major).
 struct BwdUnit {
   int b, g, kb;
   int part;     // which G / split query heads of the group
@@ -193,13 +196,25 @@ struct BwdUnit {
 
 __device__ __forceinline__ BwdUnit decode_bwd_unit(const BwdParams& p, int u) {
   BwdUnit w;
-  const int groups = p.B * p.Hkv * p.split;
-  const int rest = u % groups;
-  w.kb = u / groups;
+  const int groups = p.Hkv * p.split;
+  int rest;
+  if (p.kv_batch_major) {
+    // batch b's units (key blocks ascending, each over its heads and parts)
+    // before batch b+1's, so one batch's Q and dO stay in L2
+    const int per_b = groups * p.nqb;
+    w.b = u / per_b;
+    const int ub = u % per_b;
+    rest = ub % groups;
+    w.kb = ub / groups;
+  } else {
+    // key blocks ascending over all batches
+    const int bgs = p.B * groups;
+    w.kb = u / bgs;
+    w.b = (u % bgs) / groups;
+    rest = u % groups;
+  }
   w.part = rest % p.split;
-  const int bg = rest / p.split;
-  w.b = bg / p.Hkv;
-  w.g = bg % p.Hkv;
+  w.g = rest / p.split;
   w.qb0 = p.causal ? w.kb : 0;
   w.nvisit = (p.G / p.split) * (p.nqb - w.qb0);
   return w;
