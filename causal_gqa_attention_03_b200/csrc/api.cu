@@ -329,6 +329,15 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   // batch-major dK/dV units when one batch alone has two units per CTA
   p.kv_batch_major =
       (B > 1 && static_cast<long long>(Hkv) * split * nqb >= 2LL * sms) ? 1 : 0;
+  // batch-major dQ units when one batch has two units per CTA and K/V
+  // (B * Hkv * T * d, both) does not fit in L2
+  int l2_bytes = 0;
+  if (cudaDeviceGetAttribute(&l2_bytes, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
+    return TESSERA_ERR_CUDA;
+  p.q_batch_major = (B > 1 && static_cast<long long>(Hq) * nqb >= 2LL * sms &&
+                     4.0 * B * Hkv * T * D > static_cast<double>(l2_bytes))
+                        ? 1
+                        : 0;
   p.dkv_part = split > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
                                                     bwd_part_offset(B, Hq, T, D))
                          : nullptr;

@@ -182,6 +182,9 @@ struct BwdParams {
   // kernel 2: 1 = batch-major unit order (set when one batch has at least
   // two units per CTA: its Q and dO then stay in L2 without costing balance)
   int kv_batch_major;
+  // kernel 3: 1 = batch-major unit order (set when one batch has at least
+  // two units per CTA and the whole K/V is larger than L2)
+  int q_batch_major;
 };
 
 // Unit u: key block kb (ascending: the longest causal extents first), then
@@ -687,10 +690,21 @@ struct DqUnit {
 
 __device__ __forceinline__ DqUnit decode_dq_unit(const BwdParams& p, int u) {
   DqUnit w;
-  const int bh = u % (p.B * p.Hq);
-  const int step = u / (p.B * p.Hq);
-  w.b = bh / p.Hq;
-  w.h = bh % p.Hq;
+  int step;
+  if (p.q_batch_major) {
+    // batch b's units (heaviest first) before batch b+1's: one batch's K and
+    // V stay in L2
+    const int per_b = p.Hq * p.nqb;
+    w.b = u / per_b;
+    const int ub = u % per_b;
+    step = ub / p.Hq;
+    w.h = ub % p.Hq;
+  } else {
+    const int bh = u % (p.B * p.Hq);
+    step = u / (p.B * p.Hq);
+    w.b = bh / p.Hq;
+    w.h = bh % p.Hq;
+  }
   w.qb = p.nqb - 1 - step;
   w.n = p.causal ? w.qb + 1 : p.nqb;
   return w;
