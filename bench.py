@@ -646,8 +646,8 @@ def varlen_line(wv, times, launches, peaks, peak_src):
 
 def time_e2e(w, q_h, k_h, v_h, steps, warmup, stream, tess, torch, dev):
     """Public API end to end: pinned host Q/K/V in, pinned host O/LSE out, through
-    tessera_attn_fwd_host (copies pipelined with the kernels over chunks of
-    query heads).  Each step returns with the outputs on the host."""
+    tessera_attn_fwd_host (copies pipelined with the kernels over pieces of
+    query heads, the library's default plan).  Each step returns with the outputs on the host."""
     staging = {"q": torch.empty(q_h.shape, dtype=torch.bfloat16, device=dev),
                "k": torch.empty(k_h.shape, dtype=torch.bfloat16, device=dev),
                "v": torch.empty(k_h.shape, dtype=torch.bfloat16, device=dev),
@@ -879,9 +879,11 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per chunk of query heads "
-                        "(16 by default: H2D copy, kernel, D2H copy; copies overlap kernels) "
-                        "-> pinned host O/LSE"},
+                "path": "tessera_attn_fwd_host: pinned host Q/K/V -> per piece of query heads "
+                        "(default plan: 8 even pieces, the last cut down to one-head pieces; "
+                        "H2D copy, kernel on one of four streams, D2H copy; copies overlap "
+                        "kernels) -> pinned host O/LSE",
+                "pieces": len(tess.tessera_attn_fwd_host_plan(w.B, w.Hq, w.Hkv, 0))},
         "gpu_launches": launches,
         "backward": backward_line(w, bwd_times, bwd_max_ms, bwd_steps, bwd_launches, bwd_ws,
                                   world, peaks, peak_src),

@@ -6,7 +6,8 @@ built in this directory (``python -m causal_gqa_attention_03_b200.build``).
 There is no fallback: if the library is missing, every call raises.
 
 Raw C-ABI names (integer pointers, sizes, stream handle):
-    tessera_attn_fwd, tessera_attn_fwd_host, tessera_attn_device_error,
+    tessera_attn_fwd, tessera_attn_fwd_host, tessera_attn_fwd_host_plan,
+    tessera_attn_device_error,
     tessera_status_str, tessera_attn_last_launch_count,
     tessera_attn_selftest_timeout, tessera_attn_bwd, tessera_attn_bwd_workspace_bytes,
     tessera_attn_bwd_workspace_bytes_kv,
@@ -35,7 +36,8 @@ import threading
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtessera_attn.so")
 
 # Symbols declared in include/tessera_attn.h.
-EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_bwd",
+EXPORTED = ("tessera_attn_fwd", "tessera_attn_fwd_host", "tessera_attn_fwd_host_plan",
+            "tessera_attn_bwd",
             "tessera_attn_bwd_workspace_bytes", "tessera_attn_bwd_workspace_bytes_kv",
             "tessera_attn_bwd_noalloc",
             "tessera_attn_bwd_noalloc_max_workspace_bytes", "tessera_attn_device_error",
@@ -83,6 +85,8 @@ def load_library() -> ctypes.CDLL:
             lib.tessera_attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci,
                                                   ci, ci, ci, ci, ctypes.c_float, ci, vp]
             lib.tessera_attn_fwd_host.restype = ci
+            lib.tessera_attn_fwd_host_plan.argtypes = [ci, ci, ci, ci, ctypes.POINTER(ci), ci]
+            lib.tessera_attn_fwd_host_plan.restype = ci
             lib.tessera_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                              ctypes.c_size_t, ci, ci, ci, ci, ci, ci,
                                              ctypes.c_float, vp]
@@ -137,6 +141,20 @@ def tessera_attn_fwd_host(q_h: int, k_h: int, v_h: int, o_h: int, lse_h: int | N
     return load_library().tessera_attn_fwd_host(
         q_h, k_h, v_h, o_h, lse_h or None, q_d, k_d, v_d, o_d, lse_d or None, B, Hq, Hkv, T, d,
         int(causal), float(scale), int(chunks), stream or None)
+
+
+def tessera_attn_fwd_host_plan(B: int, Hq: int, Hkv: int, chunks: int) -> list:
+    """The pieces (s0, s1, h0, h1) tessera_attn_fwd_host cuts a problem into.
+
+    Host only (no CUDA call); raises TesseraError on invalid sizes.
+    """
+    lib = load_library()
+    n = lib.tessera_attn_fwd_host_plan(B, Hq, Hkv, chunks, None, 0)
+    if n < 0:
+        raise TesseraError(-n, "tessera_attn_fwd_host_plan")
+    buf = (ctypes.c_int * (4 * max(n, 1)))()
+    lib.tessera_attn_fwd_host_plan(B, Hq, Hkv, chunks, buf, n)
+    return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
 
 
 def tessera_attn_bwd(q: int, k: int, v: int, o: int, lse: int, dout: int, dq: int, dk: int,

@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "tessera_attn.h"
 #include "attn_fwd_sm100.cuh"
@@ -195,9 +196,14 @@ int launch_d(int d, const void* q, const void* k, const void* v, void* o, float*
 
 // Streams and events of the host-buffer pipeline, created on first use per
 // device and kept for the life of the process.
+// The pieces' kernels go round-robin over kPipeKernelStreams streams, so a
+// piece whose inputs have arrived starts on the SMs that the previous piece's
+// last (heaviest) units leave idle instead of waiting for that kernel to end.
+constexpr int kPipeKernelStreams = 4;
 struct HostPipe {
   bool ready = false;
   cudaStream_t in = nullptr, out = nullptr;
+  cudaStream_t run[kPipeKernelStreams] = {};
   cudaEvent_t start = nullptr, in_done = nullptr, k_done = nullptr, out_done = nullptr;
 };
 std::mutex g_pipe_mu;
@@ -214,6 +220,10 @@ void host_pipe_reset(HostPipe& h) {
     if (*s != nullptr) cudaStreamDestroy(*s);
     *s = nullptr;
   }
+  for (cudaStream_t& s : h.run) {
+    if (s != nullptr) cudaStreamDestroy(s);
+    s = nullptr;
+  }
   h.ready = false;
 }
 
@@ -222,6 +232,8 @@ HostPipe* host_pipe(int dev) {
   if (h.ready) return &h;
   bool ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess;
+  for (cudaStream_t& s : h.run)
+    ok = ok && cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess;
   for (cudaEvent_t* e : {&h.start, &h.in_done, &h.k_done, &h.out_done})
     ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
@@ -665,6 +677,77 @@ extern "C" int tessera_attn_fwd_varlen(const void* q, const void* k, const void*
   return launch<128>(q, k, v, o, lse, B, Hq, Hkv, max_seqlen, causal, scale, s, cu, total);
 }
 
+// One piece of the host-buffer pipeline: whole slices [s0, s1) (h0 = 0,
+// h1 = G), or query heads [h0, h1) of the one slice s0 (s1 = s0 + 1).
+struct HostPiece {
+  int s0, s1, h0, h1;
+};
+
+// `target` pieces: contiguous ranges of whole slices while target <= slices;
+// otherwise every slice cut into `split` runs of G/split query heads (split
+// the smallest divisor of G that is at least ceil(target / slices), else G).
+void plan_even(int slices, int G, int target, std::vector<HostPiece>& out) {
+  if (target <= slices) {
+    for (int c = 0; c < target; ++c) {
+      const int s0 = static_cast<int>(static_cast<long long>(slices) * c / target);
+      const int s1 = static_cast<int>(static_cast<long long>(slices) * (c + 1) / target);
+      if (s1 > s0) out.push_back({s0, s1, 0, G});
+    }
+    return;
+  }
+  const int want = (target + slices - 1) / slices;
+  int split = G;
+  for (int s_ = want; s_ < G; ++s_)
+    if (G % s_ == 0) {
+      split = s_;
+      break;
+    }
+  for (int sl = 0; sl < slices; ++sl)
+    for (int r = 0; r < split; ++r)
+      out.push_back({sl, sl + 1, r * (G / split), (r + 1) * (G / split)});
+}
+
+// The pieces of tessera_attn_fwd_host, in queue order.  chunks > 0: the even
+// plan above.  chunks == 0: the even plan for 8 pieces with its last piece
+// tapered: its whole slices but the last stay one piece, and the last slice's
+// final min(G, 4) query heads become one piece each (the rest of that slice
+// one piece before them).  The pipeline ends with the last piece's kernel and
+// download, so one-head last pieces shorten that drain.
+std::vector<HostPiece> plan_host_pieces(int slices, int G, int chunks) {
+  std::vector<HostPiece> out;
+  plan_even(slices, G, chunks > 0 ? chunks : 8, out);
+  if (chunks > 0 || out.empty()) return out;
+  const HostPiece last = out.back();
+  out.pop_back();
+  const int sl = last.s1 - 1;
+  if (last.s1 - last.s0 > 1) out.push_back({last.s0, sl, 0, G});
+  const int tail = (last.h1 - last.h0) < 4 ? (last.h1 - last.h0) : 4;
+  if (last.h1 - tail > last.h0) out.push_back({sl, sl + 1, last.h0, last.h1 - tail});
+  for (int h = last.h1 - tail; h < last.h1; ++h) out.push_back({sl, sl + 1, h, h + 1});
+  return out;
+}
+
+extern "C" int tessera_attn_fwd_host_plan(int B, int Hq, int Hkv, int chunks, int* pieces,
+                                          int max_pieces) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || chunks < 0 || max_pieces < 0 ||
+      (max_pieces > 0 && pieces == nullptr) || static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return -TESSERA_ERR_INVALID_ARG;
+  std::vector<HostPiece> plan;
+  try {
+    plan = plan_host_pieces(static_cast<int>(static_cast<long long>(B) * Hkv), Hq / Hkv, chunks);
+  } catch (...) {
+    return -TESSERA_ERR_INVALID_ARG;
+  }
+  const int n = static_cast<int>(plan.size());
+  for (int i = 0; i < n && i < max_pieces; ++i) {
+    pieces[4 * i + 0] = plan[i].s0;
+    pieces[4 * i + 1] = plan[i].s1;
+    pieces[4 * i + 2] = plan[i].h0;
+    pieces[4 * i + 3] = plan[i].h1;
+  }
+  return n;
+}
+
 extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
                                      float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d,
                                      float* lse_d, int B, int Hq, int Hkv, int T, int d,
@@ -677,27 +760,15 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
   if ((lse_h == nullptr) != (lse_d == nullptr) || chunks < 0) return TESSERA_ERR_INVALID_ARG;
   if (empty) return TESSERA_OK;
   if (!q_h || !k_h || !v_h || !o_h) return TESSERA_ERR_INVALID_ARG;
-  // Chunks are contiguous ranges of the B*Hkv (batch, key/value head) slices,
-  // each one launch over a [1, n*G, T, d] view of the buffers; or, when more
-  // chunks than slices are asked for, each slice is cut into `split` runs of
-  // G/split query heads (split divides G), one launch each over a
-  // [1, G/split, T, d] view with that slice's K/V, uploaded with its first
-  // run.  Smaller pieces shorten the pipeline's fill (the first upload) and
-  // drain (the last kernel and download).
   const int slices = static_cast<int>(static_cast<long long>(B) * Hkv);
   const int G = Hq / Hkv;
-  const int target = chunks == 0 ? 16 : chunks;
-  int split = 1;
-  if (target > slices) {
-    const int want = (target + slices - 1) / slices;
-    split = G;
-    for (int s_ = want; s_ < G; ++s_)
-      if (G % s_ == 0) {
-        split = s_;
-        break;
-      }
+  std::vector<HostPiece> pieces;
+  try {
+    pieces = plan_host_pieces(slices, G, chunks);
+  } catch (...) {  // no host memory for the plan (one entry per piece, at most B*Hq)
+    return TESSERA_ERR_INVALID_ARG;
   }
-  const int n_chunks = split > 1 ? slices * split : (target < slices ? target : slices);
+  const int n_pieces = static_cast<int>(pieces.size());
   const size_t kv_slice = static_cast<size_t>(T) * d * 2;   // bytes of one K (or V) head
   const size_t q_head = kv_slice;                           // bytes of one Q (or O) head
   const size_t lse_head = static_cast<size_t>(T) * 4;       // bytes of one head's LSE rows
@@ -716,22 +787,9 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
   const auto c8 = [](const void* p, size_t off) { return static_cast<const char*>(p) + off; };
   const auto m8 = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
   int launches = 0;
-  for (int c = 0; c < n_chunks; ++c) {
-    // this chunk: slices [s0, s1) (whole groups) or query heads [h0, h1) of slice s0
-    int s0, s1, h0, h1;
-    if (split > 1) {
-      s0 = c / split;
-      s1 = s0 + 1;
-      h0 = (c % split) * (G / split);
-      h1 = h0 + G / split;
-    } else {
-      s0 = static_cast<int>(static_cast<long long>(slices) * c / n_chunks);
-      s1 = static_cast<int>(static_cast<long long>(slices) * (c + 1) / n_chunks);
-      h0 = 0;
-      h1 = G;
-    }
+  for (int c = 0; c < n_pieces; ++c) {
+    const int s0 = pieces[c].s0, s1 = pieces[c].s1, h0 = pieces[c].h0, h1 = pieces[c].h1;
     const int n = s1 - s0;
-    if (n == 0) continue;
     const bool whole = (h0 == 0 && h1 == G);
     const int nq = whole ? n * G : h1 - h0;  // query heads of the launch
     const size_t qo = q_head * (static_cast<size_t>(s0) * G + h0);
@@ -743,17 +801,18 @@ extern "C" int tessera_attn_fwd_host(const void* q_h, const void* k_h, const voi
          cudaMemcpyAsync(m8(v_d, ko), c8(v_h, ko), kv_slice * n, cudaMemcpyHostToDevice, hp->in) !=
              cudaSuccess))
       return TESSERA_ERR_CUDA;
+    cudaStream_t run = hp->run[launches % kPipeKernelStreams];
     if (cudaMemcpyAsync(m8(q_d, qo), c8(q_h, qo), q_head * nq, cudaMemcpyHostToDevice, hp->in) !=
             cudaSuccess ||
         cudaEventRecord(hp->in_done, hp->in) != cudaSuccess ||
-        cudaStreamWaitEvent(s, hp->in_done, 0) != cudaSuccess)
+        cudaStreamWaitEvent(run, hp->in_done, 0) != cudaSuccess)
       return TESSERA_ERR_CUDA;
     const int lst = launch_d(d, m8(q_d, qo), m8(k_d, ko), m8(v_d, ko), m8(o_d, qo),
                              lse_d ? reinterpret_cast<float*>(m8(lse_d, lo)) : nullptr, 1, nq, n,
-                             T, causal, scale, s);
+                             T, causal, scale, run);
     if (lst != TESSERA_OK) return lst;
     ++launches;
-    if (cudaEventRecord(hp->k_done, s) != cudaSuccess ||
+    if (cudaEventRecord(hp->k_done, run) != cudaSuccess ||
         cudaStreamWaitEvent(hp->out, hp->k_done, 0) != cudaSuccess ||
         cudaMemcpyAsync(m8(o_h, qo), c8(o_d, qo), q_head * nq, cudaMemcpyDeviceToHost, hp->out) !=
             cudaSuccess)

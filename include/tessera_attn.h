@@ -190,15 +190,23 @@ int tessera_attn_bwd_noalloc(const void *q, const void *k, const void *v, const 
 /*
  * The same operation on host buffers, pipelined over the host link.  (The
  * pages describe the kernel only; this transfer pipeline is this library's.)
- * The B*Hkv (batch, key/value head) slices are cut into `chunks` contiguous
- * ranges, or, when `chunks` exceeds B*Hkv, each slice is cut into `split`
- * runs of G/split query heads (split = the smallest divisor of G that is at
- * least ceil(chunks / (B*Hkv)), else G; the slice's K/V go with its first
- * run).  For each piece Q (and K/V) are copied host -> device, the kernel of
- * tessera_attn_fwd runs on it, and O/LSE are copied device -> host.  Copies
- * run on two streams the library creates per device on first use (kept for
- * the life of the process), so one range's copies overlap the others' kernels
- * and copies; the kernels run on `stream`.
+ * The problem is cut into pieces along the B*Hkv (batch, key/value head)
+ * slices: a piece is a range of whole slices, or a run of query heads of one
+ * slice (the slice's K/V go with its first run).  With `chunks` > 0 the plan
+ * is even: `chunks` contiguous ranges of whole slices, or, when `chunks`
+ * exceeds B*Hkv, every slice cut into `split` runs of G/split query heads
+ * (split = the smallest divisor of G that is at least ceil(chunks / (B*Hkv)),
+ * else G).  With `chunks` = 0 the plan is the even one for 8 with its last
+ * piece tapered: that piece's whole slices but the last stay one piece, and
+ * the last slice's final min(G', 4) query heads (G' the heads of that piece
+ * within the slice) become one piece each, the rest of them one piece before.
+ * tessera_attn_fwd_host_plan lists the pieces.  For each piece Q (and K/V)
+ * are copied host -> device, the kernel of tessera_attn_fwd runs on it, and
+ * O/LSE are copied device -> host.  Copies run on two streams and the kernels
+ * round-robin on four more that the library creates per device on first use
+ * (kept for the life of the process), so one piece's copies overlap the
+ * others' kernels and copies, and a piece's kernel starts on the SMs the
+ * previous piece's last units leave idle.
  *
  * q_h, k_h, v_h  host inputs, layouts as in tessera_attn_fwd.  Page-locked
  *                memory (cudaHostAlloc / cudaHostRegister) lets the copies
@@ -206,21 +214,34 @@ int tessera_attn_bwd_noalloc(const void *q, const void *k, const void *v, const 
  * o_h, lse_h     host outputs; lse_h may be NULL (then lse_d must be NULL).
  * q_d .. lse_d   device buffers of the full sizes, owned by the caller, with
  *                the rules of tessera_attn_fwd; they also hold the results.
- * chunks         0: the library's choice (16, as above); 1..B*Hkv: that many
- *                ranges of whole slices; more: slices cut by query heads.
- *                Every choice gives the same bits as one tessera_attn_fwd.
+ * chunks         0: the tapered plan; > 0: the even plan, as above.  Every
+ *                plan gives the same bits as one tessera_attn_fwd.
  * stream         the host outputs are complete once the work queued on
  *                `stream` before the call returns has finished plus this
  *                call's work: synchronise `stream` before reading them.
  *
  * Arguments are checked as in tessera_attn_fwd (plus non-NULL host pointers
  * and chunks >= 0) before any CUDA call.  Calls are serialised by a mutex.
- * tessera_attn_last_launch_count() then reports the number of launches.
+ * tessera_attn_last_launch_count() then reports the number of launches (one
+ * per piece).
  */
 int tessera_attn_fwd_host(const void *q_h, const void *k_h, const void *v_h, void *o_h,
                           float *lse_h, void *q_d, void *k_d, void *v_d, void *o_d,
                           float *lse_d, int B, int Hq, int Hkv, int T, int d, int causal,
                           float scale, int chunks, tessera_stream_t stream);
+
+/*
+ * The pieces tessera_attn_fwd_host cuts a [B, Hq | Hkv, T, d] problem into for
+ * `chunks`, in queue order.  Host only: no CUDA call.  Writes min(count,
+ * max_pieces) entries of four ints to `pieces`: s0, s1, h0, h1, meaning
+ * slices [s0, s1) whole (h0 = 0, h1 = G) or query heads [h0, h1) of slice s0
+ * (s1 = s0 + 1), a slice being one (batch, key/value head) pair in batch-major
+ * order.  `pieces` may be NULL when max_pieces is 0.  Returns the count, or
+ * -TESSERA_ERR_INVALID_ARG for B, Hq, Hkv < 1, Hq % Hkv != 0, chunks < 0,
+ * max_pieces < 0, or a NULL `pieces` with max_pieces > 0.
+ */
+int tessera_attn_fwd_host_plan(int B, int Hq, int Hkv, int chunks, int *pieces,
+                               int max_pieces);
 
 /*
  * One decoding step over a block-paged key/value cache.  The pages list a

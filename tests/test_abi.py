@@ -105,6 +105,55 @@ def test_host_entry_argument_checks_before_any_cuda_call(lib, kw, status):
     assert tess.tessera_attn_last_launch_count() == 0
 
 
+def plan_by_header_rule(B, Hq, Hkv, chunks):
+    """The pieces of tessera_attn_fwd_host as its header states the rule."""
+    slices, G = B * Hkv, Hq // Hkv
+    target = chunks if chunks > 0 else 8
+    if target <= slices:
+        cuts = [slices * c // target for c in range(target + 1)]
+        out = [(a, b, 0, G) for a, b in zip(cuts, cuts[1:]) if b > a]
+    else:
+        want = -(-target // slices)
+        split = next((s for s in range(want, G) if G % s == 0), G)
+        r = G // split
+        out = [(sl, sl + 1, i * r, (i + 1) * r) for sl in range(slices) for i in range(split)]
+    if chunks > 0:
+        return out
+    s0, s1, h0, h1 = out.pop()
+    if s1 - s0 > 1:
+        out.append((s0, s1 - 1, 0, G))
+    tail = min(h1 - h0, 4)
+    if h1 - tail > h0:
+        out.append((s1 - 1, s1, h0, h1 - tail))
+    return out + [(s1 - 1, s1, h, h + 1) for h in range(h1 - tail, h1)]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv", [(1, 32, 8), (1, 32, 1), (1, 32, 32), (4, 4, 4), (1, 2, 1),
+                                      (3, 12, 4), (2, 6, 3), (64, 8, 8)])
+@pytest.mark.parametrize("chunks", [0, 1, 3, 8, 40, 1000])
+def test_host_plan_follows_the_rule_and_covers_every_head_once(lib, B, Hq, Hkv, chunks):
+    plan = tess.tessera_attn_fwd_host_plan(B, Hq, Hkv, chunks)
+    assert plan == plan_by_header_rule(B, Hq, Hkv, chunks)
+    G = Hq // Hkv
+    heads = []
+    for s0, s1, h0, h1 in plan:
+        assert (h0, h1) == (0, G) or (s1 == s0 + 1 and 0 <= h0 < h1 <= G)
+        heads += [sl * G + h for sl in range(s0, s1) for h in range(h0, h1)]
+    assert heads == list(range(B * Hq))
+
+
+def test_host_plan_headline_shape_tapers_to_single_heads(lib):
+    # [1, 32 | 8, T, d]: seven one-slice pieces, then the last slice head by head
+    plan = tess.tessera_attn_fwd_host_plan(1, 32, 8, 0)
+    assert plan == [(s, s + 1, 0, 4) for s in range(7)] + [(7, 8, h, h + 1) for h in range(4)]
+
+
+@pytest.mark.parametrize("args", [(0, 8, 8, 0), (1, 8, 3, 0), (1, 8, 8, -1), (1, 0, 1, 0)])
+def test_host_plan_rejects_bad_sizes(lib, args):
+    n = lib.tessera_attn_fwd_host_plan(*args, None, 0)
+    assert n == -1
+
+
 def call_bwd(**kw):
     a = dict(GOOD, dout=ALIGNED + 0x5000000, dq=ALIGNED + 0x6000000, dk=ALIGNED + 0x7000000,
              dv=ALIGNED + 0x8000000, ws=ALIGNED + 0x9000000, ws_bytes=None)

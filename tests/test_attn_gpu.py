@@ -288,17 +288,6 @@ def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
     check(o.numpy(), lse.numpy(), ro, rlse, "after self-test")
 
 
-def host_launches(B, Hq, Hkv, chunks):
-    """Launches tessera_attn_fwd_host makes, by the rule in its header."""
-    slices, G = B * Hkv, Hq // Hkv
-    target = 16 if chunks == 0 else chunks
-    if target <= slices:
-        return target
-    want = -(-target // slices)
-    split = next((s for s in range(want, G) if G % s == 0), G)
-    return slices * split if split > 1 else slices
-
-
 @pytest.mark.parametrize("B,Hq,Hkv,T,d,causal,chunks", [
     (1, 32, 8, 1000, 128, True, 0), (2, 6, 3, 129, 64, True, 4), (3, 4, 2, 77, 128, True, 1),
     (2, 8, 2, 300, 64, False, 100), (1, 2, 1, 1, 64, True, 0),
@@ -310,7 +299,7 @@ def test_host_pipeline_matches_device_call_bitwise(B, Hq, Hkv, T, d, causal, chu
     o_ref, lse_ref = run_gpu(q, k, v, causal, scale)
     qp, kp, vp = q.pin_memory(), k.pin_memory(), v.pin_memory()
     o_h, lse_h = tess.attn_fwd_host(qp, kp, vp, causal=causal, scale=scale, chunks=chunks)
-    assert tess.tessera_attn_last_launch_count() == host_launches(B, Hq, Hkv, chunks)
+    assert tess.tessera_attn_last_launch_count() == len(tess.tessera_attn_fwd_host_plan(B, Hq, Hkv, chunks))
     assert tess.tessera_attn_device_error() == 0
     assert torch.equal(o_h.float(), o_ref) and torch.equal(lse_h, lse_ref)
 
