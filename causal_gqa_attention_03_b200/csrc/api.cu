@@ -102,14 +102,19 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   if (cudaGetDevice(&dev) != cudaSuccess) return TESSERA_ERR_CUDA;
   static std::atomic<int> sm_count[64];
   if (dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
+  static std::atomic<long long> l2_size[64];
   int sms = sm_count[dev].load(std::memory_order_acquire);
+  long long l2_bytes = l2_size[dev].load(std::memory_order_acquire);
   if (sms == 0) {
+    int l2 = 0;
     if (cudaFuncSetAttribute(tessera::attn_fwd_sm100_kernel<D>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        sms <= 0)
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || sms <= 0)
       return TESSERA_ERR_CUDA;
+    l2_bytes = l2;
+    l2_size[dev].store(l2_bytes, std::memory_order_release);
     sm_count[dev].store(sms, std::memory_order_release);
   }
 
@@ -143,6 +148,30 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
   if (units > 0x7fffffffLL) return TESSERA_ERR_INVALID_ARG;
   p.num_units = static_cast<int>(units);
+  // Positions r of one step: consecutive ones share a (batch, K/V head) slice.
+  const int r_per_slice = p.pair_heads ? p.G / 2 : p.G;
+  const int nsteps = static_cast<int>(units / p.units_per_step);
+  p.r_group = p.units_per_step;
+  if (cu_seqlens != nullptr) {
+    p.r_group = p.units_per_step / B;  // one sequence per group
+  } else {
+    // When the whole K/V exceeds L2, walk groups of slices whose K/V fits in
+    // half of it, each with at least two units per CTA, sizes evened out.
+    const long long slice_bytes = 2LL * T * D * 2;
+    const long long slices = static_cast<long long>(B) * Hkv;
+    if (slices * slice_bytes > l2_bytes) {
+      long long per = (l2_bytes / 2) / slice_bytes;
+      const long long min_per = (2LL * sms + static_cast<long long>(r_per_slice) * nsteps - 1) /
+                                (static_cast<long long>(r_per_slice) * nsteps);
+      if (per < min_per) per = min_per;
+      if (per < 1) per = 1;
+      if (per < slices) {
+        const long long groups = (slices + per - 1) / per;
+        per = (slices + groups - 1) / groups;
+        p.r_group = static_cast<int>(per * r_per_slice);
+      }
+    }
+  }
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);

@@ -114,6 +114,7 @@ struct FwdParams {
   int nqb;                   // ceil(T / 128)
   int pair_heads;            // 1: tiles are heads (2p, 2p+1) of a group; 0: q-blocks (2p, 2p+1)
   int units_per_step;        // units sharing one position in the heaviest-first order
+  int r_group;               // positions r of a step walked together (units_per_step: all)
   int num_units;
   __nv_bfloat16* o;
   float* lse;
@@ -139,16 +140,19 @@ struct Unit {
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit w;
   int step, r;
-  if (p.cu_seqlens != nullptr) {
-    // Packed sequences: sequence-major (all of sequence 0's units, heaviest
-    // first, then sequence 1's, ...), so the CTAs work on about one
-    // sequence's keys and values at a time and those stay in L2.
-    const int per_seq_step = p.units_per_step / p.B;
-    const int per_seq = per_seq_step * (p.pair_heads ? p.nqb : (p.nqb + 1) >> 1);
-    const int b = u / per_seq;
-    const int rest = u % per_seq;
-    step = rest / per_seq_step;
-    r = b * per_seq_step + rest % per_seq_step;
+  if (p.r_group < p.units_per_step) {
+    // Grouped: the units of positions r in [0, r_group), heaviest first, then
+    // those of [r_group, 2 r_group), ...  Consecutive positions share a
+    // (batch, key/value head) slice, so the CTAs work on one group's keys and
+    // values at a time and those stay in L2: one sequence of a packed batch,
+    // or as many slices as half of L2 holds when the whole K/V does not fit.
+    const int nsteps = p.num_units / p.units_per_step;
+    const int per_group = p.r_group * nsteps;
+    const int gi = u / per_group;
+    const int rest = u % per_group;
+    const int rg = min(p.r_group, p.units_per_step - gi * p.r_group);
+    step = rest / rg;
+    r = gi * p.r_group + rest % rg;
   } else {
     step = u / p.units_per_step;
     r = u % p.units_per_step;
