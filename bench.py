@@ -776,7 +776,7 @@ def main():
     if err != 0:
         raise SystemExit(f"device-side error in the decode step (code {err})")
 
-    # the same serving batch at head dimension 64 (CUDA-core decode kernel)
+    # the same serving batch at head dimension 64
     wd64 = inputs.DECODE_D64
     d64_times, d64_launches, d64_ws, d64_flushed = time_decode(
         wd64, dec_steps, 3, flush, stream, tess, torch, dev, sample_key="decode_d64")

@@ -567,52 +567,17 @@ int check_decode_args(const void* q, const void* k_cache, const void* v_cache,
   return TESSERA_OK;
 }
 
+// The tensor-core kernel, GT = the largest power of two up to 16 dividing the
+// G query heads of a group: query heads per item.
 template <int D, int GT>
-int launch_decode(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
-                  cudaStream_t stream) {
-  using C = tessera::DecodeCfg<D, GT>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
-  static std::atomic<int> attr_set[64];
-  if (attr_set[dev].load(std::memory_order_acquire) == 0) {
-    if (cudaFuncSetAttribute(tessera::paged_decode_partial_kernel<D, GT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-      return TESSERA_ERR_CUDA;
-    attr_set[dev].store(1, std::memory_order_release);
-  }
-  int launches = 0;
-  if (p.nslot > 0) {
-    const long long rows = static_cast<long long>(p.num_blocks) * p.Hkv * p.bs;
-    CUtensorMap tm_k, tm_v;
-    if (!make_cache_map(&tm_k, k_cache, rows, D, p.rows_per_box) ||
-        !make_cache_map(&tm_v, v_cache, rows, D, p.rows_per_box))
-      return TESSERA_ERR_CUDA;
-    const int sms = sm_count(dev);
-    if (sms <= 0) return TESSERA_ERR_CUDA;
-    const unsigned grid = static_cast<unsigned>(sms);  // persistent: one CTA per SM
-    tessera::paged_decode_partial_kernel<D, GT>
-        <<<grid, tessera::kDecodeThreads, C::SMEM, stream>>>(tm_k, tm_v, p);
-    if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-    ++launches;
-  }
-  const long long warps = static_cast<long long>(p.B) * p.Hq;  // one merge CTA each
-  tessera::paged_decode_merge_kernel<D><<<static_cast<unsigned>(warps), 256, 0, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
-  g_last_launches = launches + 1;
-  return TESSERA_OK;
-}
-
-// Head dimension 128: the tensor-core kernel, GT = the largest power of two
-// up to 16 dividing G query heads per item.
-template <int GT>
 int launch_decode_tc(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
                      cudaStream_t stream) {
-  using C = tessera::DecTcCfg;
+  using C = tessera::DecTcCfg<D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TESSERA_ERR_CUDA;
   static std::atomic<int> attr_set[64];
   if (attr_set[dev].load(std::memory_order_acquire) == 0) {
-    if (cudaFuncSetAttribute(tessera::paged_decode_tc_kernel<GT>,
+    if (cudaFuncSetAttribute(tessera::paged_decode_tc_kernel<D, GT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
       return TESSERA_ERR_CUDA;
     attr_set[dev].store(1, std::memory_order_release);
@@ -622,42 +587,35 @@ int launch_decode_tc(const void* k_cache, const void* v_cache, tessera::DecodePa
   if (p.nslot > 0) {
     const long long rows = static_cast<long long>(p.num_blocks) * p.Hkv * p.bs;
     CUtensorMap tm_k, tm_v, tm_q;
-    if (!make_cache_map_atoms(&tm_k, k_cache, rows, p.rows_per_box) ||
-        !make_cache_map_atoms(&tm_v, v_cache, rows, p.rows_per_box) ||
-        !make_cache_map(&tm_q, p.q, static_cast<long long>(p.B) * p.Hq, 128, GT))
+    const bool kv_ok = D == 128 ? make_cache_map_atoms(&tm_k, k_cache, rows, p.rows_per_box) &&
+                                      make_cache_map_atoms(&tm_v, v_cache, rows, p.rows_per_box)
+                                : make_cache_map(&tm_k, k_cache, rows, D, p.rows_per_box) &&
+                                      make_cache_map(&tm_v, v_cache, rows, D, p.rows_per_box);
+    if (!kv_ok || !make_cache_map(&tm_q, p.q, static_cast<long long>(p.B) * p.Hq, D, GT))
       return TESSERA_ERR_CUDA;
     const int sms = sm_count(dev);
     if (sms <= 0) return TESSERA_ERR_CUDA;
-    tessera::paged_decode_tc_kernel<GT><<<static_cast<unsigned>(sms), tessera::kDecTcThreads,
-                                          C::SMEM, stream>>>(tm_k, tm_v, tm_q, p);
+    tessera::paged_decode_tc_kernel<D, GT><<<static_cast<unsigned>(sms), tessera::kDecTcThreads,
+                                             C::SMEM, stream>>>(tm_k, tm_v, tm_q, p);
     if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
     ++launches;
   }
   const long long heads = static_cast<long long>(p.B) * p.Hq;  // one merge CTA each
-  tessera::paged_decode_merge_kernel<128><<<static_cast<unsigned>(heads), 256, 0, stream>>>(p);
+  tessera::paged_decode_merge_kernel<D><<<static_cast<unsigned>(heads), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return TESSERA_ERR_CUDA;
   g_last_launches = launches + 1;
   return TESSERA_OK;
 }
 
 template <int D>
-int launch_decode_d(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
-                    cudaStream_t stream) {
+int launch_decode_tc_d(const void* k_cache, const void* v_cache, tessera::DecodeParams& p,
+                       cudaStream_t stream) {
   const int G = p.G;
-  if (G % 8 == 0) {
-    p.zgroups = G / 8;
-    return launch_decode<D, 8>(k_cache, v_cache, p, stream);
-  }
-  if (G % 4 == 0) {
-    p.zgroups = G / 4;
-    return launch_decode<D, 4>(k_cache, v_cache, p, stream);
-  }
-  if (G % 2 == 0) {
-    p.zgroups = G / 2;
-    return launch_decode<D, 2>(k_cache, v_cache, p, stream);
-  }
-  p.zgroups = G;
-  return launch_decode<D, 1>(k_cache, v_cache, p, stream);
+  if (G % 16 == 0) return launch_decode_tc<D, 16>(k_cache, v_cache, p, stream);
+  if (G % 8 == 0) return launch_decode_tc<D, 8>(k_cache, v_cache, p, stream);
+  if (G % 4 == 0) return launch_decode_tc<D, 4>(k_cache, v_cache, p, stream);
+  if (G % 2 == 0) return launch_decode_tc<D, 2>(k_cache, v_cache, p, stream);
+  return launch_decode_tc<D, 1>(k_cache, v_cache, p, stream);
 }
 
 }  // namespace
@@ -953,13 +911,8 @@ extern "C" int tessera_attn_decode(const void* q, const void* k_cache, const voi
   p.slots = ws ? reinterpret_cast<int*>(ws + heads_slots * (d + 2)) : nullptr;
   p.launch_id = g_launch_counter.fetch_add(1, std::memory_order_relaxed);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_decode_d<64>(k_cache, v_cache, p, s);
-  const int G = p.G;
-  if (G % 16 == 0) return launch_decode_tc<16>(k_cache, v_cache, p, s);
-  if (G % 8 == 0) return launch_decode_tc<8>(k_cache, v_cache, p, s);
-  if (G % 4 == 0) return launch_decode_tc<4>(k_cache, v_cache, p, s);
-  if (G % 2 == 0) return launch_decode_tc<2>(k_cache, v_cache, p, s);
-  return launch_decode_tc<1>(k_cache, v_cache, p, s);
+  if (d == 64) return launch_decode_tc_d<64>(k_cache, v_cache, p, s);
+  return launch_decode_tc_d<128>(k_cache, v_cache, p, s);
 }
 
 extern "C" int tessera_rmsnorm(const void* x, const void* w, void* y, int rows, int dim,

@@ -222,7 +222,7 @@ class DecodeWorkload:
 # (Hq=32, Hkv=8, d=128) serving 64 sequences with contexts up to 16384 tokens.
 DECODE = DecodeWorkload("decode_b64_hq32_hkv8_d128_bs16_len1to16384", B=64, Hq=32, Hkv=8,
                         d=128, bs=16, max_len=16384, seed=11)
-# The same serving batch at head dimension 64 (the CUDA-core decode kernel).
+# The same serving batch at head dimension 64.
 DECODE_D64 = DecodeWorkload("decode_b64_hq32_hkv8_d64_bs16_len1to16384", B=64, Hq=32, Hkv=8,
                             d=64, bs=16, max_len=16384, seed=11)
 
