@@ -258,6 +258,28 @@ def test_lse_may_be_omitted_and_results_repeat_bitwise():
     assert torch.equal(o1, o2) and torch.equal(o1, o3) and torch.equal(l1, l3)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,T,d", [(8, 32, 32, 2048, 128), (8, 16, 8, 8192, 128),
+                                          (8, 8, 4, 32768, 64)])
+def test_l2_grouped_unit_order_matches_per_batch_calls_bitwise(B, Hq, Hkv, T, d):
+    # K/V larger than L2, so the units walk groups of (batch, K/V head) slices;
+    # one batch alone fits and keeps the global order.  Units never share
+    # arithmetic, so the order must not change a bit.
+    dev = torch.device("cuda:0")
+    kv_bytes = 2 * B * Hkv * T * d * 2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    assert kv_bytes > l2 and kv_bytes // B <= l2
+    g = torch.Generator(device=dev)
+    g.manual_seed(31)
+    q, k, v = (torch.randn((B, h, T, d), generator=g, device=dev).to(torch.bfloat16)
+               for h in (Hq, Hkv, Hkv))
+    o, lse = tess.attn_fwd(q, k, v)
+    for b in range(B):
+        ob, lb = tess.attn_fwd(q[b:b + 1], k[b:b + 1], v[b:b + 1])
+        assert torch.equal(ob, o[b:b + 1]) and torch.equal(lb, lse[b:b + 1]), b
+    torch.cuda.synchronize()
+    assert tess.tessera_attn_device_error() == 0
+
+
 def test_empty_inputs_launch_nothing():
     dev = torch.device("cuda:0")
     q = torch.empty((0, 4, 16, 64), dtype=torch.bfloat16, device=dev)
