@@ -623,7 +623,8 @@ def noncausal_line(wn, times, max_ms, steps, launches, world, peaks, peak_src):
             "config": {"workload": wn.name, "B": wn.B, "T": wn.T, "Hq": wn.Hq, "Hkv": wn.Hkv,
                        "d": wn.d, "causal": False},
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": None,
+                         "unit": UNIT, "frac": round(achieved / peak, 4),
+                         "traffic": traffic_bytes("noncausal", wn.name),
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          **north_star_roofline(achieved, wn)},
             "gpu_launches": launches, "l2": "flushed before every timed step"}
@@ -688,7 +689,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--only", choices=["forward", "backward", "decode", "prologue", "varlen"],
+    ap.add_argument("--only", choices=["forward", "backward", "decode", "decode_d64", "noncausal",
+                                       "prologue", "varlen"],
                     help="time one extra leg alone and print its object (for profiling it)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -932,11 +934,17 @@ def one_leg(args, tess, torch, dev, world, rank, local):
         times, launches, ws = time_backward(w, q, k, v, g, args.steps, args.warmup, flush,
                                             stream, tess, torch)
         max_ms = max_over_ranks(sum(times), dev)
-    elif args.only == "decode":
-        wd = inputs.DECODE
+    elif args.only in ("decode", "decode_d64"):
+        wd = inputs.DECODE if args.only == "decode" else inputs.DECODE_D64
         times, launches, ws, flushed = time_decode(wd, args.steps, args.warmup, flush, stream,
-                                                   tess, torch,
-                                          dev)
+                                                   tess, torch, dev)
+        max_ms = max_over_ranks(sum(times), dev)
+    elif args.only == "noncausal":
+        wn = dataclasses.replace(w, causal=False, name=w.name + "_noncausal")
+        q, k, v = (t.to(dev) for t in inputs.make_qkv(w.B, w.Hq, w.Hkv, w.T, w.d,
+                                                     rank_seed(w.seed, rank), w.sigma_qk))
+        times, launches, _, _ = time_kernel(wn, q, k, v, args.steps, args.warmup, flush, stream,
+                                            tess, torch)
         max_ms = max_over_ranks(sum(times), dev)
     elif args.only == "varlen":
         times, launches = time_varlen(inputs.VARLEN, args.steps, args.warmup, flush, stream, tess,
@@ -969,9 +977,11 @@ def one_leg(args, tess, torch, dev, world, rank, local):
     elif args.only == "backward":
         line = backward_line(w, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
         line["config"] = {"workload": args.workload}
-    elif args.only == "decode":
+    elif args.only in ("decode", "decode_d64"):
         line = decode_line(wd, times, max_ms, args.steps, launches, ws, world, peaks, peak_src,
                            flushed)
+    elif args.only == "noncausal":
+        line = noncausal_line(wn, times, max_ms, args.steps, launches, world, peaks, peak_src)
     elif args.only == "varlen":
         line = varlen_line(inputs.VARLEN, times, launches, peaks, peak_src)
     else:
@@ -1018,7 +1028,7 @@ def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak
             "unit": "GB/s", "steps": steps, "ms_per_step": round(max_ms / steps, 5),
             "config": wd.describe(),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic_bytes("decode", wd.name),
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic_bytes("decode" if wd.d == 128 else "decode_d64", wd.name),
                          "peak_source": f"{peak_src} hbm_gbs",
                          "bytes_per_step": nbytes,
                          "byte_count": "K and V rows of every cached token, q, o, lse, "
@@ -1046,9 +1056,10 @@ def north_star_roofline(achieved: float, w) -> dict:
 # The kernel headers each leg is built from: a leg's DRAM-traffic record in
 # profiles/traffic.json stays valid while they are unchanged.
 _FWD_SOURCES = ["attn_fwd_sm100.cuh", "exp2_fma.cuh", "sm100_ptx.cuh"]
-LEG_SOURCES = {"forward": _FWD_SOURCES, "varlen": _FWD_SOURCES,
+LEG_SOURCES = {"forward": _FWD_SOURCES, "varlen": _FWD_SOURCES, "noncausal": _FWD_SOURCES,
                "backward": ["attn_bwd_sm100.cuh"] + _FWD_SOURCES,
                "decode": ["paged_decode_tc.cuh", "paged_decode.cuh"] + _FWD_SOURCES,
+               "decode_d64": ["paged_decode_tc.cuh", "paged_decode.cuh"] + _FWD_SOURCES,
                "rmsnorm": ["prologue.cuh"], "rope_qkv": ["prologue.cuh"]}
 
 
