@@ -626,7 +626,7 @@ def noncausal_line(wn, times, max_ms, steps, launches, world, peaks, peak_src):
                          "unit": UNIT, "frac": round(achieved / peak, 4),
                          "traffic": traffic_bytes("noncausal", wn.name),
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         **north_star_roofline(achieved, wn)},
+                         **nominal_roofline(achieved, wn)},
             "gpu_launches": launches, "l2": "flushed before every timed step"}
 
 
@@ -851,7 +851,7 @@ def main():
                 "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
                 "flops_per_launch": w.flops, "io_bytes_per_launch": w.io_bytes,
-                **north_star_roofline(achieved, w)}
+                **nominal_roofline(achieved, w)}
     if "bf16_tflops_sustained" in peaks:
         # long runs settle at the power cap: the sustained GEMM figure beside it
         roofline["frac_of_sustained"] = round(achieved / float(peaks["bf16_tflops_sustained"]), 4)
@@ -973,7 +973,7 @@ def one_leg(args, tess, torch, dev, world, rank, local):
                 "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                              "unit": UNIT, "frac": round(achieved / peak, 4), "traffic": traffic_bytes("forward", w.name),
                              "peak_source": f"{peak_src} bf16_tflops (burst)",
-                             **north_star_roofline(achieved, w)}}
+                             **nominal_roofline(achieved, w)}}
     elif args.only == "backward":
         line = backward_line(w, times, max_ms, args.steps, launches, ws, world, peaks, peak_src)
         line["config"] = {"workload": args.workload}
@@ -1042,15 +1042,15 @@ def decode_line(wd, times, max_ms, steps, launches, ws_bytes, world, peaks, peak
                                 "lines are written back during the step"}
 
 
-def north_star_roofline(achieved: float, w) -> dict:
+def nominal_roofline(achieved: float, w) -> dict:
     """The target's own roofline for a forward launch: the lesser of the
     nominal dense bf16 rate (2.25 PFLOP/s) and the I/O bytes (Q, K, V, O, LSE)
     over a nominal 8 TB/s, with the target of 60 % of it for the largest
     causal workload."""
     roof = min(NOMINAL_BF16_TFLOPS, w.flops / w.io_bytes * NOMINAL_HBM_GBS * 1e9 / 1e12)
     frac = achieved / roof
-    return {"north_star_peak": round(roof, 1), "frac_north_star": round(frac, 4),
-            "north_star_target_frac": 0.60, "north_star_target_met": bool(frac >= 0.60)}
+    return {"nominal_peak": round(roof, 1), "frac_nominal": round(frac, 4),
+            "target_frac_nominal": 0.60, "target_met": bool(frac >= 0.60)}
 
 
 # The kernel headers each leg is built from: a leg's DRAM-traffic record in
