@@ -80,3 +80,26 @@ def test_reference_arm_non_zero_ranks_exit_quietly():
                         "--gpus", "2", "--steps", "1", "--warmup", "3"],
                        capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_every_traffic_record_matches_the_current_kernel_sources():
+    # bench.py reports a leg's DRAM traffic only while the record's source sha
+    # matches the kernel headers it was captured from; a stale record would
+    # silently turn into a null.
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        records = json.load(f)["records"]
+    assert set(records) == set(bench.LEG_SOURCES)
+    for leg, rec in records.items():
+        assert rec["kernel_source_sha"] == bench.kernel_source_sha(leg), leg
+        assert rec["bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"], leg
+        assert bench.traffic_bytes(leg, rec["workload"]) == rec["bytes_per_launch"], leg
+
+
+def test_nominal_roofline_of_the_headline_workload():
+    from causal_gqa_attention_03_b200 import inputs
+    w = inputs.WORKLOADS[inputs.LARGEST]
+    r = bench.nominal_roofline(1350.0, w)
+    # tensor-bound: the I/O bytes over 8 TB/s allow far more than 2.25 PFLOP/s
+    assert r["nominal_peak"] == 2250.0
+    assert r["frac_nominal"] == 0.6 and r["target_met"]
+    assert not bench.nominal_roofline(1349.0, w)["target_met"]
